@@ -1,0 +1,142 @@
+"""CPU oracle of the routed MoE FFN forward pass (fp64, plain C + OpenMP).
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, the smoke check in
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import this
+package.  It shares no code with the CUDA path (``sparse_mixture_experts_19_b200``);
+both read their inputs from the seeded generator in ``moe_inputs``.
+
+What it computes, per token (see ``moe_oracle.c`` for the sources):
+score -> top-k (ties to the lower expert index) -> softmax over the k selected
+scores -> capacity drop in token order -> weighted sum of the selected SwiGLU
+experts (+ the always-on shared expert).
+
+Parity pins of every function here live in ``tests/test_oracle.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+
+DTYPE_CODE = {"f32": 0, "bf16": 1}
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into libmoe_oracle.so (gcc -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        _lib.oracle_route.argtypes = [i64, i32, i32, i32, i32, P, P, P, P, P, P]
+        _lib.oracle_permute.argtypes = [i64, i32, i32, i64, P, P, P, P, P, P]
+        _lib.oracle_moe_tokens.argtypes = [i64, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P,
+                                           P, P, P, i64, P, P]
+        for f in (_lib.oracle_route, _lib.oracle_permute, _lib.oracle_moe_tokens):
+            f.restype = ctypes.c_int
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _c(a, dt=None):
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=dt) if dt is not None else np.ascontiguousarray(a)
+
+
+def route(x, router_w, router_b, k: int, dtype: str):
+    """fp64 logits [T,E], topk_idx int32 [T,k], topk_w fp64 [T,k]."""
+    x, router_w = _c(x), _c(router_w)
+    router_b = _c(router_b, np.float32)
+    T, H = x.shape
+    E = router_w.shape[0]
+    logits = np.empty((T, E), np.float64)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    rc = _L().oracle_route(T, H, E, k, DTYPE_CODE[dtype], _ptr(x), _ptr(router_w), _ptr(router_b),
+                           _ptr(logits), _ptr(idx), _ptr(w))
+    if rc != 0:
+        raise ValueError(f"oracle_route failed ({rc})")
+    return logits, idx, w
+
+
+def permute(topk_idx, E: int, capacity: int = 0) -> dict:
+    """Grouping by expert with capacity drop in token order (all int32)."""
+    topk_idx = _c(topk_idx, np.int32)
+    T, k = topk_idx.shape
+    counts = np.empty(E, np.int32)
+    dropped = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    perm_rows = np.empty(T * k, np.int32)
+    row_of = np.empty(T * k, np.int32)
+    rc = _L().oracle_permute(T, k, E, int(capacity), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                             _ptr(perm_rows), _ptr(row_of), _ptr(dropped))
+    if rc != 0:
+        raise ValueError(f"oracle_permute failed ({rc})")
+    return dict(counts=counts, offsets=offsets, perm_rows=perm_rows, row_of=row_of.reshape(T, k),
+                dropped=dropped)
+
+
+def moe_tokens(x, w_gate, w_up, w_down, topk_idx, topk_w, dtype: str, row_of=None,
+               ws_gate=None, ws_up=None, ws_down=None, tokens=None) -> np.ndarray:
+    """fp64 output rows y[t] for the listed tokens (all tokens if None)."""
+    x, w_gate, w_up, w_down = _c(x), _c(w_gate), _c(w_up), _c(w_down)
+    ws_gate, ws_up, ws_down = _c(ws_gate), _c(ws_up), _c(ws_down)
+    topk_idx = _c(topk_idx, np.int32)
+    topk_w = _c(topk_w, np.float64)
+    row_of = _c(row_of, np.int32)
+    T, H = x.shape
+    E, I, _ = w_gate.shape
+    k = topk_idx.shape[1]
+    Is = 0 if ws_gate is None else ws_gate.shape[0]
+    tok = None if tokens is None else _c(tokens, np.int32)
+    n = T if tok is None else tok.shape[0]
+    y = np.empty((n, H), np.float64)
+    rc = _L().oracle_moe_tokens(T, H, I, E, k, Is, DTYPE_CODE[dtype], _ptr(x), _ptr(w_gate), _ptr(w_up),
+                                _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(topk_idx),
+                                _ptr(topk_w), _ptr(row_of), n, _ptr(tok), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle_moe_tokens failed ({rc})")
+    return y
+
+
+def topk_margin(logits: np.ndarray, k: int) -> np.ndarray:
+    """Gap between the k-th and (k+1)-th largest logit of each token (inf if k == E)."""
+    T, E = logits.shape
+    if k >= E:
+        return np.full(T, np.inf)
+    part = -np.sort(-logits, axis=1)
+    return part[:, k - 1] - part[:, k]
+
+
+def forward(wl, inp: dict, tokens=None) -> dict:
+    """The whole layer for workload ``wl`` (a ``moe_inputs.Workload``).
+
+    Routing and grouping run over all T tokens; the FFN output is evaluated
+    for ``tokens`` (all tokens if None).
+    """
+    logits, idx, w = route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+    perm = permute(idx, wl.E, wl.capacity())
+    y = moe_tokens(inp["x"], inp["w_gate"], inp["w_up"], inp["w_down"], idx, w, wl.dtype,
+                   row_of=perm["row_of"], ws_gate=inp["ws_gate"], ws_up=inp["ws_up"],
+                   ws_down=inp["ws_down"], tokens=tokens)
+    return dict(logits=logits, topk_idx=idx, topk_w=w, y=y, margin=topk_margin(logits, wl.k), **perm)

@@ -1,0 +1,324 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+Each test pins one step of the method to an independent fact:
+  * library routines: transformers' eager MoE modules (the gpt-oss top-k
+    router with bias and softmax over the selected logits; the Mixtral packed
+    experts), numpy / torch float64 matmuls;
+  * closed forms: the two-way softmax is the logistic function; k = 1 gives
+    weight 1; bias-only scores with hand-worked selections and weights;
+  * special cases: top_k = E is the dense softmax mixture; E = k = 1 is a
+    plain SwiGLU FFN;
+  * brute force over all k-subsets on tiny shapes;
+  * invariants: weights sum to 1, counts sum to T*k, capacity bookkeeping,
+    unselected experts do not matter, token-permutation invariance;
+  * hand-built golden fixtures under tests/golden/.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f64(a, dtype):
+    """Exact fp64 view of generator output (bf16 bits or float32)."""
+    return (mi.bf16_bits_to_f32(a) if dtype == "bf16" else a).astype(np.float64)
+
+
+def small(T=37, H=48, I=40, E=6, k=2, dtype="f32", **kw):
+    return mi.Workload("pin", T=T, H=H, I=I, E=E, k=k, dtype=dtype, **kw)
+
+
+# ---------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("E,k", [(8, 2), (32, 4), (16, 1)])
+def test_route_matches_transformers_topk_softmax_router(dtype, E, k):
+    """gpt-oss router in transformers: logits with bias, top-k, softmax over the k (fp64)."""
+    from transformers import GptOssConfig
+    from transformers.models.gpt_oss.modeling_gpt_oss import GptOssTopKRouter
+
+    wl = small(T=50, H=40, E=E, k=k, dtype=dtype, zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    cfg = GptOssConfig(hidden_size=wl.H, num_local_experts=E, num_experts_per_tok=k)
+    r = GptOssTopKRouter(cfg).double()
+    with torch.no_grad():
+        r.weight.copy_(torch.from_numpy(f64(inp["router_w"], dtype)))
+        r.bias.copy_(torch.from_numpy(inp["router_b"].astype(np.float64)))
+        logits_ref, w_ref, idx_ref = r(torch.from_numpy(f64(inp["x"], dtype)))
+    logits, idx, w = oracle.route(inp["x"], inp["router_w"], inp["router_b"], k, dtype)
+    np.testing.assert_allclose(logits, logits_ref.numpy(), rtol=0, atol=1e-12)
+    assert np.array_equal(idx, idx_ref.numpy())
+    np.testing.assert_allclose(w, w_ref.numpy(), rtol=0, atol=1e-14)
+
+
+def test_route_logits_equal_float64_matmul_plus_bias():
+    wl = small(T=64, H=96, E=16, k=3, dtype="bf16", zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    logits, _, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+    ref = f64(inp["x"], "bf16") @ f64(inp["router_w"], "bf16").T + inp["router_b"].astype(np.float64)
+    np.testing.assert_allclose(logits, ref, rtol=0, atol=1e-12)
+
+
+def test_route_brute_force_subsets():
+    """The selected set maximises the sum of scores over all k-subsets; equal sums
+    go to the lexicographically smallest sorted tuple (lower indices first)."""
+    rng_wl = small(T=40, H=8, E=7, k=3, dtype="f32")
+    inp = mi.make_inputs(rng_wl)
+    # force some exact ties: a bias with repeated values and a zero-input token
+    inp["x"][:5] = 0.0
+    inp["router_b"] = np.array([0.5, 1.0, 1.0, -2.0, 1.0, 0.5, 0.0], np.float32)
+    logits, idx, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], 3, "f32")
+    for t in range(rng_wl.T):
+        best, best_key = None, None
+        for sub in itertools.combinations(range(7), 3):
+            key = (-math.fsum(logits[t, list(sub)]), sub)
+            if best_key is None or key < best_key:
+                best, best_key = sub, key
+        # sum-maximal sets can differ only under ties; with ties the lower
+        # indices win elementwise, which is the lexicographic minimum here
+        assert tuple(sorted(idx[t])) == best, t
+    # ordering within a token: score descending, then index ascending
+    for t in range(rng_wl.T):
+        keys = [(-logits[t, e], e) for e in idx[t]]
+        assert keys == sorted(keys)
+
+
+def test_route_ties_golden():
+    g = json.load(open(os.path.join(GOLDEN, "route_ties.json")))
+    for case in g["cases"]:
+        b = np.array(case["bias"], np.float32)
+        E, k, H = len(b), case["k"], 4
+        x = np.zeros((3, H), np.float32)
+        rw = mi.normal(0, 99, (E, H), 1.0, "f32")
+        _, idx, w = oracle.route(x, rw, b, k, "f32")
+        for t in range(3):
+            assert idx[t].tolist() == case["topk_idx"]
+            if case["topk_w"] is not None:
+                np.testing.assert_allclose(w[t], case["topk_w"], rtol=0, atol=1e-7)
+
+
+def test_two_way_softmax_is_logistic_and_k1_weight_is_one():
+    wl = small(T=200, H=32, E=8, k=2)
+    inp = mi.make_inputs(wl)
+    logits, idx, w = oracle.route(inp["x"], inp["router_w"], None, 2, "f32")
+    d = logits[np.arange(wl.T), idx[:, 0]] - logits[np.arange(wl.T), idx[:, 1]]
+    np.testing.assert_allclose(w[:, 0], 1.0 / (1.0 + np.exp(-d)), rtol=0, atol=1e-15)
+    _, _, w1 = oracle.route(inp["x"], inp["router_w"], None, 1, "f32")
+    assert np.all(w1 == 1.0)
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (128, 8), (256, 8)])
+def test_weights_sum_to_one_and_follow_scores(E, k):
+    wl = small(T=300, H=64, E=E, k=k, dtype="bf16", zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    logits, idx, w = oracle.route(inp["x"], inp["router_w"], inp["router_b"], k, "bf16")
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=0, atol=1e-15)
+    assert np.all(w > 0)
+    assert np.all(np.diff(w, axis=1) <= 0)
+    # softmax over all E, take top-k, renormalise == top-k then softmax over the k
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    pk = np.take_along_axis(p, idx, 1)
+    np.testing.assert_allclose(pk / pk.sum(1, keepdims=True), w, rtol=0, atol=1e-15)
+    # the selected probabilities are the k largest of the full softmax
+    assert np.all(pk.min(1) >= np.sort(p, 1)[:, -k] - 1e-15)
+
+
+# ---------------------------------------------------------------- grouping
+
+@pytest.mark.parametrize("name", ["capacity_toy.json", "capacity_toy_k2.json"])
+def test_permute_golden(name):
+    g = json.load(open(os.path.join(GOLDEN, name)))
+    r = oracle.permute(np.array(g["topk_idx"], np.int32), g["E"], g["capacity"])
+    for key in ("counts", "dropped", "offsets", "perm_rows", "row_of"):
+        assert r[key].tolist() == g[key], key
+
+
+@pytest.mark.parametrize("cf", [0.0, 1.0, 1.25, 2.0])
+def test_permute_invariants(cf):
+    wl = small(T=3000, H=16, E=128, k=8, dtype="f32", zipf_s=1.1, capacity_factor=cf)
+    inp = mi.make_inputs(wl)
+    _, idx, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, "f32")
+    C = wl.capacity()
+    r = oracle.permute(idx, wl.E, C)
+    counts, dropped, off = r["counts"], r["dropped"], r["offsets"]
+    assert counts.sum() == wl.T * wl.k
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=wl.E))
+    kept = np.minimum(counts, C) if C > 0 else counts
+    assert np.array_equal(np.diff(off), kept)
+    assert np.array_equal(dropped, counts - kept)
+    assert kept.sum() + dropped.sum() == wl.T * wl.k
+    R = off[-1]
+    pr, ro = r["perm_rows"], r["row_of"].ravel()
+    assert np.all(pr[R:] == -1) and np.all(pr[:R] >= 0)
+    assert np.array_equal(ro[pr[:R]], np.arange(R))          # bijection rows <-> kept slots
+    assert (ro >= 0).sum() == R
+    for e in range(wl.E):
+        rows = pr[off[e]:off[e + 1]]
+        assert np.all(idx.ravel()[rows] == e)
+        tok = rows // wl.k
+        assert np.all(np.diff(tok) > 0)                      # ascending token order
+        if C > 0 and counts[e] > C:                          # the earliest C tokens are kept
+            all_tok = np.nonzero((idx == e).any(1))[0]
+            assert np.array_equal(tok, all_tok[:C])
+
+
+# ---------------------------------------------------------------- experts
+
+def _mixtral_experts(inp, dtype, E, H, I):
+    from transformers import MixtralConfig
+    from transformers.models.mixtral.modeling_mixtral import MixtralExperts
+
+    cfg = MixtralConfig(hidden_size=H, intermediate_size=I, num_local_experts=E, hidden_act="silu")
+    m = MixtralExperts(cfg).double()
+    with torch.no_grad():
+        gu = np.concatenate([f64(inp["w_gate"], dtype), f64(inp["w_up"], dtype)], axis=1)
+        m.gate_up_proj.copy_(torch.from_numpy(gu))
+        m.down_proj.copy_(torch.from_numpy(f64(inp["w_down"], dtype)))
+    return m
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_experts_match_transformers_mixtral_experts(dtype):
+    """Weighted sum of the selected SwiGLU experts == transformers' eager packed experts."""
+    wl = small(T=45, H=40, I=24, E=6, k=2, dtype=dtype)
+    inp = mi.make_inputs(wl)
+    _, idx, w = oracle.route(inp["x"], inp["router_w"], None, wl.k, dtype)
+    y = oracle.moe_tokens(inp["x"], inp["w_gate"], inp["w_up"], inp["w_down"], idx, w, dtype)
+    m = _mixtral_experts(inp, dtype, wl.E, wl.H, wl.I)
+    with torch.no_grad():
+        ref = m(torch.from_numpy(f64(inp["x"], dtype)), torch.from_numpy(idx.astype(np.int64)),
+                torch.from_numpy(w)).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_full_layer_matches_transformers_mixtral_block():
+    """Mixtral's block: softmax over all E (float32), top-k, renormalise."""
+    from transformers import MixtralConfig
+    from transformers.models.mixtral.modeling_mixtral import MixtralSparseMoeBlock
+
+    wl = small(T=64, H=32, I=48, E=8, k=2, dtype="f32")
+    inp = mi.make_inputs(wl)
+    cfg = MixtralConfig(hidden_size=wl.H, intermediate_size=wl.I, num_local_experts=wl.E,
+                        num_experts_per_tok=wl.k, hidden_act="silu")
+    blk = MixtralSparseMoeBlock(cfg).double().eval()
+    with torch.no_grad():
+        blk.gate.weight.copy_(torch.from_numpy(f64(inp["router_w"], "f32")))
+        gu = np.concatenate([f64(inp["w_gate"], "f32"), f64(inp["w_up"], "f32")], axis=1)
+        blk.experts.gate_up_proj.copy_(torch.from_numpy(gu))
+        blk.experts.down_proj.copy_(torch.from_numpy(f64(inp["w_down"], "f32")))
+        ref = blk(torch.from_numpy(f64(inp["x"], "f32"))[None])[0].numpy()
+    out = oracle.forward(wl, inp)
+    assert np.all(out["margin"] > 1e-5)
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-5, atol=1e-6)
+
+
+def test_single_expert_is_dense_swiglu_ffn():
+    """E = k = 1: weight exactly 1 and y = W_d (silu(W_g x) * W_u x) via torch float64."""
+    wl = small(T=20, H=24, I=56, E=1, k=1, dtype="bf16")
+    inp = mi.make_inputs(wl)
+    out = oracle.forward(wl, inp)
+    assert np.all(out["topk_w"] == 1.0) and np.all(out["topk_idx"] == 0)
+    x = torch.from_numpy(f64(inp["x"], "bf16"))
+    g = torch.from_numpy(f64(inp["w_gate"], "bf16")[0])
+    u = torch.from_numpy(f64(inp["w_up"], "bf16")[0])
+    d = torch.from_numpy(f64(inp["w_down"], "bf16")[0])
+    ref = torch.nn.functional.linear(torch.nn.functional.silu(x @ g.T) * (x @ u.T), d).numpy()
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_swiglu_closed_form_scalar():
+    """H = I = 1, unit weights: y = silu(x) * x = x^2 / (1 + e^-x)."""
+    x = np.array([[2.0], [-3.0], [0.0], [0.5]], np.float32)
+    one = np.ones((1, 1, 1), np.float32)
+    y = oracle.moe_tokens(x, one, one, one, np.zeros((4, 1), np.int32), np.ones((4, 1)), "f32")
+    for t, v in enumerate([2.0, -3.0, 0.0, 0.5]):
+        assert y[t, 0] == pytest.approx(v * v / (1.0 + math.exp(-v)), rel=1e-15, abs=1e-300)
+
+
+def test_shared_expert_is_added_with_weight_one():
+    wl = small(T=30, H=40, I=24, E=6, k=2, dtype="bf16", I_shared=32)
+    inp = mi.make_inputs(wl)
+    out = oracle.forward(wl, inp)
+    routed = oracle.moe_tokens(inp["x"], inp["w_gate"], inp["w_up"], inp["w_down"], out["topk_idx"],
+                               out["topk_w"], "bf16")
+    sh = {"w_gate": inp["ws_gate"][None], "w_up": inp["ws_up"][None], "w_down": inp["ws_down"][None]}
+    m = _mixtral_experts(sh, "bf16", 1, wl.H, wl.I_shared)
+    with torch.no_grad():
+        ref = m(torch.from_numpy(f64(inp["x"], "bf16")), torch.zeros((wl.T, 1), dtype=torch.int64),
+                torch.ones((wl.T, 1), dtype=torch.float64)).numpy()
+    np.testing.assert_allclose(out["y"] - routed, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_top_k_equal_E_is_dense_softmax_mixture():
+    """With k = E every expert is chosen: y = sum_e softmax(l)_e FFN_e(x)."""
+    wl = small(T=25, H=32, I=20, E=5, k=5, dtype="f32")
+    inp = mi.make_inputs(wl)
+    out = oracle.forward(wl, inp)
+    l = f64(inp["x"], "f32") @ f64(inp["router_w"], "f32").T
+    p = torch.softmax(torch.from_numpy(l), dim=1)
+    m = _mixtral_experts(inp, "f32", wl.E, wl.H, wl.I)
+    dense = np.zeros((wl.T, wl.H))
+    x = torch.from_numpy(f64(inp["x"], "f32"))
+    with torch.no_grad():
+        for e in range(wl.E):   # every expert on every token, mixed by the full softmax
+            ye = m(x, torch.full((wl.T, 1), e, dtype=torch.int64), torch.ones((wl.T, 1), dtype=torch.float64))
+            dense += p[:, e:e + 1].numpy() * ye.numpy()
+    np.testing.assert_allclose(out["y"], dense, rtol=1e-12, atol=1e-13)
+
+
+def test_unselected_experts_do_not_change_output():
+    wl = small(T=6, H=32, I=16, E=16, k=2, dtype="bf16")
+    inp = mi.make_inputs(wl)
+    out = oracle.forward(wl, inp)
+    unused = sorted(set(range(wl.E)) - set(out["topk_idx"].ravel().tolist()))
+    assert unused
+    inp2 = dict(inp)
+    for key in ("w_gate", "w_up", "w_down"):
+        inp2[key] = inp[key].copy()
+        inp2[key][unused] = mi.normal(7, 77, inp[key][unused].shape, 3.0, "bf16")
+    out2 = oracle.forward(wl, inp2)
+    assert np.array_equal(out["y"], out2["y"])
+
+
+def test_token_permutation_invariance():
+    wl = small(T=40, H=32, I=16, E=8, k=3, dtype="bf16", I_shared=8)
+    inp = mi.make_inputs(wl)
+    out = oracle.forward(wl, inp)
+    pi = mi.permutation(3, 1, wl.T)
+    inp2 = dict(inp, x=inp["x"][pi])
+    out2 = oracle.forward(wl, inp2)
+    assert np.array_equal(out2["y"], out["y"][pi])
+    assert np.array_equal(out2["topk_idx"], out["topk_idx"][pi])
+
+
+def test_dropped_pairs_contribute_nothing():
+    wl = small(T=400, H=32, I=16, E=8, k=2, dtype="f32", capacity_factor=0.5)
+    inp = mi.make_inputs(wl)
+    out = oracle.forward(wl, inp)
+    ro = out["row_of"]
+    assert (ro < 0).any()
+    w_kept = np.where(ro >= 0, out["topk_w"], 0.0)
+    y_ref = oracle.moe_tokens(inp["x"], inp["w_gate"], inp["w_up"], inp["w_down"], out["topk_idx"],
+                              w_kept, "f32")
+    np.testing.assert_allclose(out["y"], y_ref, rtol=1e-13, atol=1e-14)
+    all_dropped = np.all(ro < 0, axis=1)
+    assert np.all(out["y"][all_dropped] == 0.0)
+
+
+def test_sampled_tokens_equal_full_evaluation():
+    wl = small(T=50, H=32, I=16, E=8, k=2, dtype="bf16")
+    inp = mi.make_inputs(wl)
+    full = oracle.forward(wl, inp)
+    tok = mi.sample_tokens(5, wl.T, 9)
+    part = oracle.forward(wl, inp, tokens=tok)
+    assert np.array_equal(part["y"], full["y"][tok])
