@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Throughput of the routed MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--T TOKENS]
+
+One step = one ``moe_forward`` call (router GEMM + top-k/softmax, grouping,
+grouped gate/up GEMM with fused SwiGLU, grouped down GEMM with fused
+weighted scatter-add, final cast) over one batch of T synthetic tokens of the
+workload (default: the Mixtral-8x7B-shaped layer, T = 4096).  Inputs are
+seeded (``moe_inputs``) and resident in HBM when the timed region starts.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch of
+T tokens with its own copy of the weights (weak scaling: tokens are
+independent, there is no data-path collective); the time is the max over
+ranks and ``value`` counts the tokens of all ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+method has) on the host cores on a bounded token sample per step; under
+torchrun only rank 0 runs it.
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at 1 B200 and % of roofline (tensor peak or HBM GB/s)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GATEUP_KERNELS = ("gateup_sm100", "gateup_simt")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_8x7b_layer")
+    ap.add_argument("--T", type=int, default=0, help="override the token count")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload(args):
+    import moe_inputs as mi
+
+    if args.workload not in mi.FULL:
+        raise SystemExit(f"unknown workload {args.workload}; one of {sorted(mi.FULL)}")
+    wl = mi.FULL[args.workload]
+    return wl.with_(T=args.T) if args.T else wl
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_of(wl):
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
+            "I_shared": wl.I_shared, "capacity_factor": wl.capacity_factor, "zipf_s": wl.zipf_s,
+            "seed": wl.seed}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                f = [c.strip() for c in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# --------------------------------------------------------------- roofline
+def layer_bytes(wl, active_experts: int) -> float:
+    """Algorithmic bytes: weights of the activated experts + x + y + router (+ shared)."""
+    elt = 2 if wl.dtype == "bf16" else 4
+    b = active_experts * 3 * wl.H * wl.I * elt
+    b += 2 * wl.T * wl.H * elt + wl.E * wl.H * elt
+    b += 3 * wl.H * wl.I_shared * elt
+    return float(b)
+
+
+def traffic_for(kernel: str, wl):
+    """DRAM bytes per launch from the committed ncu summary, if it is for this
+    kernel, this workload and the kernel's current source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(kernel)
+    if not d or d.get("workload") != wl.name or d.get("T") != wl.T:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
+        return None
+    return float(d["dram_bytes_per_launch"])
+
+
+# ----------------------------------------------------------------- oracle
+def oracle_tokens_per_s(wl, inp, target_s: float, seed: int = 3):
+    """The fp64 CPU oracle on a bounded token sample: (tokens/s, n, seconds, threads)."""
+    import moe_inputs as mi
+    import oracle
+
+    def run(n):
+        tok = mi.sample_tokens(seed, wl.T, n)
+        xs = inp["x"][tok]
+        t0 = time.perf_counter()
+        _, idx, w = oracle.route(xs, inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+        oracle.moe_tokens(xs, inp["w_gate"], inp["w_up"], inp["w_down"], idx, w, wl.dtype,
+                          ws_gate=inp["ws_gate"], ws_up=inp["ws_up"], ws_down=inp["ws_down"])
+        return time.perf_counter() - t0
+
+    t1 = run(2) / 2
+    n = int(max(2, min(wl.T, target_s / max(t1, 1e-6))))
+    dt = run(n)
+    return n / dt, n, dt, oracle.threads()
+
+
+# -------------------------------------------------------------- the arms
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    # the reference arm runs on rank 0's host cores alone: no process group
+    if world > 1 and args.impl == "ours" and not dist.is_initialized():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    return world, rank, local
+
+
+def run_reference(args, wl, world, rank):
+    """The CPU oracle as the reference arm: rank 0 only."""
+    if rank != 0:
+        return None
+    import moe_inputs as mi
+
+    inp = mi.make_inputs(wl)
+    per_step = min(10.0, 150.0 / max(1, args.steps + args.warmup))
+    import oracle
+
+    oracle.build()
+    # calibrate the sample once, then time W + K steps of that sample
+    _, n, _, _ = oracle_tokens_per_s(wl, inp, per_step)
+    times = []
+    for s in range(args.warmup + args.steps):
+        tok = mi.sample_tokens(100 + s, wl.T, n)
+        xs = inp["x"][tok]
+        t0 = time.perf_counter()
+        _, idx, w = oracle.route(xs, inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+        oracle.moe_tokens(xs, inp["w_gate"], inp["w_up"], inp["w_down"], idx, w, wl.dtype,
+                          ws_gate=inp["ws_gate"], ws_up=inp["ws_up"], ws_down=inp["ws_down"])
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = n * len(times) / total
+    sample = f"{n} seeded tokens per step (routing + expert FFN, fp64), steps {args.steps}"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def run_ours(args, wl, world, rank, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import moe_inputs as mi
+    import sparse_mixture_experts_19_b200 as moe
+    from sparse_mixture_experts_19_b200 import build as moe_build
+
+    moe_build.build()
+    moe.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = mi.make_inputs(wl)
+
+    def to_dev(a):
+        if a is None:
+            return None
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    d = {k: to_dev(v) for k, v in inp.items()}
+    cfg = moe.config(wl.T, wl.H, wl.I, wl.E, wl.k, wl.I_shared, wl.capacity_factor, wl.dtype)
+    ws = moe.workspace(cfg, dev)
+    y = torch.empty((wl.T, wl.H), dtype=d["x"].dtype, device=dev)
+    counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x_in):
+        moe.moe_forward(cfg, x_in, d["router_w"], d["router_b"], d["w_gate"], d["w_up"], d["w_down"],
+                        d["ws_gate"], d["ws_up"], d["ws_down"], y, None, counts, None, ws, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(d["x"])
+    torch.cuda.synchronize(dev)
+    if moe.moe_get_device_status(cfg, ws) != 0:
+        raise SystemExit("device check flags set during warm-up")
+    active = int((counts > 0).sum().item())
+
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        gpu_uuid = None
+
+    # ---- timed region: device time of K steps, kernels traced live
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_uuid) as clocks:
+        moe.moe_trace_begin(64 * args.steps)
+        start.record(stream)
+        for _ in range(args.steps):
+            step(d["x"])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        trace = moe.moe_trace_end(64 * args.steps)
+    barrier()
+    ms = max_over_ranks(start.elapsed_time(stop))
+    clk = clocks.summary()
+
+    # ---- end to end: pinned host x -> device, forward, y -> pinned host
+    x_host = d["x"].cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+
+    tokens = wl.T * args.steps * world
+    value = tokens / (ms / 1e3)
+    pk, pk_kind = peaks()
+
+    # ---- roofline of the dominant kernel (grouped gate/up GEMM + SwiGLU)
+    per_kernel = {}
+    for name, t in trace:
+        per_kernel.setdefault(name, []).append(t)
+    dom = next((k for k in GATEUP_KERNELS if k in per_kernel), None)
+    roof = None
+    if dom:
+        t_avg = sum(per_kernel[dom]) / len(per_kernel[dom]) / 1e3
+        kept = wl.T * wl.k
+        if wl.capacity_factor > 0:
+            kept = int(np.minimum(counts.cpu().numpy(), wl.capacity()).sum())
+        flops = 2.0 * kept * 2 * wl.H * wl.I + 2.0 * wl.T * 2 * wl.H * wl.I_shared
+        achieved = flops / t_avg / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic_for(dom, wl),
+                "peak_kind": f"{pk_kind} bf16 dense, sustained", "launch_ms": t_avg * 1e3,
+                "flops_per_launch": flops}
+    F = wl.flops()
+    B = layer_bytes(wl, active)
+    t_roof = max(F / (pk["bf16_tflops_sustained"] * 1e12), B / (pk["hbm_gbs"] * 1e9))
+    t_step = ms / args.steps / 1e3
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": dict(config_of(wl), l2="inputs larger than L2: %.1f GB of expert weights read per step"
+                       % (active * 3 * wl.H * wl.I * 2 / 1e9), parallelism=f"replicas{world}"),
+        "roofline": roof,
+        "layer_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / t_step, "flops": F, "bytes": B,
+                           "bound": "tensor" if F / (pk["bf16_tflops_sustained"] * 1e12) >= B / (pk["hbm_gbs"] * 1e9) else "hbm",
+                           "peak_kind": pk_kind},
+        "kernels_ms_per_step": {k: sum(v) / args.steps for k, v in per_kernel.items()},
+        "gpu_launches": len(trace),
+        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, dt, threads = oracle_tokens_per_s(wl, inp, 12.0)
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                               "sample": f"{n} seeded tokens of the workload (routing + expert FFN, fp64), {dt:.1f} s"}
+    return out
+
+
+def main():
+    args = parse_args()
+    wl = workload(args)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        out = run_reference(args, wl, world, rank)
+    else:
+        out = run_ours(args, wl, world, rank, local)
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+    try:
+        import torch.distributed as dist
+
+        if dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,211 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed Mixture-of-Experts FFN layer.
+ *
+ * The layer computes, for every token t of x [T, H]:
+ *
+ *   l[t, e]  = x[t] . router_w[e] + router_b[e]                 (router scores)
+ *   S_t      = the top_k experts by score (ties: lower index)     (selection)
+ *   w[t, j]  = softmax over the top_k selected scores            (gating)
+ *   y[t]     = sum_{j kept} w[t,j] * FFN_{S_t[j]}(x[t])  (+ shared FFN(x[t]))
+ *   FFN_e(v) = W_down[e] (silu(W_gate[e] v) * (W_up[e] v))         (SwiGLU)
+ *
+ * Sources (page title, section):
+ *   "MoE稀疏架构是什么？从原理到落地的系统解读", section 四 (one forward pass:
+ *     router scores, top-k, softmax over the chosen scores, weighted sum of
+ *     the chosen experts; unchosen experts are not evaluated); section 三.1
+ *     (the router is a small linear layer); section 三.2 (capacity-limited
+ *     token dropping).
+ *   "Mixture of Experts (MoEs) in Transformers", section Weight Loading
+ *     Refactor (all experts packed in one [E, out, in] tensor; gate = w1,
+ *     up = w3, down = w2), section Expert Backend (grouped_mm: tokens sorted
+ *     and grouped by expert id, then one grouped GEMM).
+ *   "模型的“分工的艺术”：MoE技术如何提升计算效率", section 3.1 (expert capacity).
+ *
+ * Readings where the pages are silent: ties go to the lower expert index;
+ * the expert FFN is SwiGLU without biases; capacity C = ceil(cf * T * k / E)
+ * with tokens served in ascending token order, a dropped (token, expert)
+ * pair contributes nothing and the token's other weights are not
+ * renormalised; a shared expert (I_shared > 0) is always applied with
+ * weight 1.
+ *
+ * Conventions for every entry point below
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major
+ *     and contiguous, 16-byte aligned.  The library never allocates, frees
+ *     or synchronises inside a compute call and keeps no pointer after the
+ *     call returns.  Work is enqueued on `stream` in stream order.
+ *   - dtype MOE_BF16: x, router_w, expert weights and y are bfloat16;
+ *     MOE_F32: all of them float32.  router_b, topk_w are always float32.
+ *   - Layouts: x, y [T, H]; router_w [E, H]; router_b [E];
+ *     w_gate, w_up [E, I, H]; w_down [E, H, I];
+ *     ws_gate, ws_up [I_shared, H]; ws_down [H, I_shared];
+ *     topk_idx int32 [T, top_k]; topk_w float32 [T, top_k].
+ *   - Slot id s = t * top_k + j names the j-th choice of token t.
+ *   - `ws` is scratch device memory of at least moe_workspace_size(cfg)
+ *     bytes, 256-byte aligned; its contents are undefined between calls,
+ *     except that device-side check flags persist until
+ *     moe_get_device_status() reads and clears them.  A new workspace must
+ *     start zeroed (or be cleared by one moe_get_device_status() call) for
+ *     those flags to mean anything.  Calls that share one workspace must be
+ *     ordered on the GPU (the same stream, or joined).
+ *   - Errors in arguments, shapes or alignment return synchronously, before
+ *     anything is enqueued.  A failed launch returns MOE_ERR_CUDA.
+ *     Data-dependent faults found on the device (an expert index out of
+ *     range fed to moe_permute) set a flag in `ws` and the offending entry
+ *     is skipped; moe_get_device_status() reports them.  No kernel traps.
+ *   - moe_last_error() gives a one-line reason for the last failure of the
+ *     calling thread.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid but outside this build's limits       */
+    MOE_ERR_WORKSPACE = 3,    /* ws too small or misaligned                  */
+    MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed        */
+    MOE_ERR_DEVICE_CHECK = 5  /* a device-side check fired (see status)      */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+typedef struct {
+    int32_t T;               /* tokens, >= 0 (0 is a valid no-op)             */
+    int32_t H;               /* hidden size, multiple of 8                     */
+    int32_t I;               /* expert intermediate size, multiple of 8        */
+    int32_t E;               /* routed experts, 1..256                         */
+    int32_t top_k;           /* 1..min(E, 8), or top_k == E when E <= 32       */
+    int32_t I_shared;        /* shared expert intermediate size, 0 = none      */
+    float capacity_factor;   /* <= 0: unlimited; else C = ceil(cf*T*top_k/E)   */
+    int32_t dtype;           /* moe_dtype_t                                    */
+} moe_config_t;
+
+/* Device-side check flags reported by moe_get_device_status(). */
+#define MOE_DEVFLAG_BAD_EXPERT_INDEX 0x1 /* moe_permute saw idx < 0 or >= E    */
+#define MOE_DEVFLAG_WAIT_TIMEOUT 0x2     /* a bounded device wait gave up      */
+
+/* Bytes of workspace every entry point below needs for `cfg`; 0 if the
+ * configuration is invalid (moe_last_error() says why). */
+size_t moe_workspace_size(const moe_config_t* cfg);
+
+/* Per-expert capacity C for cfg (0 = unlimited). */
+int64_t moe_capacity(const moe_config_t* cfg);
+
+/*
+ * moe_route -- router scores, top-k selection and softmax over the
+ * selected scores ("MoE稀疏架构是什么？从原理到落地的系统解读", sections 三.1
+ * and 四).  Scores are accumulated in float32 and never rounded to bf16.
+ *   x [T,H], router_w [E,H], router_b [E] float32 or NULL
+ *   -> topk_idx [T,top_k] int32: chosen experts, score descending, ties to
+ *      the lower index; topk_w [T,top_k] float32: softmax of those scores.
+ */
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* router_w,
+                       const float* router_b, int32_t* topk_idx, float* topk_w, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_permute -- group (token, slot) pairs by expert, with capacity drop in
+ * token order ("Mixture of Experts (MoEs) in Transformers", section Expert
+ * Backend: grouped_mm sorts tokens by expert id; "MoE稀疏架构是什么？…",
+ * section 三.2: capacity-limited dropping).
+ *   topk_idx [T,top_k] int32 ->
+ *   counts [E]      pairs per expert before the capacity cut
+ *   dropped [E]     pairs per expert beyond the capacity
+ *   offsets [E+1]   first kept row of each expert; offsets[E] = kept rows R
+ *   perm_rows [T*top_k]  slot id of each row; an expert's rows in ascending
+ *                   token order; entries >= R are set to -1
+ *   row_of [T*top_k]     row of each slot, -1 if dropped
+ * Every output is a pure function of topk_idx (bit-reproducible).
+ * An index outside [0, E) sets MOE_DEVFLAG_BAD_EXPERT_INDEX and the slot is
+ * treated as dropped without being counted.
+ */
+moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
+                         int32_t* offsets, int32_t* perm_rows, int32_t* row_of, int32_t* dropped,
+                         void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_grouped_ffn -- every kept row through its expert's SwiGLU FFN, as
+ * grouped GEMMs over the rows of each expert ("Mixture of Experts (MoEs) in
+ * Transformers", section Expert Backend, grouped_mm).
+ *   x [T,H]; perm_rows, offsets as produced by moe_permute;
+ *   w_gate, w_up [E,I,H]; w_down [E,H,I]; shared weights or NULLs;
+ *   -> expert_out float32 [T*top_k + (I_shared ? T : 0), H]:
+ *      row r < offsets[E] holds FFN_e(x[perm_rows[r] / top_k]) (unweighted);
+ *      row T*top_k + t holds the shared expert's FFN(x[t]).
+ *      Rows in [offsets[E], T*top_k) are left untouched.
+ * Intermediate activations are rounded to the layer dtype (bf16 for
+ * MOE_BF16) between the two GEMMs; accumulation is float32.
+ */
+moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const int32_t* perm_rows,
+                             const int32_t* offsets, const void* w_gate, const void* w_up,
+                             const void* w_down, const void* ws_gate, const void* ws_up,
+                             const void* ws_down, float* expert_out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/*
+ * moe_combine -- weighted un-permute ("MoE稀疏架构是什么？…", section 四:
+ * the output is the weight-scaled sum of the chosen experts' outputs).
+ *   y[t] = sum_{j : row_of[t,j] >= 0} topk_w[t,j] * expert_out[row_of[t,j]]
+ *          + (I_shared ? expert_out[T*top_k + t] : 0),  summed in float32
+ *   in order j = 0..top_k-1 then the shared row, rounded once to the dtype.
+ */
+moe_status_t moe_combine(const moe_config_t* cfg, const float* expert_out, const int32_t* row_of,
+                         const float* topk_w, void* y, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/*
+ * moe_forward -- the whole layer, the C form of the pages' moe_forward(x,
+ * experts, router, top_k) ("MoE稀疏架构是什么？…", section 四): route,
+ * group, grouped gate/up GEMM with the SwiGLU fused in its epilogue, grouped
+ * down GEMM with the routing-weight scale and the scatter-add fused in its
+ * epilogue, then one cast to the layer dtype.
+ *   y [T,H] (layer dtype).  Optional outputs (NULL to skip): topk_idx_out
+ *   [T,top_k] int32, counts_out [E] and dropped_out [E] int32.
+ * The summation order of the up to top_k + 1 terms of a y element is not
+ * fixed (float32 atomics), so y may differ between runs in the last bits.
+ */
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* router_w,
+                         const float* router_b, const void* w_gate, const void* w_up,
+                         const void* w_down, const void* ws_gate, const void* ws_up,
+                         const void* ws_down, void* y, int32_t* topk_idx_out, int32_t* counts_out,
+                         int32_t* dropped_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Waits for `stream`, then returns the device check flags (MOE_DEVFLAG_*)
+ * accumulated in `ws` since the last call and clears them.  Returns
+ * MOE_ERR_DEVICE_CHECK if any flag was set, MOE_OK otherwise. */
+moe_status_t moe_get_device_status(const moe_config_t* cfg, void* ws, size_t ws_bytes,
+                                   moe_stream_t stream, int32_t* flags_out);
+
+/* Static strings; never NULL. */
+const char* moe_status_string(moe_status_t status);
+const char* moe_last_error(void);
+
+/*
+ * Kernel tracing (for measurement).  While tracing is on, every kernel the
+ * library enqueues is bracketed by two CUDA events on its stream; up to
+ * `max_launches` launches are recorded.  moe_trace_end() waits for the
+ * recorded events, writes for each launch its kernel name and its duration
+ * in milliseconds, and turns tracing off.  Host-side only; no device
+ * memory is allocated.  Not thread-safe: one tracing session at a time.
+ */
+typedef struct {
+    const char* name; /* static string */
+    float ms;
+} moe_trace_record_t;
+
+moe_status_t moe_trace_begin(int32_t max_launches);
+moe_status_t moe_trace_end(moe_trace_record_t* records, int32_t max_records, int32_t* n_records);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -50,7 +50,14 @@ def _L():
                                            P, P, P, i64, P, P]
         for f in (_lib.oracle_route, _lib.oracle_permute, _lib.oracle_moe_tokens):
             f.restype = ctypes.c_int
+        _lib.oracle_threads.argtypes = []
+        _lib.oracle_threads.restype = ctypes.c_int
     return _lib
+
+
+def threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(_L().oracle_threads())
 
 
 def _ptr(a):
@@ -140,3 +147,20 @@ def forward(wl, inp: dict, tokens=None) -> dict:
                    row_of=perm["row_of"], ws_gate=inp["ws_gate"], ws_up=inp["ws_up"],
                    ws_down=inp["ws_down"], tokens=tokens)
     return dict(logits=logits, topk_idx=idx, topk_w=w, y=y, margin=topk_margin(logits, wl.k), **perm)
+
+
+def weights_for(logits: np.ndarray, sel: np.ndarray) -> np.ndarray:
+    """Softmax over the given selection's scores (fp64), the gating step of the
+    method for a selection made elsewhere (a near-tie resolved differently)."""
+    l = np.take_along_axis(np.asarray(logits, np.float64), np.asarray(sel, np.int64), 1)
+    e = np.exp(l - l.max(1, keepdims=True))
+    return e / e.sum(1, keepdims=True)
+
+
+def expert_rows(x, w_gate, w_up, w_down, tokens, experts, dtype: str) -> np.ndarray:
+    """FFN_e(x[t]) (unweighted, fp64) for each (token, expert) pair.  For the
+    shared expert pass its weights as [1, Is, H] / [1, H, Is] and expert 0."""
+    tokens = np.asarray(tokens, np.int64)
+    xs = np.ascontiguousarray(np.asarray(x)[tokens])
+    e = np.asarray(experts, np.int32).reshape(-1, 1)
+    return moe_tokens(xs, w_gate, w_up, w_down, e, np.ones(e.shape), dtype)

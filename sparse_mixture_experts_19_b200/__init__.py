@@ -1,0 +1,221 @@
+"""Routed MoE FFN layer for B200 (sm_100a): Python binding of ``libmoe.so``.
+
+Every entry point of the C ABI (``include/moe.h``) has a function of the
+same name here.  This module only marshals arguments (torch tensors ->
+device pointers, the current CUDA stream); every step of the layer runs in
+the library's CUDA kernels.  There is no CPU fallback: if the library is
+missing or cannot load, calls raise ``MoeError``.
+
+``forward(...)`` is the convenience form of ``moe_forward`` that allocates
+the output and the workspace with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK"}
+DEVFLAG_BAD_EXPERT_INDEX = 0x1
+DEVFLAG_WAIT_TIMEOUT = 0x2
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class moe_config_t(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("top_k", ctypes.c_int32), ("I_shared", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+class moe_trace_record_t(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("ms", ctypes.c_float)]
+
+
+_P = ctypes.c_void_p
+_SIGS = {
+    "moe_workspace_size": ([ctypes.POINTER(moe_config_t)], ctypes.c_size_t),
+    "moe_capacity": ([ctypes.POINTER(moe_config_t)], ctypes.c_int64),
+    "moe_route": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_permute": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+                    ctypes.c_int),
+    "moe_grouped_ffn": ([ctypes.POINTER(moe_config_t)] + [_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_combine": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_forward": ([ctypes.POINTER(moe_config_t)] + [_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_get_device_status": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_size_t, _P,
+                               ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
+    "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "moe_last_error": ([], ctypes.c_char_p),
+    "moe_trace_begin": ([ctypes.c_int32], ctypes.c_int),
+    "moe_trace_end": ([ctypes.POINTER(moe_trace_record_t), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)],
+                      ctypes.c_int),
+}
+
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load libmoe.so (built by ``sparse_mixture_experts_19_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise MoeError(4, f"{p} is missing; build it with `python -m sparse_mixture_experts_19_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (args, res) in _SIGS.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGS)
+
+
+def _check(status: int):
+    if status != 0:
+        raise MoeError(status, load().moe_last_error().decode())
+
+
+def config(T: int, H: int, I: int, E: int, top_k: int, I_shared: int = 0,
+           capacity_factor: float = 0.0, dtype: str = "bf16") -> moe_config_t:
+    return moe_config_t(T, H, I, E, top_k, I_shared, capacity_factor,
+                        MOE_BF16 if dtype == "bf16" else MOE_F32)
+
+
+def workspace_size(cfg: moe_config_t) -> int:
+    n = load().moe_workspace_size(ctypes.byref(cfg))
+    if n == 0:
+        raise MoeError(1, load().moe_last_error().decode())
+    return n
+
+
+def capacity(cfg: moe_config_t) -> int:
+    return load().moe_capacity(ctypes.byref(cfg))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise MoeError(1, "tensor is not on a CUDA device")
+    if not t.is_contiguous():
+        raise MoeError(1, "tensor is not contiguous")
+    return t.data_ptr()
+
+
+def _ws(ws):
+    return _ptr(ws), (ws.numel() * ws.element_size() if ws is not None and not isinstance(ws, int) else 0)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def workspace(cfg: moe_config_t, device="cuda"):
+    """A zeroed torch byte tensor big enough for cfg (torch allocations are
+    256-byte aligned; zeroed so the device check flags start clear)."""
+    import torch
+
+    return torch.zeros(workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def moe_route(cfg, x, router_w, router_b, topk_idx, topk_w, ws, stream=None):
+    p, n = _ws(ws)
+    _check(load().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(topk_idx),
+                            _ptr(topk_w), p, n, _stream(stream)))
+
+
+def moe_permute(cfg, topk_idx, counts, offsets, perm_rows, row_of, dropped, ws, stream=None):
+    p, n = _ws(ws)
+    _check(load().moe_permute(ctypes.byref(cfg), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                              _ptr(perm_rows), _ptr(row_of), _ptr(dropped), p, n, _stream(stream)))
+
+
+def moe_grouped_ffn(cfg, x, perm_rows, offsets, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
+                    expert_out, ws, stream=None):
+    p, n = _ws(ws)
+    _check(load().moe_grouped_ffn(ctypes.byref(cfg), _ptr(x), _ptr(perm_rows), _ptr(offsets), _ptr(w_gate),
+                                  _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down),
+                                  _ptr(expert_out), p, n, _stream(stream)))
+
+
+def moe_combine(cfg, expert_out, row_of, topk_w, y, ws, stream=None):
+    p, n = _ws(ws)
+    _check(load().moe_combine(ctypes.byref(cfg), _ptr(expert_out), _ptr(row_of), _ptr(topk_w), _ptr(y),
+                              p, n, _stream(stream)))
+
+
+def moe_forward(cfg, x, router_w, router_b, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y,
+                topk_idx_out=None, counts_out=None, dropped_out=None, ws=None, stream=None):
+    p, n = _ws(ws)
+    _check(load().moe_forward(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(w_gate),
+                              _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y),
+                              _ptr(topk_idx_out), _ptr(counts_out), _ptr(dropped_out), p, n,
+                              _stream(stream)))
+
+
+def moe_get_device_status(cfg, ws, stream=None) -> int:
+    """Waits for the stream; returns the device check flags (and clears them)."""
+    p, n = _ws(ws)
+    flags = ctypes.c_int32(0)
+    st = load().moe_get_device_status(ctypes.byref(cfg), p, n, _stream(stream), ctypes.byref(flags))
+    if st not in (0, 5):
+        _check(st)
+    return flags.value
+
+
+def moe_status_string(status: int) -> str:
+    return load().moe_status_string(status).decode()
+
+
+def moe_last_error() -> str:
+    return load().moe_last_error().decode()
+
+
+def moe_trace_begin(max_launches: int):
+    _check(load().moe_trace_begin(max_launches))
+
+
+def moe_trace_end(max_records: int = 4096) -> list[tuple[str, float]]:
+    recs = (moe_trace_record_t * max_records)()
+    n = ctypes.c_int32(0)
+    _check(load().moe_trace_end(recs, max_records, ctypes.byref(n)))
+    return [(recs[i].name.decode(), recs[i].ms) for i in range(n.value)]
+
+
+def forward(x, router_w, w_gate, w_up, w_down, top_k: int, router_b=None, ws_gate=None, ws_up=None,
+            ws_down=None, capacity_factor: float = 0.0, ws=None, topk_idx_out=None, counts_out=None,
+            dropped_out=None, stream=None):
+    """y = MoE(x): the pages' moe_forward(x, experts, router, top_k) on the GPU."""
+    import torch
+
+    T, H = x.shape
+    E, I, _ = w_gate.shape
+    Is = 0 if ws_gate is None else ws_gate.shape[0]
+    dtype = "bf16" if x.dtype == torch.bfloat16 else "f32"
+    cfg = config(T, H, I, E, top_k, Is, capacity_factor, dtype)
+    if ws is None:
+        ws = workspace(cfg, x.device)
+    y = torch.empty_like(x)
+    moe_forward(cfg, x, router_w, router_b, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y,
+                topk_idx_out, counts_out, dropped_out, ws, stream)
+    return y

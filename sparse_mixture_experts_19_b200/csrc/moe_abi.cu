@@ -1,0 +1,368 @@
+// Host side of the C ABI declared in include/moe.h: argument checks,
+// workspace carving, launch sequencing, status codes and kernel tracing.
+// No entry point allocates device memory or synchronises, except
+// moe_get_device_status (documented to wait) and moe_trace_end.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <vector>
+
+#include "common.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ errors
+static thread_local char g_last_error[256] = "";
+
+static moe_status_t fail(moe_status_t st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+static moe_status_t cuda_fail(cudaError_t e, const char* where) {
+    return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// ----------------------------------------------------------------- tracing
+namespace {
+struct TraceState {
+    bool on = false;
+    int max = 0;
+    int n = 0;
+    bool open = false;  // a launch has been started and not yet closed
+    std::vector<const char*> names;
+    std::vector<cudaEvent_t> ev;
+};
+TraceState g_trace;
+}  // namespace
+
+void trace_before(const char* name, cudaStream_t st) {
+    if (!g_trace.on || g_trace.n >= g_trace.max) return;
+    if (cudaEventRecord(g_trace.ev[2 * g_trace.n], st) != cudaSuccess) return;
+    g_trace.names[g_trace.n] = name;
+    g_trace.open = true;
+}
+
+void trace_after(cudaStream_t st) {
+    if (!g_trace.on || !g_trace.open) return;
+    g_trace.open = false;
+    if (cudaEventRecord(g_trace.ev[2 * g_trace.n + 1], st) == cudaSuccess) g_trace.n++;
+}
+
+// --------------------------------------------------------------- the plan
+static moe_status_t check_config(const moe_config_t* c) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+    if (c->T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %d < 0", c->T);
+    if (c->H < 8 || c->H % 8) return fail(MOE_ERR_INVALID_ARG, "H = %d must be a positive multiple of 8", c->H);
+    if (c->I < 8 || c->I % 8) return fail(MOE_ERR_INVALID_ARG, "I = %d must be a positive multiple of 8", c->I);
+    if (c->E < 1 || c->E > kMaxExperts) return fail(MOE_ERR_INVALID_ARG, "E = %d outside 1..%d", c->E, kMaxExperts);
+    bool k_ok = (c->top_k >= 1 && c->top_k <= c->E && c->top_k <= 8) || (c->top_k == c->E && c->E <= kMaxTopK);
+    if (!k_ok) return fail(MOE_ERR_INVALID_ARG, "top_k = %d must be in 1..min(E,8), or equal E <= 32", c->top_k);
+    if (c->I_shared < 0 || c->I_shared % 8) return fail(MOE_ERR_INVALID_ARG, "I_shared = %d must be 0 or a positive multiple of 8", c->I_shared);
+    if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype = %d unknown", c->dtype);
+    if (!isfinite(c->capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is not finite");
+    if ((int64_t)c->T * c->top_k > INT32_MAX / 2) return fail(MOE_ERR_UNSUPPORTED, "T * top_k too large");
+    return MOE_OK;
+}
+
+static int64_t capacity_of(const moe_config_t* c) {
+    if (c->capacity_factor <= 0.f) return 0;
+    double C = ceil((double)c->capacity_factor * (double)c->T * (double)c->top_k / (double)c->E);
+    return C < 1.0 ? 1 : (int64_t)C;
+}
+
+static size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+// Fills the plan; with ws == nullptr only sizes are computed.
+static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
+    p->T = c->T;
+    p->H = c->H;
+    p->I = c->I;
+    p->E = c->E;
+    p->k = c->top_k;
+    p->Is = c->I_shared;
+    p->S = p->T * p->k;
+    p->cap = capacity_of(c);
+    p->bf16 = (c->dtype == MOE_BF16);
+    p->nchunks = (p->S + kPermuteChunk - 1) / kPermuteChunk;
+    p->h_rows = p->S + (p->Is ? p->T : 0);
+    p->I_max = p->I > p->Is ? p->I : p->Is;
+    const size_t elt = p->bf16 ? 2 : 4;
+    size_t off = 0;
+    char* base = (char*)ws;
+    auto take = [&](size_t bytes) -> void* {
+        void* r = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return r;
+    };
+    p->flags = (int32_t*)take(64);
+    p->topk_idx = (int32_t*)take(sizeof(int32_t) * p->S);
+    p->topk_w = (float*)take(sizeof(float) * p->S);
+    p->chunk_base = (int32_t*)take(sizeof(int32_t) * p->nchunks * p->E);
+    p->counts = (int32_t*)take(sizeof(int32_t) * p->E);
+    p->dropped = (int32_t*)take(sizeof(int32_t) * p->E);
+    p->offsets = (int32_t*)take(sizeof(int32_t) * (p->E + 2));
+    p->perm_rows = (int32_t*)take(sizeof(int32_t) * p->S);
+    p->row_of = (int32_t*)take(sizeof(int32_t) * p->S);
+    p->xperm = take(elt * p->S * p->H);
+    p->h = take(elt * (p->S * p->I + p->T * p->Is));
+    p->yacc = (float*)take(sizeof(float) * p->T * p->H);
+    p->bytes = off;
+}
+
+static moe_status_t plan_for(const moe_config_t* c, void* ws, size_t ws_bytes, Plan* p) {
+    moe_status_t st = check_config(c);
+    if (st != MOE_OK) return st;
+    make_plan(c, nullptr, p);
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+    if ((uintptr_t)ws % kWsAlign) return fail(MOE_ERR_WORKSPACE, "workspace not %d-byte aligned", kWsAlign);
+    if (ws_bytes < p->bytes)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, p->bytes);
+    make_plan(c, ws, p);
+    return MOE_OK;
+}
+
+static bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15) == 0; }
+
+#define REQUIRE_PTR(ptr)                                                                    \
+    do {                                                                                    \
+        if (!(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", #ptr);                   \
+        if (!aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #ptr); \
+    } while (0)
+
+#define OPTIONAL_PTR(ptr)                                                                   \
+    do {                                                                                    \
+        if ((ptr) && !aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #ptr); \
+    } while (0)
+
+#define CUDA_TRY(expr, where)                           \
+    do {                                                \
+        cudaError_t e_ = (expr);                        \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+    } while (0)
+
+static moe_status_t check_shared(const Plan& p, const void* a, const void* b, const void* c) {
+    if (p.Is > 0) {
+        REQUIRE_PTR(a);
+        REQUIRE_PTR(b);
+        REQUIRE_PTR(c);
+    }
+    return MOE_OK;
+}
+
+// The grouped FFN of moe_forward / moe_grouped_ffn, after routing and grouping.
+static moe_status_t run_ffn(const Plan& p, const void* x, const void* w_gate, const void* w_up,
+                            const void* w_down, const void* ws_gate, const void* ws_up,
+                            const void* ws_down, int mode, float* out, cudaStream_t st) {
+    CUDA_TRY(launch_gather_rows(p, x, p.perm_rows, p.offsets, p.xperm, st), "gather_rows");
+    CUDA_TRY(launch_gateup_simt(p, p.xperm, x, p.offsets, w_gate, w_up, ws_gate, ws_up, p.h, st),
+             "gateup");
+    CUDA_TRY(launch_down_simt(p, p.h, p.offsets, p.perm_rows, p.topk_w, w_down, ws_down, mode, out, st),
+             "down");
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config_t* cfg) {
+    if (check_config(cfg) != MOE_OK) return 0;
+    Plan p;
+    make_plan(cfg, nullptr, &p);
+    return p.bytes;
+}
+
+int64_t moe_capacity(const moe_config_t* cfg) {
+    if (check_config(cfg) != MOE_OK) return -1;
+    return capacity_of(cfg);
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* router_w,
+                       const float* router_b, int32_t* topk_idx, float* topk_w, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    if (p.T == 0) return MOE_OK;
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(router_w);
+    OPTIONAL_PTR(router_b);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    cudaStream_t st = (cudaStream_t)stream;
+    CUDA_TRY(launch_router_simt(p, x, router_w, router_b, topk_idx, topk_w, nullptr, st), "router");
+    return MOE_OK;
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
+                         int32_t* offsets, int32_t* perm_rows, int32_t* row_of, int32_t* dropped,
+                         void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    REQUIRE_PTR(counts);
+    REQUIRE_PTR(offsets);
+    REQUIRE_PTR(dropped);
+    if (p.S > 0) {
+        REQUIRE_PTR(topk_idx);
+        REQUIRE_PTR(perm_rows);
+        REQUIRE_PTR(row_of);
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    CUDA_TRY(launch_permute(p, topk_idx, counts, offsets, perm_rows, row_of, dropped, st), "permute");
+    return MOE_OK;
+}
+
+moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const int32_t* perm_rows,
+                             const int32_t* offsets, const void* w_gate, const void* w_up,
+                             const void* w_down, const void* ws_gate, const void* ws_up,
+                             const void* ws_down, float* expert_out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    if (p.T == 0) return MOE_OK;
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(perm_rows);
+    REQUIRE_PTR(offsets);
+    REQUIRE_PTR(w_gate);
+    REQUIRE_PTR(w_up);
+    REQUIRE_PTR(w_down);
+    REQUIRE_PTR(expert_out);
+    if ((s = check_shared(p, ws_gate, ws_up, ws_down)) != MOE_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the grouped kernels read the plan's copies of perm_rows and offsets [E+2]
+    CUDA_TRY(launch_offsets_from_user(p, offsets, st), "offsets");
+    CUDA_TRY(cudaMemcpyAsync(p.perm_rows, perm_rows, sizeof(int32_t) * p.S, cudaMemcpyDeviceToDevice, st),
+             "perm_rows copy");
+    return run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 0, expert_out, st);
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const float* expert_out, const int32_t* row_of,
+                         const float* topk_w, void* y, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    if (p.T == 0) return MOE_OK;
+    REQUIRE_PTR(expert_out);
+    REQUIRE_PTR(row_of);
+    REQUIRE_PTR(topk_w);
+    REQUIRE_PTR(y);
+    CUDA_TRY(launch_combine(p, expert_out, row_of, topk_w, y, (cudaStream_t)stream), "combine");
+    return MOE_OK;
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* router_w,
+                         const float* router_b, const void* w_gate, const void* w_up,
+                         const void* w_down, const void* ws_gate, const void* ws_up,
+                         const void* ws_down, void* y, int32_t* topk_idx_out, int32_t* counts_out,
+                         int32_t* dropped_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    OPTIONAL_PTR(topk_idx_out);
+    OPTIONAL_PTR(counts_out);
+    OPTIONAL_PTR(dropped_out);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (p.T == 0) {
+        if (counts_out) CUDA_TRY(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * p.E, st), "memset");
+        if (dropped_out) CUDA_TRY(cudaMemsetAsync(dropped_out, 0, sizeof(int32_t) * p.E, st), "memset");
+        return MOE_OK;
+    }
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(router_w);
+    OPTIONAL_PTR(router_b);
+    REQUIRE_PTR(w_gate);
+    REQUIRE_PTR(w_up);
+    REQUIRE_PTR(w_down);
+    REQUIRE_PTR(y);
+    if ((s = check_shared(p, ws_gate, ws_up, ws_down)) != MOE_OK) return s;
+
+    int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
+    int32_t* counts = counts_out ? counts_out : p.counts;
+    int32_t* dropped = dropped_out ? dropped_out : p.dropped;
+    CUDA_TRY(launch_router_simt(p, x, router_w, router_b, idx, p.topk_w, p.yacc, st), "router");
+    CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
+    if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.yacc, st)) != MOE_OK)
+        return s;
+    CUDA_TRY(launch_finalize(p, p.yacc, y, st), "finalize");
+    return MOE_OK;
+}
+
+moe_status_t moe_get_device_status(const moe_config_t* cfg, void* ws, size_t ws_bytes,
+                                   moe_stream_t stream, int32_t* flags_out) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t flags = 0;
+    CUDA_TRY(cudaMemcpyAsync(&flags, p.flags, sizeof(int32_t), cudaMemcpyDeviceToHost, st), "flags read");
+    CUDA_TRY(cudaStreamSynchronize(st), "stream sync");
+    CUDA_TRY(cudaMemsetAsync(p.flags, 0, sizeof(int32_t), st), "flags clear");
+    CUDA_TRY(cudaStreamSynchronize(st), "stream sync");
+    if (flags_out) *flags_out = flags;
+    if (flags) return fail(MOE_ERR_DEVICE_CHECK, "device check flags 0x%x", flags);
+    return MOE_OK;
+}
+
+const char* moe_status_string(moe_status_t status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_error(void) { return g_last_error; }
+
+moe_status_t moe_trace_begin(int32_t max_launches) {
+    if (max_launches <= 0) return fail(MOE_ERR_INVALID_ARG, "max_launches = %d", max_launches);
+    if (g_trace.on) return fail(MOE_ERR_INVALID_ARG, "tracing already on");
+    g_trace = TraceState();
+    g_trace.ev.resize(2 * (size_t)max_launches);
+    g_trace.names.resize(max_launches);
+    for (auto& e : g_trace.ev)
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            for (auto& f : g_trace.ev)
+                if (f) cudaEventDestroy(f);
+            g_trace = TraceState();
+            return fail(MOE_ERR_CUDA, "cudaEventCreate failed");
+        }
+    g_trace.max = max_launches;
+    g_trace.on = true;
+    return MOE_OK;
+}
+
+moe_status_t moe_trace_end(moe_trace_record_t* records, int32_t max_records, int32_t* n_records) {
+    if (!g_trace.on) return fail(MOE_ERR_INVALID_ARG, "tracing is off");
+    moe_status_t st = MOE_OK;
+    int n = g_trace.n;
+    if (n > 0 && cudaEventSynchronize(g_trace.ev[2 * n - 1]) != cudaSuccess)
+        st = fail(MOE_ERR_CUDA, "cudaEventSynchronize failed");
+    int w = 0;
+    for (int i = 0; i < n && st == MOE_OK && records && w < max_records; ++i, ++w) {
+        float ms = 0.f;
+        cudaEventElapsedTime(&ms, g_trace.ev[2 * i], g_trace.ev[2 * i + 1]);
+        records[w].name = g_trace.names[i];
+        records[w].ms = ms;
+    }
+    if (n_records) *n_records = w;
+    for (auto& e : g_trace.ev) cudaEventDestroy(e);
+    g_trace = TraceState();
+    return st;
+}
+
+}  // extern "C"

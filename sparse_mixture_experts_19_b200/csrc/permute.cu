@@ -1,0 +1,187 @@
+// Grouping of (token, slot) pairs by expert, with capacity drop in token order.
+//
+// "Mixture of Experts (MoEs) in Transformers", section Expert Backend
+// (grouped_mm sorts tokens by expert id and groups them); "MoE稀疏架构是什么？
+// 从原理到落地的系统解读", section 三.2 (capacity-limited token dropping).
+//
+// Three passes over the T*k slot ids, all bit-reproducible:
+//   1. chunk histogram: hist[c][e] = pairs of expert e in slot chunk c;
+//   2. one block per layer: exclusive scan of hist over chunks (in place), so
+//      base[c][e] = pairs of e in earlier chunks; counts, capacity cut,
+//      dropped, and the exclusive scan over experts -> offsets;
+//   3. stable scatter: each chunk walks its slots in order, 32 at a time,
+//      ranking equal experts inside a warp with __match_any_sync, so the
+//      rank of a pair is the number of earlier slots of the same expert.
+//      Slot order is token-major, hence ranks follow ascending token order,
+//      and a pair is kept iff its rank < C.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kHistThreads = 256;
+constexpr int kScanThreads = 256;  // >= kMaxExperts
+constexpr int kScatterWarps = 4;
+
+__global__ void __launch_bounds__(kHistThreads) permute_hist_kernel(
+    const int32_t* __restrict__ idx, int64_t S, int E, int32_t* __restrict__ hist,
+    int32_t* __restrict__ flags) {
+    __shared__ int32_t h[kMaxExperts];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int64_t s0 = (int64_t)blockIdx.x * kPermuteChunk;
+    const int64_t s1 = min(S, s0 + kPermuteChunk);
+    bool bad = false;
+    for (int64_t s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
+        int e = idx[s];
+        if (e >= 0 && e < E)
+            atomicAdd(&h[e], 1);
+        else
+            bad = true;
+    }
+    if (bad) set_flag(flags, MOE_DEVFLAG_BAD_EXPERT_INDEX);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = h[e];
+}
+
+__global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(
+    int32_t* __restrict__ hist, int64_t nchunks, int E, int64_t cap, int32_t* __restrict__ counts,
+    int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
+    int32_t shared_rows) {
+    __shared__ int32_t kept_s[kScanThreads];
+    const int e = threadIdx.x;
+    int32_t total = 0;
+    if (e < E) {
+        for (int64_t c = 0; c < nchunks; ++c) {
+            int32_t v = hist[c * E + e];
+            hist[c * E + e] = total;
+            total += v;
+        }
+    }
+    int32_t kept = (cap > 0 && total > cap) ? (int32_t)cap : total;
+    if (e < E) {
+        counts[e] = total;
+        dropped[e] = total - kept;
+    }
+    kept_s[e] = (e < E) ? kept : 0;
+    __syncthreads();
+    // inclusive Hillis-Steele scan over the (at most 256) experts
+    for (int o = 1; o < kScanThreads; o <<= 1) {
+        int32_t v = (e >= o) ? kept_s[e - o] : 0;
+        __syncthreads();
+        kept_s[e] += v;
+        __syncthreads();
+    }
+    // offsets_ws [E+2] feeds the GEMMs; offsets_out [E+1] is the caller's copy
+    if (e < E) {
+        int32_t excl = kept_s[e] - kept;
+        offsets_ws[e] = excl;
+        offsets_out[e] = excl;
+    }
+    if (e == 0) {
+        int32_t R = kept_s[E - 1];
+        offsets_ws[E] = R;
+        offsets_ws[E + 1] = R + shared_rows;
+        offsets_out[E] = R;
+    }
+}
+
+__global__ void __launch_bounds__(kScatterWarps * 32) permute_scatter_kernel(
+    const int32_t* __restrict__ idx, int64_t S, int E, int64_t cap,
+    const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of) {
+    __shared__ int32_t run[kScatterWarps][kMaxExperts];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t c = (int64_t)blockIdx.x * kScatterWarps + warp;
+    const int64_t s0 = c * kPermuteChunk;
+    if (s0 >= S) return;
+    for (int e = lane; e < E; e += 32) run[warp][e] = base[c * E + e];
+    __syncwarp();
+    const int64_t s1 = min(S, s0 + kPermuteChunk);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t sb = s0; sb < s1; sb += 32) {
+        int64_t s = sb + lane;
+        int e = (s < s1) ? idx[s] : -1;
+        bool valid = (e >= 0 && e < E);
+        int key = valid ? e : -1;
+        uint32_t peers = __match_any_sync(0xffffffffu, key);
+        int32_t rank = 0;
+        if (valid) rank = run[warp][e] + __popc(peers & lt);
+        __syncwarp();
+        if (valid && (peers & lt) == 0) run[warp][e] += __popc(peers);  // lowest peer updates
+        __syncwarp();
+        if (s < s1) {
+            if (valid && (cap <= 0 || rank < cap)) {
+                int32_t row = offsets[e] + rank;
+                perm_rows[row] = (int32_t)s;
+                row_of[s] = row;
+            } else {
+                row_of[s] = -1;
+            }
+        }
+    }
+}
+
+// perm_rows entries at and past R are set to -1.
+__global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_t S,
+                                         const int32_t* __restrict__ offsets, int E) {
+    const int64_t R = offsets[E];
+    for (int64_t r = R + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < S;
+         r += (int64_t)gridDim.x * blockDim.x)
+        perm_rows[r] = -1;
+}
+
+__global__ void offsets_from_user_kernel(const int32_t* __restrict__ user, int E,
+                                         int32_t shared_rows, int32_t* __restrict__ ws_off) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) ws_off[e] = user[e];
+    if (threadIdx.x == 0) ws_off[E + 1] = user[E] + shared_rows;
+}
+
+}  // namespace
+
+cudaError_t launch_offsets_from_user(const Plan& p, const int32_t* offsets, cudaStream_t st) {
+    trace_before("offsets_from_user", st);
+    offsets_from_user_kernel<<<1, 256, 0, st>>>(offsets, (int)p.E, (int32_t)(p.Is > 0 ? p.T : 0),
+                                                p.offsets);
+    trace_after(st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
+                           int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
+                           int32_t* dropped, cudaStream_t st) {
+    if (p.S == 0) {
+        // nothing routed: all counts and offsets are zero
+        cudaError_t e1 = cudaMemsetAsync(counts, 0, sizeof(int32_t) * p.E, st);
+        if (e1 == cudaSuccess) e1 = cudaMemsetAsync(dropped, 0, sizeof(int32_t) * p.E, st);
+        if (e1 == cudaSuccess) e1 = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p.E + 1), st);
+        if (e1 == cudaSuccess && offsets != p.offsets)
+            e1 = cudaMemsetAsync(p.offsets, 0, sizeof(int32_t) * (p.E + 1), st);
+        if (e1 == cudaSuccess) {
+            // offsets[E+1] = shared rows (T = 0 here, so also 0)
+            e1 = cudaMemsetAsync(p.offsets + p.E, 0, sizeof(int32_t) * 2, st);
+        }
+        return e1;
+    }
+    const int E = (int)p.E;
+    trace_before("permute_hist", st);
+    permute_hist_kernel<<<(unsigned)p.nchunks, kHistThreads, 0, st>>>(topk_idx, p.S, E,
+                                                                       p.chunk_base, p.flags);
+    trace_after(st);
+    trace_before("permute_scan", st);
+    permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
+        p.chunk_base, p.nchunks, E, p.cap, counts, dropped, offsets, p.offsets,
+        (int32_t)(p.Is > 0 ? p.T : 0));
+    trace_after(st);
+    trace_before("permute_scatter", st);
+    unsigned blocks = (unsigned)((p.nchunks + kScatterWarps - 1) / kScatterWarps);
+    permute_scatter_kernel<<<blocks, kScatterWarps * 32, 0, st>>>(
+        topk_idx, p.S, E, p.cap, p.chunk_base, p.offsets, perm_rows, row_of);
+    trace_after(st);
+    trace_before("permute_fill_tail", st);
+    permute_fill_tail_kernel<<<64, 256, 0, st>>>(perm_rows, p.S, p.offsets, E);
+    trace_after(st);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

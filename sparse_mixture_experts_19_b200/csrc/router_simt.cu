@@ -1,0 +1,153 @@
+// Router scores + top-k + softmax over the selected scores, CUDA-core version.
+//
+// "MoE稀疏架构是什么？从原理到落地的系统解读", section 三.1 (a small linear
+// router gives one score per expert) and section 四 (keep the top-k scores,
+// softmax over those k).  Scores accumulate in float32 FMAs.  This kernel
+// serves the float32 layer, where tensor cores would round the inputs.
+//
+// One block scores 32 tokens against all E experts: x and router-weight
+// chunks of 32 columns are staged in shared memory as float; each thread owns
+// up to 32 (token, expert) accumulators.  The scores then go to shared memory
+// and each warp selects the top-k of 4 tokens with warp arg-max rounds.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTB = 32;  // tokens per block
+constexpr int kHC = 32;  // hidden columns per chunk
+constexpr int kThreads = 256;
+
+// Warp-wide arg-max of (v, e): larger v wins, equal v -> lower e wins.
+__device__ __forceinline__ void warp_argmax(float& v, int& e) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        int oe = __shfl_xor_sync(0xffffffffu, e, o);
+        if (ov > v || (ov == v && oe < e)) {
+            v = ov;
+            e = oe;
+        }
+    }
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads) router_simt_kernel(
+    int T, int H, int E, int k, const TIn* __restrict__ x, const TIn* __restrict__ wr,
+    const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    float* __restrict__ yacc) {
+    __shared__ float xs[kTB][kHC + 1];
+    // weights chunk [E][kHC+1] during the scores, then scores [kTB][E+1]
+    __shared__ float buf[kMaxExperts * (kHC + 1)];
+
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.x * kTB;
+    const int P = kTB * E;  // (token, expert) pairs of this block
+
+    float acc[kTB * kMaxExperts / kThreads];
+#pragma unroll
+    for (int i = 0; i < kTB * kMaxExperts / kThreads; ++i) acc[i] = 0.f;
+
+    for (int h0 = 0; h0 < H; h0 += kHC) {
+        for (int q = tid; q < kTB * kHC; q += kThreads) {
+            int r = q / kHC, c = q % kHC;
+            int t = t0 + r, h = h0 + c;
+            xs[r][c] = (t < T && h < H) ? to_f32(x[(int64_t)t * H + h]) : 0.f;
+        }
+        for (int q = tid; q < E * kHC; q += kThreads) {
+            int r = q / kHC, c = q % kHC;
+            int h = h0 + c;
+            buf[r * (kHC + 1) + c] = (h < H) ? to_f32(wr[(int64_t)r * H + h]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kTB * kMaxExperts / kThreads; ++i) {
+            int p = tid + i * kThreads;
+            if (p < P) {
+                int r = p / E, e = p % E;
+                float s = acc[i];
+#pragma unroll 8
+                for (int c = 0; c < kHC; ++c) s = fmaf(xs[r][c], buf[e * (kHC + 1) + c], s);
+                acc[i] = s;
+            }
+        }
+        __syncthreads();
+    }
+
+    // scores -> shared memory (bias added here, before selection)
+#pragma unroll
+    for (int i = 0; i < kTB * kMaxExperts / kThreads; ++i) {
+        int p = tid + i * kThreads;
+        if (p < P) {
+            int r = p / E, e = p % E;
+            buf[r * (E + 1) + e] = acc[i] + (b ? b[e] : 0.f);
+        }
+    }
+    __syncthreads();
+
+    const int warp = tid / 32, lane = tid % 32;
+    for (int r = warp; r < kTB; r += kThreads / 32) {
+        int t = t0 + r;
+        if (t >= T) break;
+        const float* l = buf + r * (E + 1);
+        // each lane holds experts lane, lane+32, ...; taken bits mark chosen ones
+        uint32_t taken = 0;
+        float sel_v[kMaxTopK];
+        int sel_e[kMaxTopK];
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+            for (int q = 0; q * 32 + lane < E; ++q) {
+                int e = q * 32 + lane;
+                float v = l[e];
+                if (!((taken >> q) & 1u) && (v > bv || (v == bv && e < be))) {
+                    bv = v;
+                    be = e;
+                }
+            }
+            warp_argmax(bv, be);
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            sel_v[j] = bv;
+            sel_e[j] = be;
+        }
+        if (lane == 0) {
+            float m = sel_v[0], z = 0.f;
+            for (int j = 0; j < k; ++j) z += expf(sel_v[j] - m);
+            float inv = 1.0f / z;
+            for (int j = 0; j < k; ++j) {
+                topk_idx[(int64_t)t * k + j] = sel_e[j];
+                topk_w[(int64_t)t * k + j] = expf(sel_v[j] - m) * inv;
+            }
+        }
+    }
+
+    // zero the combine accumulator rows of these tokens
+    if (yacc) {
+        int rows = min(kTB, T - t0);
+        float4* dst = reinterpret_cast<float4*>(yacc + (int64_t)t0 * H);
+        int64_t n4 = (int64_t)rows * H / 4;
+        for (int64_t q = tid; q < n4; q += kThreads) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_w,
+                               const float* router_b, int32_t* topk_idx, float* topk_w,
+                               float* yacc_zero, cudaStream_t st) {
+    if (p.T == 0) return cudaSuccess;
+    dim3 grid((unsigned)((p.T + kTB - 1) / kTB));
+    trace_before("router_simt", st);
+    if (p.bf16)
+        router_simt_kernel<bf16><<<grid, kThreads, 0, st>>>(
+            (int)p.T, (int)p.H, (int)p.E, (int)p.k, (const bf16*)x, (const bf16*)router_w,
+            router_b, topk_idx, topk_w, yacc_zero);
+    else
+        router_simt_kernel<float><<<grid, kThreads, 0, st>>>(
+            (int)p.T, (int)p.H, (int)p.E, (int)p.k, (const float*)x, (const float*)router_w,
+            router_b, topk_idx, topk_w, yacc_zero);
+    trace_after(st);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

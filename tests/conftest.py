@@ -21,6 +21,8 @@ def gpu_lib():
     if not torch.cuda.is_available():
         pytest.fail("GPU test collected on a machine without CUDA")
     import sparse_mixture_experts_19_b200 as moe
+    from sparse_mixture_experts_19_b200 import build
 
+    build.build()
     moe.load()
     return moe
