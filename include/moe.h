@@ -133,6 +133,32 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32
                          void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_permute_noalloc -- moe_permute for callers that cannot allocate
+ * device memory: code running inside an allocator or memory-pool callback,
+ * plugins whose host application owns every device allocation, serving
+ * loops that forbid allocation after start-up.  The pages have no
+ * counterpart of this entry point; it only changes where the scratch lives.
+ *   Same arguments, outputs and bit-exact results as moe_permute, without
+ *   `ws`: the grouping kernels' scratch (about 520 KB) is a fixed array in
+ *   the library's device memory, which every GPU that loads the library
+ *   holds until the process exits.  This call allocates nothing (no
+ *   cudaMalloc, no allocating library routine).
+ *   Limit: T * top_k <= 1048576 slots (E <= 256 as everywhere); larger
+ *   inputs return MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *   The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before any
+ *   stream capture.
+ *   Every call on a device shares the one array, which keeps the last
+ *   call's contents; calls that overlap on the GPU (concurrent streams)
+ *   race and give wrong results, so order them.  An expert index outside
+ *   [0, E) is skipped as in moe_permute but not reported: there is no
+ *   workspace to hold the flag.
+ */
+moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
+                                 int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
+                                 int32_t* dropped, moe_stream_t stream);
+
+/*
  * moe_grouped_ffn -- every kept row through its expert's SwiGLU FFN, as
  * grouped GEMMs over the rows of each expert ("Mixture of Experts (MoEs) in
  * Transformers", section Expert Backend, grouped_mm).

@@ -47,6 +47,7 @@ _SIGS = {
     "moe_route": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_permute": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
                     ctypes.c_int),
+    "moe_permute_noalloc": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_grouped_ffn": ([ctypes.POINTER(moe_config_t)] + [_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_combine": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_forward": ([ctypes.POINTER(moe_config_t)] + [_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int),
@@ -148,6 +149,15 @@ def moe_permute(cfg, topk_idx, counts, offsets, perm_rows, row_of, dropped, ws, 
     p, n = _ws(ws)
     _check(load().moe_permute(ctypes.byref(cfg), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
                               _ptr(perm_rows), _ptr(row_of), _ptr(dropped), p, n, _stream(stream)))
+
+
+def moe_permute_noalloc(cfg, topk_idx, counts, offsets, perm_rows, row_of, dropped, stream=None):
+    """moe_permute without a workspace, for callers that cannot allocate device
+    memory (allocator callbacks, host-owned memory, allocation-free serving
+    loops): the scratch is a fixed static array inside the library.  Limit
+    T*top_k <= 1048576; concurrent calls on one device race."""
+    _check(load().moe_permute_noalloc(ctypes.byref(cfg), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                      _ptr(perm_rows), _ptr(row_of), _ptr(dropped), _stream(stream)))
 
 
 def moe_grouped_ffn(cfg, x, perm_rows, offsets, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,

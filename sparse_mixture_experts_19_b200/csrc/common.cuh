@@ -15,6 +15,7 @@ constexpr int kMaxTopK = 32;     // k <= 8, or k == E <= 32 (dense case)
 constexpr int kMaxExperts = 256;
 constexpr int kPermuteChunk = 2048;  // slots per histogram chunk in moe_permute
 constexpr int kWsAlign = 256;
+constexpr int64_t kNoAllocMaxSlots = 1 << 20;  // T*k limit of moe_permute_noalloc
 
 // Everything the kernels of one call need, carved out of the caller's workspace.
 struct Plan {
@@ -58,6 +59,10 @@ cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_
 cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
                            int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
                            int32_t* dropped, cudaStream_t st);
+// moe_permute with the scratch in a static device array; sizes.S <= kNoAllocMaxSlots.
+cudaError_t launch_permute_noalloc(const Plan& sizes, const int32_t* topk_idx, int32_t* counts,
+                                   int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
+                                   int32_t* dropped, cudaStream_t st);
 // plan offsets [E+2] from a caller's offsets [E+1] (appends the shared rows).
 cudaError_t launch_offsets_from_user(const Plan& p, const int32_t* offsets, cudaStream_t st);
 cudaError_t launch_gather_rows(const Plan& p, const void* x, const int32_t* perm_rows,

@@ -221,6 +221,32 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32
     return MOE_OK;
 }
 
+moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
+                                 int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
+                                 int32_t* dropped, moe_stream_t stream) {
+    moe_status_t s = check_config(cfg);
+    if (s != MOE_OK) return s;
+    Plan p;
+    make_plan(cfg, nullptr, &p);  // sizes only: this entry point takes no workspace
+    if (p.S > kNoAllocMaxSlots)
+        return fail(MOE_ERR_UNSUPPORTED,
+                    "moe_permute_noalloc handles at most %lld slots (T*top_k) in its static scratch; "
+                    "got %lld, use moe_permute with a workspace",
+                    (long long)kNoAllocMaxSlots, (long long)p.S);
+    REQUIRE_PTR(counts);
+    REQUIRE_PTR(offsets);
+    REQUIRE_PTR(dropped);
+    if (p.S > 0) {
+        REQUIRE_PTR(topk_idx);
+        REQUIRE_PTR(perm_rows);
+        REQUIRE_PTR(row_of);
+    }
+    CUDA_TRY(launch_permute_noalloc(p, topk_idx, counts, offsets, perm_rows, row_of, dropped,
+                                    (cudaStream_t)stream),
+             "permute_noalloc");
+    return MOE_OK;
+}
+
 moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const int32_t* perm_rows,
                              const int32_t* offsets, const void* w_gate, const void* w_up,
                              const void* w_down, const void* ws_gate, const void* ws_up,

@@ -14,6 +14,8 @@
 //      rank of a pair is the number of earlier slots of the same expert.
 //      Slot order is token-major, hence ranks follow ascending token order,
 //      and a pair is kept iff its rank < C.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -182,6 +184,63 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
     permute_fill_tail_kernel<<<64, 256, 0, st>>>(perm_rows, p.S, p.offsets, E);
     trace_after(st);
     return cudaGetLastError();
+}
+
+
+// ------------------------------------------------------------------------
+// Allocation-free variant (moe_permute_noalloc).  Some callers cannot call
+// cudaMalloc at the point where they group tokens: code running inside a
+// framework's custom allocator or memory-pool callback, plugins whose host
+// application owns every device allocation, and tight serving loops that
+// forbid allocation after start-up.  For them the scratch of the grouping
+// kernels (per-chunk histograms, the offsets copy and a flag word) lives in
+// this fixed file-scope device array instead of a caller workspace.  Every
+// GPU that loads the library holds it until the process exits.
+namespace {
+
+constexpr int64_t kNoAllocChunks = kNoAllocMaxSlots / kPermuteChunk;
+constexpr int64_t kNoAllocInts = kNoAllocChunks * kMaxExperts + 2 * (kMaxExperts + 2) + 64;
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocInts];
+
+// Device address of g_noalloc_scratch on each device, looked up once per
+// device (with that device current).  In host code the array's name is only
+// a host-side stand-in, never a device address.
+std::mutex g_noalloc_mu;
+int32_t* g_noalloc_ptr[64] = {};
+
+cudaError_t noalloc_scratch(int32_t** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = static_cast<int32_t*>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_permute_noalloc(const Plan& sizes, const int32_t* topk_idx, int32_t* counts,
+                                   int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
+                                   int32_t* dropped, cudaStream_t st) {
+    if (sizes.S > kNoAllocMaxSlots) return cudaErrorInvalidValue;
+    int32_t* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+    Plan p = sizes;
+    p.chunk_base = scratch;                                 // [kNoAllocChunks * E]
+    p.offsets = scratch + kNoAllocChunks * kMaxExperts;     // [E + 2]
+    p.flags = p.offsets + 2 * (kMaxExperts + 2);            // flag word, cleared per call
+    e = cudaMemsetAsync(p.flags, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
+    return launch_permute(p, topk_idx, counts, offsets, perm_rows, row_of, dropped, st);
 }
 
 }  // namespace moe
