@@ -168,7 +168,11 @@ def oracle_tokens_per_s(wl, inp, target_s: float, seed: int = 3):
                           ws_gate=inp["ws_gate"], ws_up=inp["ws_up"], ws_down=inp["ws_down"])
         return time.perf_counter() - t0
 
-    t1 = run(2) / 2
+    # calibrate on enough tokens to keep every OpenMP thread busy
+    import oracle as _o
+
+    nc = max(2, 2 * _o.threads())
+    t1 = run(min(nc, wl.T)) / min(nc, wl.T)
     n = int(max(2, min(wl.T, target_s / max(t1, 1e-6))))
     dt = run(n)
     return n / dt, n, dt, oracle.threads()
@@ -339,14 +343,15 @@ def run_ours(args, wl, world, rank, local):
             kept = int(np.minimum(counts.cpu().numpy(), wl.capacity()).sum())
         flops = 2.0 * kept * 2 * wl.H * wl.I + 2.0 * wl.T * 2 * wl.H * wl.I_shared
         achieved = flops / t_avg / 1e12
-        peak = pk["bf16_tflops_sustained"]
+        # the timed region lasts well under a second at full SM clock: burst peak
+        peak = pk["bf16_tflops"]
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic_for(dom, wl),
-                "peak_kind": f"{pk_kind} bf16 dense, sustained", "launch_ms": t_avg * 1e3,
-                "flops_per_launch": flops}
+                "peak_kind": f"{pk_kind} bf16 dense, burst", "launch_ms": t_avg * 1e3,
+                "flops_per_launch": flops, "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
     F = wl.flops()
     B = layer_bytes(wl, active)
-    t_roof = max(F / (pk["bf16_tflops_sustained"] * 1e12), B / (pk["hbm_gbs"] * 1e9))
+    t_roof = max(F / (pk["bf16_tflops"] * 1e12), B / (pk["hbm_gbs"] * 1e9))
     t_step = ms / args.steps / 1e3
 
     out = {
@@ -357,8 +362,8 @@ def run_ours(args, wl, world, rank, local):
                        % (active * 3 * wl.H * wl.I * 2 / 1e9), parallelism=f"replicas{world}"),
         "roofline": roof,
         "layer_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / t_step, "flops": F, "bytes": B,
-                           "bound": "tensor" if F / (pk["bf16_tflops_sustained"] * 1e12) >= B / (pk["hbm_gbs"] * 1e9) else "hbm",
-                           "peak_kind": pk_kind},
+                           "bound": "tensor" if F / (pk["bf16_tflops"] * 1e12) >= B / (pk["hbm_gbs"] * 1e9) else "hbm",
+                           "peak_kind": f"{pk_kind} (bf16 burst, HBM copy)"},
         "kernels_ms_per_step": {k: sum(v) / args.steps for k, v in per_kernel.items()},
         "gpu_launches": len(trace),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s",

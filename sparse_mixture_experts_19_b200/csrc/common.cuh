@@ -15,6 +15,7 @@ constexpr int kMaxTopK = 32;     // k <= 8, or k == E <= 32 (dense case)
 constexpr int kMaxExperts = 256;
 constexpr int kPermuteChunk = 2048;  // slots per histogram chunk in moe_permute
 constexpr int kWsAlign = 256;
+constexpr int kGemmTileRows = 128;  // rows per tile of the tcgen05 grouped GEMMs
 constexpr int64_t kNoAllocMaxSlots = 1 << 20;  // T*k limit of moe_permute_noalloc
 
 // Everything the kernels of one call need, carved out of the caller's workspace.
@@ -33,6 +34,7 @@ struct Plan {
     int32_t* counts;      // [E]
     int32_t* dropped;     // [E]
     int32_t* offsets;     // [E + 2]: routed rows, offsets[E+1] = offsets[E] + shared rows
+    int32_t* mtile_prefix;  // [E + 1]: prefix over experts of ceil(kept rows / 128)
     int32_t* perm_rows;   // [S]
     int32_t* row_of;      // [S]
     void* xperm;          // [S, H] layer dtype: x rows in grouped order
@@ -76,6 +78,12 @@ cudaError_t launch_gateup_simt(const Plan& p, const void* xperm, const void* x,
 cudaError_t launch_down_simt(const Plan& p, const void* h, const int32_t* offsets,
                              const int32_t* perm_rows, const float* topk_w, const void* w_down,
                              const void* ws_down, int mode, float* out, cudaStream_t st);
+// tcgen05 grouped GEMMs (bf16): h = silu(X W_g^T) * (X W_u^T); out = h W_d^T
+// (mode 0: float32 rows; mode 1: weighted atomic add into yacc[token]).
+cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate, const void* w_up,
+                                const void* ws_gate, const void* ws_up, cudaStream_t st);
+cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_down, int mode,
+                              float* out, cudaStream_t st);
 cudaError_t launch_finalize(const Plan& p, const float* yacc, void* y, cudaStream_t st);
 cudaError_t launch_combine(const Plan& p, const float* expert_out, const int32_t* row_of,
                            const float* topk_w, void* y, cudaStream_t st);

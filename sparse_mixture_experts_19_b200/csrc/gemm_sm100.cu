@@ -1,0 +1,489 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// "Mixture of Experts (MoEs) in Transformers", section Expert Backend: the
+// grouped_mm backend sorts tokens by expert and runs one grouped GEMM;
+// section Weight Loading Refactor: experts packed as [E, out, in] tensors.
+// "MoE稀疏架构是什么？从原理到落地的系统解读", section 四: the output is the
+// routing-weighted sum of the selected experts' outputs.
+//
+// Two kernels from one template:
+//   gate/up:  h = silu(X W_g[e]^T) * (X W_u[e]^T), rounded to bf16.  One MMA
+//             of N = 256 covers 128 gate rows and the 128 matching up rows,
+//             so G and U of a tile land side by side in one TMEM accumulator
+//             and the SwiGLU is applied in the epilogue.
+//   down:     out = h W_d[e]^T; the epilogue multiplies row r by its routing
+//             weight and adds it into the float32 accumulator of its token
+//             (vector atomics), or stores float32 rows (stage API).
+//
+// Groups: 0..E-1 routed experts (rows offsets[g]..offsets[g+1] of the
+// grouped activations), group E the shared expert (token rows of x / hs).
+// A tile is 128 rows x BN columns of one group; tiles of one expert are
+// ordered m-fastest inside each weight column block so CTAs running side by
+// side share the same weight slice through L2.
+//
+// Persistent CTA per SM, 192 threads: warp 0 issues TMA loads into a 4-stage
+// shared-memory ring, warp 1 issues tcgen05.mma (one thread) and owns the
+// TMEM (2 accumulators x 256 columns, so the epilogue of one tile overlaps
+// the main loop of the next), warps 2-5 drain TMEM (one 32-lane quadrant
+// each).  Every wait is bounded; a timeout sets MOE_DEVFLAG_WAIT_TIMEOUT and
+// the CTA unwinds and frees its TMEM.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;   // tile rows = MMA M
+constexpr int kBK = 64;    // K per stage: one 128-byte swizzle atom of bf16
+constexpr int kStages = 4;
+constexpr int kBRows = 256;  // B rows per stage = MMA N
+constexpr int kABytes = kBM * kBK * 2;
+constexpr int kBBytes = kBRows * kBK * 2;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kAccCols = 256;
+constexpr int kTmemCols = 2 * kAccCols;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kIdesc = idesc_bf16(kBM, kBRows);
+
+struct GemmArgs {
+    const int32_t* offsets;       // [E+2]
+    const int32_t* mtile_prefix;  // [E+1] prefix of ceil(rows_e / 128)
+    int32_t* flags;
+    int E, T, has_shared;
+    int N, Ns;  // output columns (routed, shared)
+    int K, Ks;  // reduction length (routed, shared)
+    bf16* h;    // gate/up: [S, N] routed, [T, Ns] shared
+    bf16* hs;
+    const int32_t* perm_rows;  // down: row -> slot
+    const float* topk_w;       // down: slot -> routing weight
+    int k;
+    float* out;  // down mode 1: yacc [T, N]; mode 0: rows [S + T, N]
+    int64_t S;
+    int mode;
+};
+
+struct Tables {
+    int32_t off[kMaxExperts + 2];
+    int32_t mtp[kMaxExperts + 1];
+};
+
+struct Sched {
+    int E, nb_r, nb_s, mt_s;
+    int64_t routed_tiles, total;
+};
+
+struct TileInfo {
+    bool shared;
+    int g, e;      // group, expert coordinate of the weight maps
+    int arow;      // first row in the A tensor (grouped rows, or token for shared)
+    int64_t row0;  // first row in grouped-row numbering (shared: offsets[E] + token)
+    int rows, n0, N, K;
+};
+
+__device__ __forceinline__ void decode_tile(int64_t t, const Tables& tb, const Sched& sc,
+                                            const GemmArgs& a, int BN, TileInfo& ti) {
+    if (t < sc.routed_tiles) {
+        const int q = (int)(t / sc.nb_r);
+        int lo = 0, hi = sc.E - 1;  // largest g with mtp[g] <= q
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (tb.mtp[mid] <= q)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int g = lo;
+        const int mt = tb.mtp[g + 1] - tb.mtp[g];
+        const int64_t local = t - (int64_t)tb.mtp[g] * sc.nb_r;
+        const int nbi = (int)(local / mt), mb = (int)(local % mt);
+        ti.shared = false;
+        ti.g = ti.e = g;
+        ti.row0 = tb.off[g] + (int64_t)mb * kBM;
+        ti.arow = (int)ti.row0;
+        const int64_t left = tb.off[g + 1] - ti.row0;
+        ti.rows = left < kBM ? (int)left : kBM;
+        ti.n0 = nbi * BN;
+        ti.N = a.N;
+        ti.K = a.K;
+    } else {
+        const int64_t local = t - sc.routed_tiles;
+        const int nbi = (int)(local / sc.mt_s), mb = (int)(local % sc.mt_s);
+        ti.shared = true;
+        ti.g = sc.E;
+        ti.e = 0;
+        ti.arow = mb * kBM;
+        ti.row0 = tb.off[sc.E] + ti.arow;
+        ti.rows = min(kBM, a.T - ti.arow);
+        ti.n0 = nbi * BN;
+        ti.N = a.Ns;
+        ti.K = a.Ks;
+    }
+}
+
+// Bounded wait that also gives up once another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int32_t* flags) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicOr(flags, MOE_DEVFLAG_WAIT_TIMEOUT);
+    return false;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+    const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+    const __grid_constant__ CUtensorMap tmBs0, const __grid_constant__ CUtensorMap tmBs1,
+    const GemmArgs a) {
+    constexpr int BN = kGateUp ? kBRows / 2 : kBRows;  // output columns per tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* tfull = empty + kStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;  // MMA completion before TMEM is freed
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    Tables* tb = reinterpret_cast<Tables*>(smem + kStages * kStageBytes + 256);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int i = threadIdx.x; i < a.E + 2; i += kThreads) tb->off[i] = a.offsets[i];
+    for (int i = threadIdx.x; i < a.E + 1; i += kThreads) tb->mtp[i] = a.mtile_prefix[i];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], kEpiThreads);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmB0);
+        if (kGateUp) tma_prefetch_map(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    Sched sc;
+    sc.E = a.E;
+    sc.nb_r = (a.N + BN - 1) / BN;
+    sc.nb_s = a.has_shared ? (a.Ns + BN - 1) / BN : 0;
+    sc.mt_s = a.has_shared ? (a.T + kBM - 1) / kBM : 0;
+    sc.routed_tiles = (int64_t)tb->mtp[a.E] * sc.nb_r;
+    sc.total = sc.routed_tiles + (int64_t)sc.mt_s * sc.nb_s;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+                TileInfo ti;
+                decode_tile(t, *tb, sc, a, BN, ti);
+                const CUtensorMap* mA = ti.shared ? &tmAs : &tmA;
+                const CUtensorMap* mB0 = ti.shared ? &tmBs0 : &tmB0;
+                const CUtensorMap* mB1 = ti.shared ? &tmBs1 : &tmB1;
+                const int nkb = (ti.K + kBK - 1) / kBK;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, a.flags)) break;
+                    uint8_t* sa = smem + s * kStageBytes;
+                    uint8_t* sb = sa + kABytes;
+                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    // every map is rank 3 (activations have depth 1): the load's
+                    // dimensionality must match the map's rank
+                    tma_load_3d(sa, mA, &full[s], kb * kBK, ti.arow, 0);
+                    if (kGateUp) {
+                        tma_load_3d(sb, mB0, &full[s], kb * kBK, ti.n0, ti.e);
+                        tma_load_3d(sb + kBBytes / 2, mB1, &full[s], kb * kBK, ti.n0, ti.e);
+                    } else {
+                        tma_load_3d(sb, mB0, &full[s], kb * kBK, ti.n0, ti.e);
+                    }
+                }
+            }
+            // Never leave with copies in flight: wait (bounded) for the last
+            // stages issued.  In a normal run these phases completed already.
+            for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0); j < it; ++j)
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&full[j % kStages], (j / kStages) & 1); ++i) {
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            for (int64_t t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x, ++tc) {
+                TileInfo ti;
+                decode_tile(t, *tb, sc, a, BN, ti);
+                const int nkb = (ti.K + kBK - 1) / kBK;
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!wait_or_abort(&tempty[acc], aph ^ 1, abort_flag, a.flags)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * kAccCols;
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!wait_or_abort(&full[s], ph, abort_flag, a.flags)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + s * kStageBytes);
+                    const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_bf16(d, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), kIdesc,
+                                 (kb | kk) != 0);
+                    mma_commit(&empty[s]);  // frees the stage once these MMAs finish
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);  // accumulator ready for the epilogue
+            }
+            // every MMA issued has finished before TMEM can be freed
+            mma_commit(drain);
+            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(drain, 0); ++i) {
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue warps 2..5
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int r = q * 32 + lane;
+        uint32_t tc = 0;
+        for (int64_t t = blockIdx.x; t < sc.total; t += gridDim.x, ++tc) {
+            TileInfo ti;
+            decode_tile(t, *tb, sc, a, BN, ti);
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
+            tc_fence_after();
+            const bool valid = r < ti.rows;
+            const uint32_t tq = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
+            if (kGateUp) {
+                bf16* dst = ti.shared ? a.hs + (int64_t)(ti.arow + r) * a.Ns
+                                      : a.h + (ti.row0 + r) * (int64_t)a.N;
+#pragma unroll 1
+                for (int j0 = 0; j0 < BN; j0 += 32) {
+                    float g[32], u[32];
+                    tmem_ld32(tq + j0, g);
+                    tmem_ld32(tq + BN + j0, u);
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int n = ti.n0 + j0 + v * 8;
+                            if (n < ti.N) {
+                                uint4 pk;
+                                pk.x = pack_bf16x2(silu_f32(g[v * 8 + 0]) * u[v * 8 + 0], silu_f32(g[v * 8 + 1]) * u[v * 8 + 1]);
+                                pk.y = pack_bf16x2(silu_f32(g[v * 8 + 2]) * u[v * 8 + 2], silu_f32(g[v * 8 + 3]) * u[v * 8 + 3]);
+                                pk.z = pack_bf16x2(silu_f32(g[v * 8 + 4]) * u[v * 8 + 4], silu_f32(g[v * 8 + 5]) * u[v * 8 + 5]);
+                                pk.w = pack_bf16x2(silu_f32(g[v * 8 + 6]) * u[v * 8 + 6], silu_f32(g[v * 8 + 7]) * u[v * 8 + 7]);
+                                *reinterpret_cast<uint4*>(dst + n) = pk;
+                            }
+                        }
+                    }
+                }
+            } else {
+                int64_t orow = 0;
+                float w = 1.f;
+                if (valid) {
+                    if (a.mode == 1) {
+                        if (ti.shared) {
+                            orow = ti.arow + r;
+                        } else {
+                            const int32_t s = a.perm_rows[ti.row0 + r];
+                            orow = s / a.k;
+                            w = a.topk_w[s];
+                        }
+                    } else {
+                        orow = ti.shared ? a.S + ti.arow + r : ti.row0 + r;
+                    }
+                }
+                float* dst = a.out + orow * (int64_t)ti.N;
+#pragma unroll 1
+                for (int j0 = 0; j0 < BN; j0 += 32) {
+                    float v[32];
+                    tmem_ld32(tq + j0, v);
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int n = ti.n0 + j0 + i * 4;
+                            if (n < ti.N) {
+                                float4 f = make_float4(w * v[4 * i], w * v[4 * i + 1], w * v[4 * i + 2], w * v[4 * i + 3]);
+                                if (a.mode == 1)
+                                    atomicAdd(reinterpret_cast<float4*>(dst + n), f);
+                                else
+                                    *reinterpret_cast<float4*>(dst + n) = f;
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor [depth][rows][inner] (inner contiguous), box {64, box_rows, 1}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+              uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {inner, rows, depth};
+    cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    static int count[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+    return count[dev] > 0 ? count[dev] : 148;
+}
+
+constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + 256 + sizeof(Tables);
+
+template <bool kGateUp>
+cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const GemmArgs& args,
+                           cudaStream_t st) {
+    constexpr int BN = kGateUp ? kBRows / 2 : kBRows;
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_sm100_kernel<kGateUp>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int64_t nb_r = (args.N + BN - 1) / BN;
+    const int64_t nb_s = args.has_shared ? (args.Ns + BN - 1) / BN : 0;
+    const int64_t ub = ((p.S + kBM - 1) / kBM + p.E) * nb_r + ((p.T + kBM - 1) / kBM) * nb_s;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), ub));
+    grouped_gemm_sm100_kernel<kGateUp><<<grid, kThreads, kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                         maps[4], maps[5], args);
+    return cudaGetLastError();
+}
+
+GemmArgs base_args(const Plan& p) {
+    GemmArgs a{};
+    a.offsets = p.offsets;
+    a.mtile_prefix = p.mtile_prefix;
+    a.flags = p.flags;
+    a.E = (int)p.E;
+    a.T = (int)p.T;
+    a.has_shared = p.Is > 0;
+    a.k = (int)p.k;
+    a.S = p.S;
+    return a;
+}
+
+}  // namespace
+
+cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate, const void* w_up,
+                                const void* ws_gate, const void* ws_up, cudaStream_t st) {
+    if (p.T == 0) return cudaSuccess;
+    bf16* h = (bf16*)p.h;
+    bf16* hs = h + p.S * p.I;
+    CUtensorMap m[6];
+    bool ok = make_map(&m[0], p.xperm, p.H, p.S, 1, kBM) &&
+              make_map(&m[2], w_gate, p.H, p.I, p.E, kBRows / 2) &&
+              make_map(&m[3], w_up, p.H, p.I, p.E, kBRows / 2);
+    if (ok && p.Is > 0)
+        ok = make_map(&m[1], x, p.H, p.T, 1, kBM) && make_map(&m[4], ws_gate, p.H, p.Is, 1, kBRows / 2) &&
+             make_map(&m[5], ws_up, p.H, p.Is, 1, kBRows / 2);
+    else {
+        m[1] = m[0];
+        m[4] = m[2];
+        m[5] = m[3];
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    GemmArgs a = base_args(p);
+    a.N = (int)p.I;
+    a.Ns = (int)p.Is;
+    a.K = a.Ks = (int)p.H;
+    a.h = h;
+    a.hs = hs;
+    trace_before("gateup_sm100", st);
+    cudaError_t e = launch_grouped<true>(p, m, a, st);
+    trace_after(st);
+    return e;
+}
+
+cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_down, int mode, float* out,
+                              cudaStream_t st) {
+    if (p.T == 0) return cudaSuccess;
+    const bf16* h = (const bf16*)p.h;
+    const bf16* hs = h + p.S * p.I;
+    CUtensorMap m[6];
+    bool ok = make_map(&m[0], h, p.I, p.S, 1, kBM) && make_map(&m[2], w_down, p.I, p.H, p.E, kBRows);
+    if (ok && p.Is > 0)
+        ok = make_map(&m[1], hs, p.Is, p.T, 1, kBM) && make_map(&m[4], ws_down, p.Is, p.H, 1, kBRows);
+    else {
+        m[1] = m[0];
+        m[4] = m[2];
+    }
+    m[3] = m[2];
+    m[5] = m[4];
+    if (!ok) return cudaErrorInvalidValue;
+    GemmArgs a = base_args(p);
+    a.N = a.Ns = (int)p.H;
+    a.K = (int)p.I;
+    a.Ks = (int)p.Is;
+    a.perm_rows = p.perm_rows;
+    a.topk_w = p.topk_w;
+    a.out = out;
+    a.mode = mode;
+    trace_before(mode ? "down_sm100_combine" : "down_sm100", st);
+    cudaError_t e = launch_grouped<false>(p, m, a, st);
+    trace_after(st);
+    return e;
+}
+
+}  // namespace moe

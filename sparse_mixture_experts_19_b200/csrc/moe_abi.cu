@@ -107,6 +107,7 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->counts = (int32_t*)take(sizeof(int32_t) * p->E);
     p->dropped = (int32_t*)take(sizeof(int32_t) * p->E);
     p->offsets = (int32_t*)take(sizeof(int32_t) * (p->E + 2));
+    p->mtile_prefix = (int32_t*)take(sizeof(int32_t) * (p->E + 1));
     p->perm_rows = (int32_t*)take(sizeof(int32_t) * p->S);
     p->row_of = (int32_t*)take(sizeof(int32_t) * p->S);
     p->xperm = take(elt * p->S * p->H);
@@ -160,10 +161,17 @@ static moe_status_t run_ffn(const Plan& p, const void* x, const void* w_gate, co
                             const void* w_down, const void* ws_gate, const void* ws_up,
                             const void* ws_down, int mode, float* out, cudaStream_t st) {
     CUDA_TRY(launch_gather_rows(p, x, p.perm_rows, p.offsets, p.xperm, st), "gather_rows");
-    CUDA_TRY(launch_gateup_simt(p, p.xperm, x, p.offsets, w_gate, w_up, ws_gate, ws_up, p.h, st),
-             "gateup");
-    CUDA_TRY(launch_down_simt(p, p.h, p.offsets, p.perm_rows, p.topk_w, w_down, ws_down, mode, out, st),
-             "down");
+    if (p.bf16) {
+        // bf16: tensor cores (tcgen05 + TMEM + TMA)
+        CUDA_TRY(launch_gateup_sm100(p, x, w_gate, w_up, ws_gate, ws_up, st), "gateup");
+        CUDA_TRY(launch_down_sm100(p, w_down, ws_down, mode, out, st), "down");
+    } else {
+        // float32: exact float32 FMAs on CUDA cores (tensor cores would round the inputs)
+        CUDA_TRY(launch_gateup_simt(p, p.xperm, x, p.offsets, w_gate, w_up, ws_gate, ws_up, p.h, st),
+                 "gateup");
+        CUDA_TRY(launch_down_simt(p, p.h, p.offsets, p.perm_rows, p.topk_w, w_down, ws_down, mode, out, st),
+                 "down");
+    }
     return MOE_OK;
 }
 

@@ -46,10 +46,38 @@ __global__ void __launch_bounds__(kHistThreads) permute_hist_kernel(
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = h[e];
 }
 
+// Inclusive scan over the 256 threads of the block (v of thread i -> sum of 0..i).
+// Starts with a barrier: callers may still be reading `sm` from earlier work.
+__device__ __forceinline__ int32_t block_scan_256(int32_t v, int32_t* sm) {
+    const int i = threadIdx.x;
+    __syncthreads();
+    sm[i] = v;
+    __syncthreads();
+    for (int o = 1; o < kScanThreads; o <<= 1) {
+        int32_t u = (i >= o) ? sm[i - o] : 0;
+        __syncthreads();
+        sm[i] += u;
+        __syncthreads();
+    }
+    int32_t r = sm[i];
+    __syncthreads();
+    return r;
+}
+
+// m-tiles of kGemmTileRows rows per expert -> exclusive prefix mtile_prefix[0..E].
+__device__ __forceinline__ void write_mtile_prefix(int32_t kept, int E, int32_t* sm,
+                                                   int32_t* mtile_prefix) {
+    const int e = threadIdx.x;
+    int32_t mt = (e < E) ? (kept + kGemmTileRows - 1) / kGemmTileRows : 0;
+    int32_t incl = block_scan_256(mt, sm);
+    if (e < E) mtile_prefix[e] = incl - mt;
+    if (e == E - 1) mtile_prefix[E] = incl;
+}
+
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(
     int32_t* __restrict__ hist, int64_t nchunks, int E, int64_t cap, int32_t* __restrict__ counts,
     int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
-    int32_t shared_rows) {
+    int32_t* __restrict__ mtile_prefix, int32_t shared_rows) {
     __shared__ int32_t kept_s[kScanThreads];
     const int e = threadIdx.x;
     int32_t total = 0;
@@ -86,6 +114,7 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(
         offsets_ws[E + 1] = R + shared_rows;
         offsets_out[E] = R;
     }
+    write_mtile_prefix(e < E ? kept : 0, E, kept_s, mtile_prefix);
 }
 
 __global__ void __launch_bounds__(kScatterWarps * 32) permute_scatter_kernel(
@@ -133,18 +162,23 @@ __global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_
         perm_rows[r] = -1;
 }
 
-__global__ void offsets_from_user_kernel(const int32_t* __restrict__ user, int E,
-                                         int32_t shared_rows, int32_t* __restrict__ ws_off) {
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) ws_off[e] = user[e];
-    if (threadIdx.x == 0) ws_off[E + 1] = user[E] + shared_rows;
+__global__ void __launch_bounds__(kScanThreads) offsets_from_user_kernel(
+    const int32_t* __restrict__ user, int E, int32_t shared_rows, int32_t* __restrict__ ws_off,
+    int32_t* __restrict__ mtile_prefix) {
+    __shared__ int32_t sm[kScanThreads];
+    const int e = threadIdx.x;
+    if (e <= E) ws_off[e] = user[e];
+    if (e == 0) ws_off[E + 1] = user[E] + shared_rows;
+    write_mtile_prefix(e < E ? user[e + 1] - user[e] : 0, E, sm, mtile_prefix);
 }
 
 }  // namespace
 
 cudaError_t launch_offsets_from_user(const Plan& p, const int32_t* offsets, cudaStream_t st) {
     trace_before("offsets_from_user", st);
-    offsets_from_user_kernel<<<1, 256, 0, st>>>(offsets, (int)p.E, (int32_t)(p.Is > 0 ? p.T : 0),
-                                                p.offsets);
+    offsets_from_user_kernel<<<1, kScanThreads, 0, st>>>(offsets, (int)p.E,
+                                                         (int32_t)(p.Is > 0 ? p.T : 0), p.offsets,
+                                                         p.mtile_prefix);
     trace_after(st);
     return cudaGetLastError();
 }
@@ -163,6 +197,7 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
             // offsets[E+1] = shared rows (T = 0 here, so also 0)
             e1 = cudaMemsetAsync(p.offsets + p.E, 0, sizeof(int32_t) * 2, st);
         }
+        if (e1 == cudaSuccess) e1 = cudaMemsetAsync(p.mtile_prefix, 0, sizeof(int32_t) * (p.E + 1), st);
         return e1;
     }
     const int E = (int)p.E;
@@ -172,7 +207,7 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
     trace_after(st);
     trace_before("permute_scan", st);
     permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
-        p.chunk_base, p.nchunks, E, p.cap, counts, dropped, offsets, p.offsets,
+        p.chunk_base, p.nchunks, E, p.cap, counts, dropped, offsets, p.offsets, p.mtile_prefix,
         (int32_t)(p.Is > 0 ? p.T : 0));
     trace_after(st);
     trace_before("permute_scatter", st);
@@ -237,6 +272,7 @@ cudaError_t launch_permute_noalloc(const Plan& sizes, const int32_t* topk_idx, i
     Plan p = sizes;
     p.chunk_base = scratch;                                 // [kNoAllocChunks * E]
     p.offsets = scratch + kNoAllocChunks * kMaxExperts;     // [E + 2]
+    p.mtile_prefix = p.offsets + (kMaxExperts + 2);         // [E + 1]
     p.flags = p.offsets + 2 * (kMaxExperts + 2);            // flag word, cleared per call
     e = cudaMemsetAsync(p.flags, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return e;
