@@ -58,6 +58,12 @@ __device__ __forceinline__ void set_flag(int32_t* flags, int32_t bit) { atomicOr
 cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_w,
                                const float* router_b, int32_t* topk_idx, float* topk_w,
                                float* yacc_zero, cudaStream_t st);
+// tcgen05 router for the bf16 layer (scores in float32 TMEM accumulators).
+cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router_w,
+                                const float* router_b, int32_t* topk_idx, float* topk_w,
+                                cudaStream_t st);
+// dst[0..n) = 0 (float32, n a multiple of 4).
+cudaError_t launch_zero_f32(float* dst, int64_t n, cudaStream_t st);
 cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
                            int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
                            int32_t* dropped, cudaStream_t st);

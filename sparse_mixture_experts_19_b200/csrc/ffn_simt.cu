@@ -157,6 +157,12 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* _
     }
 }
 
+__global__ void zero_f32_kernel(float4* __restrict__ dst, int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 template <typename TOut>
 __global__ void finalize_kernel(const float4* __restrict__ yacc, TOut* __restrict__ y, int64_t n4) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
@@ -254,6 +260,15 @@ cudaError_t launch_down_simt(const Plan& p, const void* h, const int32_t* offset
             p.S, p.T, (int)p.E, (int)p.k, (int)p.H, (int)p.I, (int)p.Is, offsets, (const float*)h,
             (const float*)hs, (const float*)w_down, nullptr, (const float*)ws_down, nullptr,
             nullptr, nullptr, perm_rows, topk_w, mode, out);
+    trace_after(st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_zero_f32(float* dst, int64_t n, cudaStream_t st) {
+    const int64_t n4 = n / 4;
+    if (n4 == 0) return cudaSuccess;
+    trace_before("zero_acc", st);
+    zero_f32_kernel<<<grid_for(n4, 256), 256, 0, st>>>((float4*)dst, n4);
     trace_after(st);
     return cudaGetLastError();
 }

@@ -27,13 +27,11 @@
 // the main loop of the next), warps 2-5 drain TMEM (one 32-lane quadrant
 // each).  Every wait is bounded; a timeout sets MOE_DEVFLAG_WAIT_TIMEOUT and
 // the CTA unwinds and frees its TMEM.
-#include <cudaTypedefs.h>
-
 #include <algorithm>
-#include <mutex>
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tma_host.cuh"
 
 namespace moe {
 namespace {
@@ -126,18 +124,6 @@ __device__ __forceinline__ void decode_tile(int64_t t, const Tables& tb, const S
         ti.N = a.Ns;
         ti.K = a.Ks;
     }
-}
-
-// Bounded wait that also gives up once another role has aborted.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              int32_t* flags) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-    }
-    *abort_flag = 1;
-    atomicOr(flags, MOE_DEVFLAG_WAIT_TIMEOUT);
-    return false;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -357,42 +343,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// bf16 tensor [depth][rows][inner] (inner contiguous), box {64, box_rows, 1}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
-              uint32_t box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {inner, rows, depth};
-    cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
-    cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-    static int count[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
-    return count[dev] > 0 ? count[dev] : 148;
-}
-
 constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + 256 + sizeof(Tables);
 
 template <bool kGateUp>
@@ -405,7 +355,7 @@ cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const Ge
     const int64_t nb_r = (args.N + BN - 1) / BN;
     const int64_t nb_s = args.has_shared ? (args.Ns + BN - 1) / BN : 0;
     const int64_t ub = ((p.S + kBM - 1) / kBM + p.E) * nb_r + ((p.T + kBM - 1) / kBM) * nb_s;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), ub));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), ub));
     grouped_gemm_sm100_kernel<kGateUp><<<grid, kThreads, kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3],
                                                                          maps[4], maps[5], args);
     return cudaGetLastError();
@@ -432,12 +382,12 @@ cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate
     bf16* h = (bf16*)p.h;
     bf16* hs = h + p.S * p.I;
     CUtensorMap m[6];
-    bool ok = make_map(&m[0], p.xperm, p.H, p.S, 1, kBM) &&
-              make_map(&m[2], w_gate, p.H, p.I, p.E, kBRows / 2) &&
-              make_map(&m[3], w_up, p.H, p.I, p.E, kBRows / 2);
+    bool ok = make_map_bf16(&m[0], p.xperm, p.H, p.S, 1, kBK, kBM) &&
+              make_map_bf16(&m[2], w_gate, p.H, p.I, p.E, kBK, kBRows / 2) &&
+              make_map_bf16(&m[3], w_up, p.H, p.I, p.E, kBK, kBRows / 2);
     if (ok && p.Is > 0)
-        ok = make_map(&m[1], x, p.H, p.T, 1, kBM) && make_map(&m[4], ws_gate, p.H, p.Is, 1, kBRows / 2) &&
-             make_map(&m[5], ws_up, p.H, p.Is, 1, kBRows / 2);
+        ok = make_map_bf16(&m[1], x, p.H, p.T, 1, kBK, kBM) && make_map_bf16(&m[4], ws_gate, p.H, p.Is, 1, kBK, kBRows / 2) &&
+             make_map_bf16(&m[5], ws_up, p.H, p.Is, 1, kBK, kBRows / 2);
     else {
         m[1] = m[0];
         m[4] = m[2];
@@ -462,9 +412,9 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     const bf16* h = (const bf16*)p.h;
     const bf16* hs = h + p.S * p.I;
     CUtensorMap m[6];
-    bool ok = make_map(&m[0], h, p.I, p.S, 1, kBM) && make_map(&m[2], w_down, p.I, p.H, p.E, kBRows);
+    bool ok = make_map_bf16(&m[0], h, p.I, p.S, 1, kBK, kBM) && make_map_bf16(&m[2], w_down, p.I, p.H, p.E, kBK, kBRows);
     if (ok && p.Is > 0)
-        ok = make_map(&m[1], hs, p.Is, p.T, 1, kBM) && make_map(&m[4], ws_down, p.Is, p.H, 1, kBRows);
+        ok = make_map_bf16(&m[1], hs, p.Is, p.T, 1, kBK, kBM) && make_map_bf16(&m[4], ws_down, p.Is, p.H, 1, kBK, kBRows);
     else {
         m[1] = m[0];
         m[4] = m[2];

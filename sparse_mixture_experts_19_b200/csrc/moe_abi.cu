@@ -206,7 +206,10 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* route
     REQUIRE_PTR(topk_idx);
     REQUIRE_PTR(topk_w);
     cudaStream_t st = (cudaStream_t)stream;
-    CUDA_TRY(launch_router_simt(p, x, router_w, router_b, topk_idx, topk_w, nullptr, st), "router");
+    if (p.bf16)
+        CUDA_TRY(launch_router_sm100(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
+    else
+        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, topk_idx, topk_w, nullptr, st), "router");
     return MOE_OK;
 }
 
@@ -324,7 +327,13 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
     int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
-    CUDA_TRY(launch_router_simt(p, x, router_w, router_b, idx, p.topk_w, p.yacc, st), "router");
+    if (p.bf16) {
+        CUDA_TRY(launch_zero_f32(p.yacc, p.T * p.H, st), "zero");
+        CUDA_TRY(launch_router_sm100(p, x, router_w, router_b, idx, p.topk_w, st), "router");
+    } else {
+        // the float32 router also zeroes the combine accumulator rows
+        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, idx, p.topk_w, p.yacc, st), "router");
+    }
     CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
     if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.yacc, st)) != MOE_OK)
         return s;

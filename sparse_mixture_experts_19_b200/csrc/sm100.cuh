@@ -60,6 +60,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     return false;
 }
 
+// Bounded wait shared by the roles of one CTA: gives up when another role
+// has set *abort_flag, or after kWaitLimit polls, in which case it sets
+// *abort_flag and the device flag `timeout_bit` in *flags.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int32_t* flags, int32_t timeout_bit = 0x2) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicOr(flags, timeout_bit);
+    return false;
+}
+
+// Unbounded-by-abort but still bounded wait used to drain in-flight work.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar, parity); ++i) {
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
