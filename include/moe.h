@@ -192,12 +192,13 @@ moe_status_t moe_combine(const moe_config_t* cfg, const float* expert_out, const
  * moe_forward -- the whole layer, the C form of the pages' moe_forward(x,
  * experts, router, top_k) ("MoE稀疏架构是什么？…", section 四): route,
  * group, grouped gate/up GEMM with the SwiGLU fused in its epilogue, grouped
- * down GEMM with the routing-weight scale and the scatter-add fused in its
- * epilogue, then one cast to the layer dtype.
+ * down GEMM with the routing-weight scale fused in its epilogue (each kept
+ * row's w * FFN_e(x) stored in the layer dtype), then the un-permute: each
+ * token's rows summed in float32 in slot order (then the shared row) and
+ * rounded once to the layer dtype.
  *   y [T,H] (layer dtype).  Optional outputs (NULL to skip): topk_idx_out
  *   [T,top_k] int32, counts_out [E] and dropped_out [E] int32.
- * The summation order of the up to top_k + 1 terms of a y element is not
- * fixed (float32 atomics), so y may differ between runs in the last bits.
+ * y is bit-reproducible for given inputs (no atomics, fixed summation order).
  */
 moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* router_w,
                          const float* router_b, const void* w_gate, const void* w_up,

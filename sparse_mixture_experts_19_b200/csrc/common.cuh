@@ -38,8 +38,8 @@ struct Plan {
     int32_t* perm_rows;   // [S]
     int32_t* row_of;      // [S]
     void* xperm;          // [S, H] layer dtype: x rows in grouped order
-    void* h;              // [h_rows, I_max] layer dtype: SwiGLU activations
-    float* yacc;          // [T, H] float32 accumulator of the combine
+    void* h;              // [S, I] + [T, Is] layer dtype: SwiGLU activations
+    void* rows;           // [S + T, H] layer dtype: routing-weighted expert output rows
     size_t bytes;         // total workspace bytes
 };
 
@@ -55,15 +55,15 @@ __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-
 __device__ __forceinline__ void set_flag(int32_t* flags, int32_t bit) { atomicOr(flags, bit); }
 
 // ---- launchers (defined in the .cu files; return the launch error) ------
+// Router for the float32 layer (CUDA cores, float32 FMAs).
 cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_w,
                                const float* router_b, int32_t* topk_idx, float* topk_w,
-                               float* yacc_zero, cudaStream_t st);
-// tcgen05 router for the bf16 layer (scores in float32 TMEM accumulators).
+                               cudaStream_t st);
+// Router for the bf16 layer (tcgen05; float32 TMEM scores, exact fp64
+// rescoring of near-boundary experts).
 cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router_w,
                                 const float* router_b, int32_t* topk_idx, float* topk_w,
                                 cudaStream_t st);
-// dst[0..n) = 0 (float32, n a multiple of 4).
-cudaError_t launch_zero_f32(float* dst, int64_t n, cudaStream_t st);
 cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
                            int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
                            int32_t* dropped, cudaStream_t st);
@@ -75,22 +75,27 @@ cudaError_t launch_permute_noalloc(const Plan& sizes, const int32_t* topk_idx, i
 cudaError_t launch_offsets_from_user(const Plan& p, const int32_t* offsets, cudaStream_t st);
 cudaError_t launch_gather_rows(const Plan& p, const void* x, const int32_t* perm_rows,
                                const int32_t* offsets, void* xperm, cudaStream_t st);
-// h = silu(X W_g^T) * (X W_u^T) for all groups (routed + shared).
+// Grouped expert GEMMs for all groups (routed + shared):
+//   gate/up: h = silu(X W_g^T) * (X W_u^T), rounded to the layer dtype;
+//   down:    mode 0 stores unweighted float32 rows h W_d^T to `out` [S + T, H];
+//            mode 1 stores topk_w-weighted rows in the layer dtype to `out`
+//            (shared rows with weight 1).
+// float32 layer: CUDA cores (exact FMAs); bf16 layer: tcgen05 + TMEM + TMA.
 cudaError_t launch_gateup_simt(const Plan& p, const void* xperm, const void* x,
                                const int32_t* offsets, const void* w_gate, const void* w_up,
                                const void* ws_gate, const void* ws_up, void* h, cudaStream_t st);
-// out = h W_d^T: mode 0 stores float32 rows to `out`; mode 1 adds
-// topk_w-weighted rows into yacc[token] (shared rows with weight 1).
 cudaError_t launch_down_simt(const Plan& p, const void* h, const int32_t* offsets,
                              const int32_t* perm_rows, const float* topk_w, const void* w_down,
-                             const void* ws_down, int mode, float* out, cudaStream_t st);
-// tcgen05 grouped GEMMs (bf16): h = silu(X W_g^T) * (X W_u^T); out = h W_d^T
-// (mode 0: float32 rows; mode 1: weighted atomic add into yacc[token]).
+                             const void* ws_down, int mode, void* out, cudaStream_t st);
 cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate, const void* w_up,
                                 const void* ws_gate, const void* ws_up, cudaStream_t st);
 cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_down, int mode,
-                              float* out, cudaStream_t st);
-cudaError_t launch_finalize(const Plan& p, const float* yacc, void* y, cudaStream_t st);
+                              void* out, cudaStream_t st);
+// y[t] = sum_j rows[row_of[t,j]] (j in order, dropped slots skipped) + rows[S + t]
+// (shared), summed in float32 and rounded once to the layer dtype.
+cudaError_t launch_combine_rows(const Plan& p, const void* rows, const int32_t* row_of, void* y,
+                                cudaStream_t st);
+// Stage API: y[t] = sum_j topk_w[t,j] * expert_out[row_of[t,j]] (+ shared row).
 cudaError_t launch_combine(const Plan& p, const float* expert_out, const int32_t* row_of,
                            const float* topk_w, void* y, cudaStream_t st);
 

@@ -7,7 +7,8 @@
 // "MoE稀疏架构是什么？从原理到落地的系统解读", section 四 (weighted sum of the
 // chosen experts' outputs).
 //
-// The GEMMs here serve the float32 layer (exact float32 FMAs, no TF32).
+// The GEMMs here serve the float32 layer (exact float32 FMAs, no TF32); the
+// gather and the combines serve both dtypes.
 // Groups: 0..E-1 are the routed experts, rows offsets[g]..offsets[g+1];
 // group E is the shared expert (rows offsets[E]..offsets[E+1], i.e. token
 // t = row - offsets[E], reading x directly).
@@ -43,7 +44,7 @@ __global__ void __launch_bounds__(kThreads) grouped_ffn_simt_kernel(
     const TIn* __restrict__ ws0, const TIn* __restrict__ ws1,  // shared expert weights
     TIn* __restrict__ h_out, TIn* __restrict__ hs_out,         // gate/up outputs
     const int32_t* __restrict__ perm_rows, const float* __restrict__ topk_w, int mode,
-    float* __restrict__ out) {
+    void* __restrict__ out) {
     __shared__ int32_t off[kMaxExperts + 2];
     __shared__ __align__(16) float As[kBK][kBM];
     __shared__ __align__(16) float Bs[kGateUp ? 2 : 1][kBK][kBN];
@@ -114,29 +115,24 @@ __global__ void __launch_bounds__(kThreads) grouped_ffn_simt_kernel(
                 int n = n0 + tx * 4 + j;
                 if (n < N) dst[n] = from_f32<TIn>(silu_f32(acc0[i][j]) * acc1[i][j]);
             }
-        } else if (mode == 0) {
-            float* dst = out + (shared ? S + (row - off[E]) : row) * (int64_t)H;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                int n = n0 + tx * 4 + j;
-                if (n < N) dst[n] = acc0[i][j];
-            }
         } else {
-            int64_t tok;
-            float w;
-            if (shared) {
-                tok = row - off[E];
-                w = 1.f;
-            } else {
-                int32_t s = perm_rows[row];
-                tok = s / k;
-                w = topk_w[s];
-            }
-            float* dst = out + tok * (int64_t)H;
+            // output row: grouped row, or S + token for the shared expert
+            const int64_t orow = shared ? S + (row - off[E]) : row;
+            if (mode == 0) {
+                float* dst = static_cast<float*>(out) + orow * (int64_t)H;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                int n = n0 + tx * 4 + j;
-                if (n < N) atomicAdd(dst + n, w * acc0[i][j]);
+                for (int j = 0; j < 4; ++j) {
+                    int n = n0 + tx * 4 + j;
+                    if (n < N) dst[n] = acc0[i][j];
+                }
+            } else {
+                const float w = shared ? 1.f : topk_w[perm_rows[row]];
+                TIn* dst = static_cast<TIn*>(out) + orow * (int64_t)H;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    int n = n0 + tx * 4 + j;
+                    if (n < N) dst[n] = from_f32<TIn>(w * acc0[i][j]);
+                }
             }
         }
     }
@@ -157,22 +153,37 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* _
     }
 }
 
-__global__ void zero_f32_kernel(float4* __restrict__ dst, int64_t n4) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
-         i += (int64_t)gridDim.x * blockDim.x)
-        dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-template <typename TOut>
-__global__ void finalize_kernel(const float4* __restrict__ yacc, TOut* __restrict__ y, int64_t n4) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+// y[t] = sum_j rows[row_of[t,j]] (+ rows[S + t]); one thread per 16-byte chunk
+// of a token's row, float32 sum in slot order, one rounding at the end.
+template <typename TV>
+__global__ void combine_rows_kernel(const TV* __restrict__ rows, const int32_t* __restrict__ row_of,
+                                    int64_t T, int H, int k, int64_t S, int shared, TV* __restrict__ y) {
+    constexpr int V = 16 / sizeof(TV);
+    const int chunks = H / V;
+    const int64_t n = T * chunks;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
-        float4 v = yacc[i];
-        TOut* d = y + i * 4;
-        d[0] = from_f32<TOut>(v.x);
-        d[1] = from_f32<TOut>(v.y);
-        d[2] = from_f32<TOut>(v.z);
-        d[3] = from_f32<TOut>(v.w);
+        const int64_t t = i / chunks;
+        const int c = (int)(i % chunks);
+        float acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.f;
+        auto add_row = [&](int64_t r) {
+            uint4 q = *reinterpret_cast<const uint4*>(rows + r * H + (int64_t)c * V);
+            const TV* e = reinterpret_cast<const TV*>(&q);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] += to_f32(e[v]);
+        };
+        for (int j = 0; j < k; ++j) {
+            const int32_t r = row_of[t * k + j];
+            if (r >= 0) add_row(r);
+        }
+        if (shared) add_row(S + t);
+        uint4 o;
+        TV* ov = reinterpret_cast<TV*>(&o);
+#pragma unroll
+        for (int v = 0; v < V; ++v) ov[v] = from_f32<TV>(acc[v]);
+        *reinterpret_cast<uint4*>(y + t * H + (int64_t)c * V) = o;
     }
 }
 
@@ -225,62 +236,42 @@ cudaError_t launch_gateup_simt(const Plan& p, const void* xperm, const void* x,
                                const void* ws_gate, const void* ws_up, void* h, cudaStream_t st) {
     if (p.T == 0) return cudaSuccess;
     dim3 grid = ffn_grid(p, p.I_max);
-    void* hs = (char*)h + p.S * p.I * (p.bf16 ? 2 : 4);
+    void* hs = (float*)h + p.S * p.I;
     trace_before("gateup_simt", st);
-    if (p.bf16)
-        grouped_ffn_simt_kernel<bf16, true><<<grid, kThreads, 0, st>>>(
-            p.S, p.T, (int)p.E, (int)p.k, (int)p.H, (int)p.I, (int)p.Is, offsets,
-            (const bf16*)xperm, (const bf16*)x, (const bf16*)w_gate, (const bf16*)w_up,
-            (const bf16*)ws_gate, (const bf16*)ws_up, (bf16*)h, (bf16*)hs, nullptr, nullptr, 0,
-            nullptr);
-    else
-        grouped_ffn_simt_kernel<float, true><<<grid, kThreads, 0, st>>>(
-            p.S, p.T, (int)p.E, (int)p.k, (int)p.H, (int)p.I, (int)p.Is, offsets,
-            (const float*)xperm, (const float*)x, (const float*)w_gate, (const float*)w_up,
-            (const float*)ws_gate, (const float*)ws_up, (float*)h, (float*)hs, nullptr, nullptr, 0,
-            nullptr);
+    grouped_ffn_simt_kernel<float, true><<<grid, kThreads, 0, st>>>(
+        p.S, p.T, (int)p.E, (int)p.k, (int)p.H, (int)p.I, (int)p.Is, offsets, (const float*)xperm,
+        (const float*)x, (const float*)w_gate, (const float*)w_up, (const float*)ws_gate,
+        (const float*)ws_up, (float*)h, (float*)hs, nullptr, nullptr, 0, nullptr);
     trace_after(st);
     return cudaGetLastError();
 }
 
 cudaError_t launch_down_simt(const Plan& p, const void* h, const int32_t* offsets,
                              const int32_t* perm_rows, const float* topk_w, const void* w_down,
-                             const void* ws_down, int mode, float* out, cudaStream_t st) {
+                             const void* ws_down, int mode, void* out, cudaStream_t st) {
     if (p.T == 0) return cudaSuccess;
     dim3 grid = ffn_grid(p, p.H);
-    const void* hs = (const char*)h + p.S * p.I * (p.bf16 ? 2 : 4);
-    trace_before(mode ? "down_simt_combine" : "down_simt", st);
-    if (p.bf16)
-        grouped_ffn_simt_kernel<bf16, false><<<grid, kThreads, 0, st>>>(
-            p.S, p.T, (int)p.E, (int)p.k, (int)p.H, (int)p.I, (int)p.Is, offsets, (const bf16*)h,
-            (const bf16*)hs, (const bf16*)w_down, nullptr, (const bf16*)ws_down, nullptr, nullptr,
-            nullptr, perm_rows, topk_w, mode, out);
-    else
-        grouped_ffn_simt_kernel<float, false><<<grid, kThreads, 0, st>>>(
-            p.S, p.T, (int)p.E, (int)p.k, (int)p.H, (int)p.I, (int)p.Is, offsets, (const float*)h,
-            (const float*)hs, (const float*)w_down, nullptr, (const float*)ws_down, nullptr,
-            nullptr, nullptr, perm_rows, topk_w, mode, out);
+    const void* hs = (const float*)h + p.S * p.I;
+    trace_before(mode ? "down_simt_weighted" : "down_simt", st);
+    grouped_ffn_simt_kernel<float, false><<<grid, kThreads, 0, st>>>(
+        p.S, p.T, (int)p.E, (int)p.k, (int)p.H, (int)p.I, (int)p.Is, offsets, (const float*)h,
+        (const float*)hs, (const float*)w_down, nullptr, (const float*)ws_down, nullptr, nullptr,
+        nullptr, perm_rows, topk_w, mode, out);
     trace_after(st);
     return cudaGetLastError();
 }
 
-cudaError_t launch_zero_f32(float* dst, int64_t n, cudaStream_t st) {
-    const int64_t n4 = n / 4;
-    if (n4 == 0) return cudaSuccess;
-    trace_before("zero_acc", st);
-    zero_f32_kernel<<<grid_for(n4, 256), 256, 0, st>>>((float4*)dst, n4);
-    trace_after(st);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_finalize(const Plan& p, const float* yacc, void* y, cudaStream_t st) {
-    const int64_t n4 = p.T * p.H / 4;
-    if (n4 == 0) return cudaSuccess;
-    trace_before("finalize", st);
+cudaError_t launch_combine_rows(const Plan& p, const void* rows, const int32_t* row_of, void* y,
+                                cudaStream_t st) {
+    const int64_t n = p.T * p.H / (p.bf16 ? 8 : 4);
+    if (n == 0) return cudaSuccess;
+    trace_before("combine_rows", st);
     if (p.bf16)
-        finalize_kernel<bf16><<<grid_for(n4, 256), 256, 0, st>>>((const float4*)yacc, (bf16*)y, n4);
+        combine_rows_kernel<bf16><<<grid_for(n, 256), 256, 0, st>>>(
+            (const bf16*)rows, row_of, p.T, (int)p.H, (int)p.k, p.S, p.Is > 0, (bf16*)y);
     else
-        finalize_kernel<float><<<grid_for(n4, 256), 256, 0, st>>>((const float4*)yacc, (float*)y, n4);
+        combine_rows_kernel<float><<<grid_for(n, 256), 256, 0, st>>>(
+            (const float*)rows, row_of, p.T, (int)p.H, (int)p.k, p.S, p.Is > 0, (float*)y);
     trace_after(st);
     return cudaGetLastError();
 }

@@ -12,8 +12,9 @@
 //             so G and U of a tile land side by side in one TMEM accumulator
 //             and the SwiGLU is applied in the epilogue.
 //   down:     out = h W_d[e]^T; the epilogue multiplies row r by its routing
-//             weight and adds it into the float32 accumulator of its token
-//             (vector atomics), or stores float32 rows (stage API).
+//             weight and stores it in bf16 at its grouped row (the combine
+//             kernel then sums each token's rows), or stores unweighted
+//             float32 rows (stage API).
 //
 // Groups: 0..E-1 routed experts (rows offsets[g]..offsets[g+1] of the
 // grouped activations), group E the shared expert (token rows of x / hs).
@@ -63,7 +64,8 @@ struct GemmArgs {
     const int32_t* perm_rows;  // down: row -> slot
     const float* topk_w;       // down: slot -> routing weight
     int k;
-    float* out;  // down mode 1: yacc [T, N]; mode 0: rows [S + T, N]
+    float* out;  // down mode 0: unweighted float32 rows [S + T, N]
+    bf16* rows;  // down mode 1: routing-weighted bf16 rows [S + T, N]
     int64_t S;
     int mode;
 };
@@ -296,36 +298,37 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
                     }
                 }
             } else {
-                int64_t orow = 0;
+                // output row: grouped row, or S + token for the shared expert
+                const int64_t orow = ti.shared ? a.S + ti.arow + r : ti.row0 + r;
                 float w = 1.f;
-                if (valid) {
-                    if (a.mode == 1) {
-                        if (ti.shared) {
-                            orow = ti.arow + r;
-                        } else {
-                            const int32_t s = a.perm_rows[ti.row0 + r];
-                            orow = s / a.k;
-                            w = a.topk_w[s];
-                        }
-                    } else {
-                        orow = ti.shared ? a.S + ti.arow + r : ti.row0 + r;
-                    }
-                }
-                float* dst = a.out + orow * (int64_t)ti.N;
+                if (valid && a.mode == 1 && !ti.shared) w = a.topk_w[a.perm_rows[ti.row0 + r]];
 #pragma unroll 1
                 for (int j0 = 0; j0 < BN; j0 += 32) {
                     float v[32];
                     tmem_ld32(tq + j0, v);
                     if (valid) {
+                        if (a.mode == 1) {
+                            bf16* dst = a.rows + orow * (int64_t)ti.N;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int n = ti.n0 + j0 + i * 4;
-                            if (n < ti.N) {
-                                float4 f = make_float4(w * v[4 * i], w * v[4 * i + 1], w * v[4 * i + 2], w * v[4 * i + 3]);
-                                if (a.mode == 1)
-                                    atomicAdd(reinterpret_cast<float4*>(dst + n), f);
-                                else
-                                    *reinterpret_cast<float4*>(dst + n) = f;
+                            for (int i = 0; i < 4; ++i) {
+                                const int n = ti.n0 + j0 + i * 8;
+                                if (n < ti.N) {
+                                    uint4 pk;
+                                    pk.x = pack_bf16x2(w * v[i * 8 + 0], w * v[i * 8 + 1]);
+                                    pk.y = pack_bf16x2(w * v[i * 8 + 2], w * v[i * 8 + 3]);
+                                    pk.z = pack_bf16x2(w * v[i * 8 + 4], w * v[i * 8 + 5]);
+                                    pk.w = pack_bf16x2(w * v[i * 8 + 6], w * v[i * 8 + 7]);
+                                    *reinterpret_cast<uint4*>(dst + n) = pk;
+                                }
+                            }
+                        } else {
+                            float* dst = a.out + orow * (int64_t)ti.N;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int n = ti.n0 + j0 + i * 4;
+                                if (n < ti.N)
+                                    *reinterpret_cast<float4*>(dst + n) =
+                                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                             }
                         }
                     }
@@ -406,7 +409,7 @@ cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate
     return e;
 }
 
-cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_down, int mode, float* out,
+cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_down, int mode, void* out,
                               cudaStream_t st) {
     if (p.T == 0) return cudaSuccess;
     const bf16* h = (const bf16*)p.h;
@@ -428,9 +431,10 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     a.Ks = (int)p.Is;
     a.perm_rows = p.perm_rows;
     a.topk_w = p.topk_w;
-    a.out = out;
+    a.out = mode == 0 ? (float*)out : nullptr;
+    a.rows = mode == 1 ? (bf16*)out : nullptr;
     a.mode = mode;
-    trace_before(mode ? "down_sm100_combine" : "down_sm100", st);
+    trace_before(mode ? "down_sm100_weighted" : "down_sm100", st);
     cudaError_t e = launch_grouped<false>(p, m, a, st);
     trace_after(st);
     return e;

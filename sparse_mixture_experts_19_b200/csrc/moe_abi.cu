@@ -112,7 +112,7 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->row_of = (int32_t*)take(sizeof(int32_t) * p->S);
     p->xperm = take(elt * p->S * p->H);
     p->h = take(elt * (p->S * p->I + p->T * p->Is));
-    p->yacc = (float*)take(sizeof(float) * p->T * p->H);
+    p->rows = take(elt * (p->S + (p->Is ? p->T : 0)) * p->H);
     p->bytes = off;
 }
 
@@ -159,7 +159,7 @@ static moe_status_t check_shared(const Plan& p, const void* a, const void* b, co
 // The grouped FFN of moe_forward / moe_grouped_ffn, after routing and grouping.
 static moe_status_t run_ffn(const Plan& p, const void* x, const void* w_gate, const void* w_up,
                             const void* w_down, const void* ws_gate, const void* ws_up,
-                            const void* ws_down, int mode, float* out, cudaStream_t st) {
+                            const void* ws_down, int mode, void* out, cudaStream_t st) {
     CUDA_TRY(launch_gather_rows(p, x, p.perm_rows, p.offsets, p.xperm, st), "gather_rows");
     if (p.bf16) {
         // bf16: tensor cores (tcgen05 + TMEM + TMA)
@@ -209,7 +209,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* route
     if (p.bf16)
         CUDA_TRY(launch_router_sm100(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
     else
-        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, topk_idx, topk_w, nullptr, st), "router");
+        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
     return MOE_OK;
 }
 
@@ -327,17 +327,14 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
     int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
-    if (p.bf16) {
-        CUDA_TRY(launch_zero_f32(p.yacc, p.T * p.H, st), "zero");
+    if (p.bf16)
         CUDA_TRY(launch_router_sm100(p, x, router_w, router_b, idx, p.topk_w, st), "router");
-    } else {
-        // the float32 router also zeroes the combine accumulator rows
-        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, idx, p.topk_w, p.yacc, st), "router");
-    }
+    else
+        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, idx, p.topk_w, st), "router");
     CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
-    if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.yacc, st)) != MOE_OK)
+    if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.rows, st)) != MOE_OK)
         return s;
-    CUDA_TRY(launch_finalize(p, p.yacc, y, st), "finalize");
+    CUDA_TRY(launch_combine_rows(p, p.rows, p.row_of, y, st), "combine_rows");
     return MOE_OK;
 }
 

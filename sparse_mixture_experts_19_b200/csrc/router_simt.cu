@@ -34,8 +34,7 @@ __device__ __forceinline__ void warp_argmax(float& v, int& e) {
 template <typename TIn>
 __global__ void __launch_bounds__(kThreads) router_simt_kernel(
     int T, int H, int E, int k, const TIn* __restrict__ x, const TIn* __restrict__ wr,
-    const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    float* __restrict__ yacc) {
+    const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     __shared__ float xs[kTB][kHC + 1];
     // weights chunk [E][kHC+1] during the scores, then scores [kTB][E+1]
     __shared__ float buf[kMaxExperts * (kHC + 1)];
@@ -120,32 +119,19 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(
             }
         }
     }
-
-    // zero the combine accumulator rows of these tokens
-    if (yacc) {
-        int rows = min(kTB, T - t0);
-        float4* dst = reinterpret_cast<float4*>(yacc + (int64_t)t0 * H);
-        int64_t n4 = (int64_t)rows * H / 4;
-        for (int64_t q = tid; q < n4; q += kThreads) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 }
 
 }  // namespace
 
 cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_w,
                                const float* router_b, int32_t* topk_idx, float* topk_w,
-                               float* yacc_zero, cudaStream_t st) {
+                               cudaStream_t st) {
     if (p.T == 0) return cudaSuccess;
     dim3 grid((unsigned)((p.T + kTB - 1) / kTB));
     trace_before("router_simt", st);
-    if (p.bf16)
-        router_simt_kernel<bf16><<<grid, kThreads, 0, st>>>(
-            (int)p.T, (int)p.H, (int)p.E, (int)p.k, (const bf16*)x, (const bf16*)router_w,
-            router_b, topk_idx, topk_w, yacc_zero);
-    else
-        router_simt_kernel<float><<<grid, kThreads, 0, st>>>(
-            (int)p.T, (int)p.H, (int)p.E, (int)p.k, (const float*)x, (const float*)router_w,
-            router_b, topk_idx, topk_w, yacc_zero);
+    router_simt_kernel<float><<<grid, kThreads, 0, st>>>((int)p.T, (int)p.H, (int)p.E, (int)p.k,
+                                                         (const float*)x, (const float*)router_w,
+                                                         router_b, topk_idx, topk_w);
     trace_after(st);
     return cudaGetLastError();
 }
