@@ -6,13 +6,22 @@
 // softmax over those k).  "模型的“分工的艺术”：MoE技术如何提升计算效率",
 // section 1.1 (the gate is a linear layer, here with an optional bias).
 //
-// One CTA scores 128 tokens against all E experts: the scores are one
-// 128 x E tile of x W_r^T, accumulated in float32 in TMEM (E padded to a
-// multiple of 16; the padding rows of the weight box read as zero).  Warp 0
-// streams x and W_r through a 4-stage TMA ring, warp 1 issues the MMAs,
-// warps 2-5 each own 32 tokens: a thread reads its token's E scores from
-// TMEM, adds the bias, keeps the k best in registers ordered by (score
-// descending, expert index ascending), and writes the softmax of those k.
+// A tile is 128 tokens x all E experts of x W_r^T, accumulated in float32 in
+// TMEM (E padded to a multiple of 16; the padding rows of the weight box
+// read as zero).  Persistent CTAs loop over token tiles: warp 0 streams x and
+// W_r through a TMA ring of up to 8 stages, warp 1 issues the MMAs into one
+// of two TMEM accumulators, warps 2-5 (one token per thread) drain the other
+// one: bias, the k best in registers ordered by (score desc, index asc), and
+// the softmax of those k.  The epilogue of one tile overlaps the loads and
+// MMAs of the next.
+//
+// Exactness of the decision.  Tensor-core float32 sums differ from exact
+// sums by a small accumulation error.  A token whose approximate k-th and
+// (k+1)-th scores are within delta (8x a bound on that error) has the
+// experts of the band [s_k - delta, s_{k+1} + delta] rescored exactly in
+// fp64 (bf16 products are exact) by warp-cooperative dot products, and its
+// selection is completed from those exact scores.  Experts above the band
+// are certainly selected, experts below it certainly not.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
@@ -24,49 +33,51 @@ using namespace sm100;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 8;
 constexpr int kThreads = 192;
 constexpr int kABytes = kBM * kBK * 2;
+constexpr int kQueue = 512;  // exact-rescoring queue entries per CTA and tile
 
 // (a, ea) ranks before (b, eb): larger score, then lower expert index.
 __device__ __forceinline__ bool ranks_before(float a, int ea, float b, int eb) {
     return a > b || (a == b && ea < eb);
 }
 
-constexpr int kQueue = 2048;  // exact-rescoring queue entries per CTA
-
 // Exact score x[t] . W_r[e] in fp64 (products of bf16 values are exact),
-// computed by one warp: lane l takes the 8-element chunks l, l+32, ...
+// computed by one warp: lane l takes the 8-element chunks l, l+32, ...; four
+// chunks per lane are loaded before any is used, into four accumulators.
 __device__ __forceinline__ double exact_score(const bf16* x, const bf16* w, int t, int e, int H, int lane) {
     const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
     const uint4* wr = reinterpret_cast<const uint4*>(w + (int64_t)e * H);
-    double acc = 0.0;
-    for (int c = lane; c < H / 8; c += 32) {
-        uint4 a = xr[c], b = wr[c];
-        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+    const int nch = H / 8;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int c = lane; c < nch; c += 128) {
+        uint4 a[4], b[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float2 fa = __bfloat1622float2(pa[i]), fb = __bfloat1622float2(pb[i]);
-            acc = fma((double)fa.x, (double)fb.x, acc);
-            acc = fma((double)fa.y, (double)fb.y, acc);
+        for (int u = 0; u < 4; ++u) {
+            const int cu = c + 32 * u;
+            a[u] = cu < nch ? xr[cu] : make_uint4(0, 0, 0, 0);
+            b[u] = cu < nch ? wr[cu] : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+            const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float2 fa = __bfloat1622float2(pa[i]), fb = __bfloat1622float2(pb[i]);
+                acc[u] = fma((double)fa.x, (double)fb.x, acc[u]);
+                acc[u] = fma((double)fa.y, (double)fb.y, acc[u]);
+            }
         }
     }
+    double sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    return acc;
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    return sum;
 }
 
-// The same exact score computed by one thread (fallback when the queue is full).
-__device__ __noinline__ double exact_score_serial(const bf16* x, const bf16* w, int t, int e, int H) {
-    double acc = 0.0;
-    for (int h = 0; h < H; ++h)
-        acc = fma((double)__bfloat162float(x[(int64_t)t * H + h]), (double)__bfloat162float(w[(int64_t)e * H + h]),
-                  acc);
-    return acc;
-}
-
-// AND of `pred` over the 128 epilogue threads (named barrier 1).
+// Reduction barriers over the 128 epilogue threads (named barrier 1).
 __device__ __forceinline__ bool epilogue_all(bool pred) {
     uint32_t out;
     asm volatile(
@@ -80,39 +91,63 @@ __device__ __forceinline__ bool epilogue_all(bool pred) {
     return out != 0;
 }
 
+__device__ __forceinline__ bool epilogue_any(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return out != 0;
+}
+
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 // KMAX: capacity of the per-thread selection (k <= KMAX).  KMAX = kMaxTopK
 // serves only k == E (every expert selected), where no decision is uncertain.
 template <int KMAX>
 __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int H, int E,
-    int Npad, int k, uint32_t tmem_cols, const float* __restrict__ bias, const bf16* __restrict__ x_rows,
-    const bf16* __restrict__ wr_rows, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int32_t* flags) {
+    int Npad, int k, int stages, uint32_t acc_cols, const float* __restrict__ bias,
+    const bf16* __restrict__ x_rows, const bf16* __restrict__ wr_rows, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w, int32_t* flags) {
     constexpr bool kDense = (KMAX == kMaxTopK);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int stage_bytes = kABytes + Npad * kBK * 2;  // a multiple of 1024
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes);
-    uint64_t* empty = full + kStages;
-    uint64_t* acc_ready = empty + kStages;
-    uint64_t* drain = acc_ready + 1;
+    uint8_t* tail = smem + stages * stage_bytes;
+    int2* qp = reinterpret_cast<int2*>(tail);                   // [kQueue] (row, expert)
+    double* qs = reinterpret_cast<double*>(qp + kQueue);       // [kQueue] exact scores
+    uint64_t* full = reinterpret_cast<uint64_t*>(qs + kQueue);  // [stages]
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* tfull = empty + kMaxStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);  // [2]: abort, queue length
-    float* bs = reinterpret_cast<float*>(smem + kStages * stage_bytes + 128);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    int* qn = reinterpret_cast<int*>(tmem_holder + 2);
+    float* bs = reinterpret_cast<float*>(tmem_holder + 4);  // [E]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     for (int e = threadIdx.x; e < E; e += kThreads) bs[e] = bias ? bias[e] : 0.f;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_ready, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 128);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, tmem_cols);
+        tmem_alloc(tmem_holder, 2 * acc_cols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -120,46 +155,58 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    const int t0 = blockIdx.x * kBM;
+    const int ntiles = (T + kBM - 1) / kBM;
     const int nkb = (H + kBK - 1) / kBK;
     if (warp == 0) {
+        // ------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_map(&tmX);
             tma_prefetch_map(&tmW);
-            int kb = 0;
-            for (; kb < nkb; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = (kb / kStages) & 1;
-                if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) break;
-                uint8_t* sa = smem + s * stage_bytes;
-                mbar_arrive_expect_tx(&full[s], stage_bytes);
-                tma_load_3d(sa, &tmX, &full[s], kb * kBK, t0, 0);
-                tma_load_3d(sa + kABytes, &tmW, &full[s], kb * kBK, 0, 0);
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) break;
+                    uint8_t* sa = smem + s * stage_bytes;
+                    mbar_arrive_expect_tx(&full[s], stage_bytes);
+                    tma_load_3d(sa, &tmX, &full[s], kb * kBK, tile * kBM, 0);
+                    tma_load_3d(sa + kABytes, &tmW, &full[s], kb * kBK, 0, 0);
+                }
             }
-            for (int j = (kb > kStages ? kb - kStages : 0); j < kb; ++j)
-                drain_wait(&full[j % kStages], (j / kStages) & 1);
+            for (uint32_t j = (it > (uint32_t)stages ? it - stages : 0); j < it; ++j)
+                drain_wait(&full[j % stages], (j / stages) & 1);
         }
     } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(kBM, Npad);
-            bool ok = true;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = (kb / kStages) & 1;
-                if (!wait_or_abort(&full[s], ph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) {
-                    ok = false;
-                    break;
-                }
+            uint32_t it = 0, tc = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!wait_or_abort(&tempty[acc], aph ^ 1, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(smem + s * stage_bytes);
-                const uint32_t b0 = a0 + kABytes;
+                const uint32_t d = tmem_base + acc * acc_cols;
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!wait_or_abort(&full[s], ph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + s * stage_bytes);
+                    const uint32_t b0 = a0 + kABytes;
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                    mma_bf16(tmem_base, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc,
-                             (kb | kk) != 0);
-                mma_commit(&empty[s]);
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_bf16(d, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc,
+                                 (kb | kk) != 0);
+                    mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
             }
-            if (ok) mma_commit(acc_ready);
             mma_commit(drain);
             drain_wait(drain, 0);
         }
@@ -167,76 +214,58 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
         // ------------------------------------------------ epilogue warps 2..5
         const int q = warp & 3;
         const int r = q * 32 + lane;  // token row of this thread within the tile
-        const int t = t0 + r;
         const int ew = warp - 2;      // epilogue warp 0..3
-        const bool ready = wait_or_abort(acc_ready, 0, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT);
-        // all four epilogue warps take the same branch, so the named barriers
-        // below are always reached by all 128 threads
-        if (epilogue_all(ready)) {
+        uint32_t tc = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            const bool ready = wait_or_abort(&tfull[acc], aph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT);
+            // all 128 epilogue threads take the same branch, so every named
+            // barrier below is reached by all of them
+            if (!epilogue_all(ready)) break;
             tc_fence_after();
-            // Every MMA has completed, so the stage buffers are free: they hold
-            // the tile's scores and the exact-rescoring queue from here on.
-            float* sc = reinterpret_cast<float*>(smem);                 // [128][E+1]
-            int2* qp = reinterpret_cast<int2*>(sc + kBM * (E + 1));      // [kQueue] (row, expert)
-            double* qs = reinterpret_cast<double*>(qp + kQueue);        // [kQueue] exact scores
-            int* qn = const_cast<int*>(abort_flag) + 1;                 // queue length
-            float* srow = sc + r * (E + 1);
-            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16);
+            const int t = tile * kBM + r;
+            const uint32_t tq = tmem_base + acc * acc_cols + ((uint32_t)(q * 32) << 16);
 
-            // pass 1: approximate scores (float32 tensor-core sums + bias), the
-            // k+1 best in registers ordered by (score desc, index asc), and the
-            // magnitude of the raw dot products for the error bound
+            // pass 1: the k (+1) best approximate scores, picked in k (+1)
+            // rounds; round j takes the best score ranking after the pick of
+            // round j-1 in the order (score desc, index asc).  Branch-free
+            // scans of the TMEM row, all state in registers.
             float tv[KMAX + 1];
             int te[KMAX + 1];
+            const int kk = k < E ? k + 1 : k;
+            float amax = 0.f;
+            float pv = INFINITY;
+            int pe = -1;
 #pragma unroll
             for (int j = 0; j <= KMAX; ++j) {
-                tv[j] = -INFINITY;
-                te[j] = 0x7fffffff;
-            }
-            const int kk = k < E ? k + 1 : k;  // also track the (k+1)-th when it exists
-            float kth_v = -INFINITY, amax = 0.f;
-            int kth_e = 0x7fffffff;
-            for (int c0 = 0; c0 < E; c0 += 32) {
-                float v[32];
-                tmem_ld32(tq + c0, v);
+                float bv = -INFINITY;
+                int be = 0x7fffffff;
+                if (j < kk) {
+                    for (int c0 = 0; c0 < E; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(tq + c0, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int e = c0 + i;
-                    if (e < E) {
-                        amax = fmaxf(amax, fabsf(v[i]));
-                        float cv = v[i] + bs[e];
-                        srow[e] = cv;
-                        int ce = e;
-                        if (ranks_before(cv, ce, kth_v, kth_e)) {
-#pragma unroll
-                            for (int j = 0; j <= KMAX; ++j) {
-                                if (j < kk && ranks_before(cv, ce, tv[j], te[j])) {
-                                    float fv = tv[j];
-                                    int fe = te[j];
-                                    tv[j] = cv;
-                                    te[j] = ce;
-                                    cv = fv;
-                                    ce = fe;
-                                }
+                        for (int i = 0; i < 32; ++i) {
+                            const int e = c0 + i;
+                            if (j == 0) amax = fmaxf(amax, (e < E) ? fabsf(v[i]) : 0.f);
+                            const float cv = v[i] + bs[e < E ? e : 0];
+                            // after the previous pick, and strictly better than the best so far
+                            // (scanning in ascending index keeps the lower index on ties)
+                            const bool after = (cv < pv) || (cv == pv && e > pe);
+                            if (e < E && after && cv > bv) {
+                                bv = cv;
+                                be = e;
                             }
-#pragma unroll
-                            for (int j = 0; j <= KMAX; ++j)
-                                if (j == kk - 1) {
-                                    kth_v = tv[j];
-                                    kth_e = te[j];
-                                }
                         }
                     }
+                    pv = bv;
+                    pe = be;
                 }
+                tv[j] = bv;
+                te[j] = be;
             }
 
-            // Decision certainty.  The tensor-core sums differ from the exact
-            // ones by at most about one float32 ulp of the running sum per
-            // 16-wide step; delta is 32x that bound.  With the k-th and (k+1)-th
-            // approximate scores more than delta apart the selection is exact.
-            // Otherwise the experts whose approximate score lies in the band
-            // [s_k - delta, s_{k+1} + delta] are rescored exactly (fp64) and the
-            // selection is completed from those exact scores.
+            // certainty of the decision
             float band_lo = 0.f, band_hi = 0.f;
             bool uncertain = false;
             int n_in = k;
@@ -247,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                     if (j == k - 1) kth = tv[j];
                     if (j == k) next = tv[j];
                 }
-                const float delta = 2.0f * (float)H * 1.1920929e-7f * fmaxf(amax, 1.0f);
+                const float delta = 0.5f * (float)H * 1.1920929e-7f * fmaxf(amax, 1.0f);
                 if (kth - next <= delta) {
                     uncertain = true;
                     band_lo = kth - delta;
@@ -259,34 +288,79 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                 }
             }
 
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (threadIdx.x == 64) *qn = 0;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            bool overflow = false;
-            if (uncertain) {
-                for (int e = 0; e < E; ++e) {
-                    const float sv = srow[e];
-                    if (sv >= band_lo && sv <= band_hi) {
-                        const int slot = atomicAdd(qn, 1);
-                        if (slot < kQueue)
-                            qp[slot] = make_int2(r, e);
-                        else
-                            overflow = true;
+            // final selection state: certain prefix + the best `need` band
+            // members by exact score (ties to the lower index)
+            const int need = k - n_in;
+            double bv[KMAX];
+            int be[KMAX];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                bv[j] = -INFINITY;
+                be[j] = 0x7fffffff;
+            }
+            // pass 2, in rounds of at most kQueue band members per tile: queue
+            // them (scores re-read from TMEM), rescore them exactly with whole
+            // warps, let each token take its own.  One round in practice.
+            int cursor = uncertain ? 0 : E;  // next expert this thread still has to scan
+            while (epilogue_any(cursor < E)) {
+                if (threadIdx.x == 64) *qn = 0;
+                epilogue_sync();
+                if (__any_sync(0xffffffffu, cursor < E)) {
+                    bool stop = false;
+                    for (int c0 = 0; c0 < E; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(tq + c0, v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int e = c0 + i;
+                            if (!stop && e >= cursor && e < E) {
+                                const float sv = v[i] + bs[e];
+                                if (sv >= band_lo && sv <= band_hi) {
+                                    const int slot = atomicAdd(qn, 1);
+                                    if (slot < kQueue) {
+                                        qp[slot] = make_int2(r, e);
+                                    } else {
+                                        stop = true;  // queue full: resume here next round
+                                        cursor = e;
+                                    }
+                                }
+                            }
+                        }
                     }
+                    if (!stop) cursor = E;
                 }
+                epilogue_sync();
+                const int nq = min(*qn, kQueue);
+                for (int i = ew; i < nq; i += 4) {
+                    const int2 pr = qp[i];
+                    const double sd = exact_score(x_rows, wr_rows, tile * kBM + pr.x, pr.y, H, lane);
+                    if (lane == 0) qs[i] = sd + (double)bs[pr.y];
+                }
+                epilogue_sync();
+                if (uncertain)
+                    for (int i = 0; i < nq; ++i) {
+                        const int2 pr = qp[i];
+                        if (pr.x != r) continue;
+                        // insert (qs[i], pr.y) into the `need` best, ties to the lower index
+                        double cv = qs[i];
+                        int ce = pr.y;
+#pragma unroll
+                        for (int j = 0; j < KMAX; ++j) {
+                            if (j < need && (cv > bv[j] || (cv == bv[j] && ce < be[j]))) {
+                                const double ov = bv[j];
+                                const int oe = be[j];
+                                bv[j] = cv;
+                                be[j] = ce;
+                                cv = ov;
+                                ce = oe;
+                            }
+                        }
+                    }
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            const int nq = min(*qn, kQueue);
-            // warp-cooperative exact rescoring: lanes split H in 8-element chunks
-            for (int i = ew; i < nq; i += 4) {
-                const int2 pr = qp[i];
-                const double sd = exact_score(x_rows, wr_rows, t0 + pr.x, pr.y, H, lane);
-                if (lane == 0) qs[i] = sd + (double)bs[pr.y];
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            // the accumulator is no longer needed: hand it back to the MMA warp
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
 
-            // final selection: certain prefix (approximate order) + the best
-            // `need` band members by exact score (ties to the lower index)
             float fv[KMAX];
             int fe[KMAX];
 #pragma unroll
@@ -295,51 +369,22 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                 fe[j] = te[j];
             }
             if (!kDense && uncertain) {
-                const int need = k - n_in;
-                double bv[KMAX];
-                int be[KMAX];
+                // move the band picks to slots n_in..k-1: n_in predicated
+                // right-shifts keep every index static (registers, no stack)
 #pragma unroll
-                for (int j = 0; j < KMAX; ++j) {
-                    bv[j] = -INFINITY;
-                    be[j] = 0x7fffffff;
-                }
-                auto offer = [&](double cv, int ce) {
+                for (int sft = 0; sft < KMAX; ++sft)
+                    if (sft < n_in) {
 #pragma unroll
-                    for (int j = 0; j < KMAX; ++j) {
-                        if (j < need && (cv > bv[j] || (cv == bv[j] && ce < be[j]))) {
-                            double ov = bv[j];
-                            int oe = be[j];
-                            bv[j] = cv;
-                            be[j] = ce;
-                            cv = ov;
-                            ce = oe;
+                        for (int j = KMAX - 1; j > 0; --j) {
+                            bv[j] = bv[j - 1];
+                            be[j] = be[j - 1];
                         }
                     }
-                };
-                for (int i = 0; i < nq; ++i) {
-                    const int2 pr = qp[i];
-                    if (pr.x == r) offer(qs[i], pr.y);
-                }
-                if (overflow) {
-                    // queue full (pathological near-ties): rescore the rest here
-                    for (int e = 0; e < E; ++e) {
-                        const float sv = srow[e];
-                        if (sv >= band_lo && sv <= band_hi) {
-                            bool queued = false;
-                            for (int i = 0; i < nq && !queued; ++i) queued = (qp[i].x == r && qp[i].y == e);
-                            if (!queued) offer(exact_score_serial(x_rows, wr_rows, t, e, H) + (double)bs[e], e);
-                        }
-                    }
-                }
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
                     if (j >= n_in && j < k) {
-#pragma unroll
-                        for (int i = 0; i < KMAX; ++i)
-                            if (i == j - n_in) {
-                                fv[j] = (float)bv[i];
-                                fe[j] = be[i];
-                            }
+                        fv[j] = (float)bv[j];
+                        fe[j] = be[j];
                     }
             }
             if (t < T) {
@@ -365,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+    if (warp == 1) tmem_dealloc(tmem_base, 2 * acc_cols);
 }
 
 }  // namespace
@@ -380,24 +425,28 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     CUtensorMap mx, mw;
     if (!make_map_bf16(&mx, x, p.H, p.T, 1, kBK, kBM) || !make_map_bf16(&mw, router_w, p.H, E, 1, kBK, Npad))
         return cudaErrorInvalidValue;
-    const size_t smem = kStages * (size_t)(kABytes + Npad * kBK * 2) + 1024 + 128 + sizeof(float) * E;
-    const dim3 grid((unsigned)((p.T + kBM - 1) / kBM));
+    const int stage_bytes = kABytes + Npad * kBK * 2;
+    const size_t fixed = 1024 + (size_t)kQueue * 16 + 8 * (2 * kMaxStages + 5) + 16 + sizeof(float) * E;
+    int stages = (int)((227 * 1024 - fixed) / stage_bytes);
+    stages = stages > kMaxStages ? kMaxStages : stages;
+    const size_t smem = (size_t)stages * stage_bytes + fixed;
+    const int ntiles = (int)((p.T + kBM - 1) / kBM);
+    const dim3 grid((unsigned)(ntiles < device_sm_count() ? ntiles : device_sm_count()));
     cudaError_t e;
     trace_before("router_sm100", st);
     if (p.k <= 8) {
         e = cudaFuncSetAttribute(router_sm100_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess)
-            router_sm100_kernel<8><<<grid, kThreads, smem, st>>>(mx, mw, (int)p.T, (int)p.H, E, Npad, (int)p.k, cols,
-                                                               router_b, (const bf16*)x, (const bf16*)router_w,
-                                                               topk_idx, topk_w, p.flags);
+            router_sm100_kernel<8><<<grid, kThreads, smem, st>>>(mx, mw, (int)p.T, (int)p.H, E, Npad, (int)p.k,
+                                                               stages, cols, router_b, (const bf16*)x,
+                                                               (const bf16*)router_w, topk_idx, topk_w, p.flags);
     } else {
         e = cudaFuncSetAttribute(router_sm100_kernel<kMaxTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e == cudaSuccess)
-            router_sm100_kernel<kMaxTopK><<<grid, kThreads, smem, st>>>(mx, mw, (int)p.T, (int)p.H, E, Npad,
-                                                                      (int)p.k, cols, router_b, (const bf16*)x,
-                                                                      (const bf16*)router_w, topk_idx, topk_w,
-                                                                      p.flags);
+            router_sm100_kernel<kMaxTopK><<<grid, kThreads, smem, st>>>(
+                mx, mw, (int)p.T, (int)p.H, E, Npad, (int)p.k, stages, cols, router_b, (const bf16*)x,
+                (const bf16*)router_w, topk_idx, topk_w, p.flags);
     }
     trace_after(st);
     return e != cudaSuccess ? e : cudaGetLastError();
