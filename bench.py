@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--workload", default="mixtral_8x7b_layer")
     ap.add_argument("--T", type=int, default=0, help="override the token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every step from the host instead of replaying a CUDA graph of the K steps")
     return ap.parse_args()
 
 
@@ -260,8 +262,9 @@ def run_ours(args, wl, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def step(x_in):
+        # enqueued on the current stream (the capture stream while a graph is recorded)
         moe.moe_forward(cfg, x_in, d["router_w"], d["router_b"], d["w_gate"], d["w_up"], d["w_down"],
-                        d["ws_gate"], d["ws_up"], d["ws_down"], y, None, counts, None, ws, stream)
+                        d["ws_gate"], d["ws_up"], d["ws_down"], y, None, counts, None, ws)
 
     def barrier():
         if world > 1:
@@ -289,42 +292,70 @@ def run_ours(args, wl, world, rank, local):
     except Exception:
         gpu_uuid = None
 
-    # ---- timed region: device time of K steps, kernels traced live
+    # ---- timed region: device time of K steps, kernels traced live.  With
+    # graphs (default) the K steps, trace events included, are captured once
+    # into one CUDA graph and the timed region is one replay of it.
+    use_graph = not args.no_graph
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        moe.moe_trace_begin(64 * args.steps)
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            for _ in range(args.steps):
+                step(d["x"])
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(gpu_uuid) as clocks:
-        moe.moe_trace_begin(64 * args.steps)
+        if not use_graph:
+            moe.moe_trace_begin(64 * args.steps)
         start.record(stream)
-        for _ in range(args.steps):
-            step(d["x"])
+        if use_graph:
+            graph.replay()
+        else:
+            for _ in range(args.steps):
+                step(d["x"])
         stop.record(stream)
         torch.cuda.synchronize(dev)
         trace = moe.moe_trace_end(64 * args.steps)
     barrier()
     ms = max_over_ranks(start.elapsed_time(stop))
     clk = clocks.summary()
+    del graph
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host
     x_host = d["x"].cpu().pin_memory()
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     x_dev = torch.empty_like(d["x"])
-    for _ in range(2):
+
+    def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
         step(x_dev)
         y_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    g2 = None
+    if use_graph:
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, capture_error_mode="thread_local"):
+            for _ in range(args.steps):
+                e2e_step()
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x_dev)
-        y_host.copy_(y, non_blocking=True)
+    if use_graph:
+        g2.replay()
+    else:
+        for _ in range(args.steps):
+            e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+    del g2
 
     tokens = wl.T * args.steps * world
     value = tokens / (ms / 1e3)
@@ -359,7 +390,8 @@ def run_ours(args, wl, world, rank, local):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": dict(config_of(wl), l2="inputs larger than L2: %.1f GB of expert weights read per step"
-                       % (active * 3 * wl.H * wl.I * 2 / 1e9), parallelism=f"replicas{world}"),
+                       % (active * 3 * wl.H * wl.I * 2 / 1e9), parallelism=f"replicas{world}",
+                       launch="cuda graph of the K steps" if use_graph else "host launches"),
         "roofline": roof,
         "layer_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / t_step, "flops": F, "bytes": B,
                            "bound": "tensor" if F / (pk["bf16_tflops"] * 1e12) >= B / (pk["hbm_gbs"] * 1e9) else "hbm",

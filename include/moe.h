@@ -223,6 +223,9 @@ const char* moe_last_error(void);
  * recorded events, writes for each launch its kernel name and its duration
  * in milliseconds, and turns tracing off.  Host-side only; no device
  * memory is allocated.  Not thread-safe: one tracing session at a time.
+ * Calls enqueued while their stream is being captured into a CUDA graph are
+ * traced through external event-record nodes: end the session after one
+ * replay of that graph to read the launches' times.
  */
 typedef struct {
     const char* name; /* static string */

@@ -352,8 +352,7 @@ template <bool kGateUp>
 cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const GemmArgs& args,
                            cudaStream_t st) {
     constexpr int BN = kGateUp ? kBRows / 2 : kBRows;
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_sm100_kernel<kGateUp>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaError_t e = ensure_smem_attr(grouped_gemm_sm100_kernel<kGateUp>, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t nb_r = (args.N + BN - 1) / BN;
     const int64_t nb_s = args.has_shared ? (args.Ns + BN - 1) / BN : 0;

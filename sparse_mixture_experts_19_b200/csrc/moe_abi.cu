@@ -41,9 +41,18 @@ struct TraceState {
 TraceState g_trace;
 }  // namespace
 
+// Inside a stream capture an event is recorded by an external event-record
+// node, so that replays of the graph record it.
+static cudaError_t trace_record(cudaEvent_t ev, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        return cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+    return cudaEventRecord(ev, st);
+}
+
 void trace_before(const char* name, cudaStream_t st) {
     if (!g_trace.on || g_trace.n >= g_trace.max) return;
-    if (cudaEventRecord(g_trace.ev[2 * g_trace.n], st) != cudaSuccess) return;
+    if (trace_record(g_trace.ev[2 * g_trace.n], st) != cudaSuccess) return;
     g_trace.names[g_trace.n] = name;
     g_trace.open = true;
 }
@@ -51,7 +60,7 @@ void trace_before(const char* name, cudaStream_t st) {
 void trace_after(cudaStream_t st) {
     if (!g_trace.on || !g_trace.open) return;
     g_trace.open = false;
-    if (cudaEventRecord(g_trace.ev[2 * g_trace.n + 1], st) == cudaSuccess) g_trace.n++;
+    if (trace_record(g_trace.ev[2 * g_trace.n + 1], st) == cudaSuccess) g_trace.n++;
 }
 
 // --------------------------------------------------------------- the plan

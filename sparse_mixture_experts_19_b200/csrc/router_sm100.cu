@@ -435,14 +435,13 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     cudaError_t e;
     trace_before("router_sm100", st);
     if (p.k <= 8) {
-        e = cudaFuncSetAttribute(router_sm100_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = ensure_smem_attr(router_sm100_kernel<8>, smem);
         if (e == cudaSuccess)
             router_sm100_kernel<8><<<grid, kThreads, smem, st>>>(mx, mw, (int)p.T, (int)p.H, E, Npad, (int)p.k,
                                                                stages, cols, router_b, (const bf16*)x,
                                                                (const bf16*)router_w, topk_idx, topk_w, p.flags);
     } else {
-        e = cudaFuncSetAttribute(router_sm100_kernel<kMaxTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
+        e = ensure_smem_attr(router_sm100_kernel<kMaxTopK>, smem);
         if (e == cudaSuccess)
             router_sm100_kernel<kMaxTopK><<<grid, kThreads, smem, st>>>(
                 mx, mw, (int)p.T, (int)p.H, E, Npad, (int)p.k, stages, cols, router_b, (const bf16*)x,
