@@ -218,7 +218,8 @@ const char* moe_last_error(void);
 
 /*
  * Kernel tracing (for measurement).  While tracing is on, every kernel the
- * library enqueues is bracketed by two CUDA events on its stream; up to
+ * library enqueues whose name contains `only` (every kernel if `only` is
+ * NULL or empty) is bracketed by two CUDA events on its stream; up to
  * `max_launches` launches are recorded.  moe_trace_end() waits for the
  * recorded events, writes for each launch its kernel name and its duration
  * in milliseconds, and turns tracing off.  Host-side only; no device
@@ -232,7 +233,7 @@ typedef struct {
     float ms;
 } moe_trace_record_t;
 
-moe_status_t moe_trace_begin(int32_t max_launches);
+moe_status_t moe_trace_begin(int32_t max_launches, const char* only);
 moe_status_t moe_trace_end(moe_trace_record_t* records, int32_t max_records, int32_t* n_records);
 
 #ifdef __cplusplus

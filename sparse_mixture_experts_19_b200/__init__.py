@@ -55,7 +55,7 @@ _SIGS = {
                                ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
     "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "moe_last_error": ([], ctypes.c_char_p),
-    "moe_trace_begin": ([ctypes.c_int32], ctypes.c_int),
+    "moe_trace_begin": ([ctypes.c_int32, ctypes.c_char_p], ctypes.c_int),
     "moe_trace_end": ([ctypes.POINTER(moe_trace_record_t), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)],
                       ctypes.c_int),
 }
@@ -201,8 +201,9 @@ def moe_last_error() -> str:
     return load().moe_last_error().decode()
 
 
-def moe_trace_begin(max_launches: int):
-    _check(load().moe_trace_begin(max_launches))
+def moe_trace_begin(max_launches: int, only: str | None = None):
+    """Trace the next launches (only kernels whose name contains `only`)."""
+    _check(load().moe_trace_begin(max_launches, None if only is None else only.encode()))
 
 
 def moe_trace_end(max_records: int = 4096) -> list[tuple[str, float]]:

@@ -64,6 +64,13 @@ cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_
 cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router_w,
                                 const float* router_b, int32_t* topk_idx, float* topk_w,
                                 cudaStream_t st);
+// Router for few tokens: one CTA per token, exact fp64 scores.
+cudaError_t launch_router_decode(const Plan& p, const void* x, const void* router_w,
+                                 const float* router_b, int32_t* topk_idx, float* topk_w,
+                                 cudaStream_t st);
+// Scores of T*E*H at most this many multiply-adds go to the per-token router
+// (its weight traffic, T*E*H*2 bytes from L2, stays small).
+constexpr int64_t kDecodeRouterMaxMacs = int64_t(1) << 26;
 cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
                            int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
                            int32_t* dropped, cudaStream_t st);

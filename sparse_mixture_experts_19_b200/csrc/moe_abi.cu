@@ -35,6 +35,7 @@ struct TraceState {
     int max = 0;
     int n = 0;
     bool open = false;  // a launch has been started and not yet closed
+    char only[64] = {};  // trace only kernels whose name contains this ("" = all)
     std::vector<const char*> names;
     std::vector<cudaEvent_t> ev;
 };
@@ -52,6 +53,7 @@ static cudaError_t trace_record(cudaEvent_t ev, cudaStream_t st) {
 
 void trace_before(const char* name, cudaStream_t st) {
     if (!g_trace.on || g_trace.n >= g_trace.max) return;
+    if (g_trace.only[0] && !strstr(name, g_trace.only)) return;
     if (trace_record(g_trace.ev[2 * g_trace.n], st) != cudaSuccess) return;
     g_trace.names[g_trace.n] = name;
     g_trace.open = true;
@@ -165,6 +167,15 @@ static moe_status_t check_shared(const Plan& p, const void* a, const void* b, co
     return MOE_OK;
 }
 
+// Router choice by size: few tokens -> per-token exact router; otherwise the
+// tensor-core router (bf16) or the CUDA-core float32 router.
+static cudaError_t run_router(const Plan& p, const void* x, const void* router_w, const float* router_b,
+                              int32_t* idx, float* w, cudaStream_t st) {
+    if (p.T * p.E * p.H <= kDecodeRouterMaxMacs) return launch_router_decode(p, x, router_w, router_b, idx, w, st);
+    if (p.bf16) return launch_router_sm100(p, x, router_w, router_b, idx, w, st);
+    return launch_router_simt(p, x, router_w, router_b, idx, w, st);
+}
+
 // The grouped FFN of moe_forward / moe_grouped_ffn, after routing and grouping.
 static moe_status_t run_ffn(const Plan& p, const void* x, const void* w_gate, const void* w_up,
                             const void* w_down, const void* ws_gate, const void* ws_up,
@@ -215,10 +226,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* route
     REQUIRE_PTR(topk_idx);
     REQUIRE_PTR(topk_w);
     cudaStream_t st = (cudaStream_t)stream;
-    if (p.bf16)
-        CUDA_TRY(launch_router_sm100(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
-    else
-        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
+    CUDA_TRY(run_router(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
     return MOE_OK;
 }
 
@@ -336,10 +344,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
     int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
-    if (p.bf16)
-        CUDA_TRY(launch_router_sm100(p, x, router_w, router_b, idx, p.topk_w, st), "router");
-    else
-        CUDA_TRY(launch_router_simt(p, x, router_w, router_b, idx, p.topk_w, st), "router");
+    CUDA_TRY(run_router(p, x, router_w, router_b, idx, p.topk_w, st), "router");
     CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
     if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.rows, st)) != MOE_OK)
         return s;
@@ -377,10 +382,14 @@ const char* moe_status_string(moe_status_t status) {
 
 const char* moe_last_error(void) { return g_last_error; }
 
-moe_status_t moe_trace_begin(int32_t max_launches) {
+moe_status_t moe_trace_begin(int32_t max_launches, const char* only) {
     if (max_launches <= 0) return fail(MOE_ERR_INVALID_ARG, "max_launches = %d", max_launches);
     if (g_trace.on) return fail(MOE_ERR_INVALID_ARG, "tracing already on");
     g_trace = TraceState();
+    if (only) {
+        strncpy(g_trace.only, only, sizeof(g_trace.only) - 1);
+        g_trace.only[sizeof(g_trace.only) - 1] = 0;
+    }
     g_trace.ev.resize(2 * (size_t)max_launches);
     g_trace.names.resize(max_launches);
     for (auto& e : g_trace.ev)

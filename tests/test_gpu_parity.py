@@ -86,6 +86,23 @@ def test_layer_edge_cases(gpu_lib, wl):
     check_layer(gpu_lib, wl)
 
 
+# The layer scores few tokens with a per-token fp64 router and many tokens
+# with the tensor-core router (T*E*H above 2^26 multiply-adds).  These cases
+# sit above that size so the tensor-core router is exercised on shapes
+# the oracle evaluates in full.
+TC_ROUTER = [
+    mi.Workload("tc_router_e256_zipf", T=600, H=512, I=64, E=256, k=8, zipf_s=1.1, I_shared=64),
+    mi.Workload("tc_router_e32", T=2100, H=1024, I=64, E=32, k=4),
+    mi.Workload("tc_router_e8_ragged", T=8300, H=1032, I=64, E=8, k=2),
+]
+
+
+@pytest.mark.parametrize("wl", TC_ROUTER, ids=[w.name for w in TC_ROUTER])
+def test_layer_tensor_core_router(gpu_lib, wl):
+    assert wl.T * wl.E * wl.H > 2 ** 26
+    check_layer(gpu_lib, wl)
+
+
 def test_all_tokens_to_one_expert(gpu_lib):
     """A router bias that sends every token to experts 0 and 1."""
     wl = mi.Workload("skew", T=400, H=128, I=64, E=8, k=2, zipf_s=0.0)
@@ -123,7 +140,7 @@ def stage_setup(moe, wl):
 
 
 @pytest.mark.parametrize("wl", [mi.SMALL["fine_grained_e256_layer"], mi.SMALL["qwen3_30b_a3b_layer"],
-                                mi.TINY], ids=["fine_small", "qwen3_small", "tiny"])
+                                mi.TINY, TC_ROUTER[0]], ids=["fine_small", "qwen3_small", "tiny", "tc_router"])
 def test_stages_route_permute_ffn_combine(gpu_lib, wl):
     moe = gpu_lib
     inp, d, cfg, ws = stage_setup(moe, wl)
