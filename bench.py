@@ -181,6 +181,24 @@ def oracle_tokens_per_s(wl, inp, target_s: float, seed: int = 3):
 
 
 # -------------------------------------------------------------- the arms
+def reduce_max(v: float, world: int, device="cpu") -> float:
+    """Max of v over the ranks of the default process group (v if world == 1)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(T: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank ran `steps` batches of T tokens; the
+    job took the slowest rank's time."""
+    return T * steps * world / (ms_max / 1e3)
+
+
 def dist_setup(args):
     import torch
     import torch.distributed as dist
@@ -271,11 +289,7 @@ def run_ours(args, wl, world, rank, local):
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, dev)
 
     for _ in range(args.warmup):
         step(d["x"])
@@ -367,7 +381,7 @@ def run_ours(args, wl, world, rank, local):
     del g2
 
     tokens = wl.T * args.steps * world
-    value = tokens / (ms / 1e3)
+    value = job_tokens_per_s(wl.T, args.steps, world, ms)
     pk, pk_kind = peaks()
 
     # ---- roofline of the dominant kernel (grouped gate/up GEMM + SwiGLU)
