@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--workload", default="mixtral_8x7b_layer")
     ap.add_argument("--T", type=int, default=0, help="override the token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", choices=["forward", "route"], default="forward",
+                    help="route: time moe_route alone (only x and the router weights are allocated)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step from the host instead of replaying a CUDA graph of the K steps")
     return ap.parse_args()
@@ -437,9 +439,56 @@ def run_ours(args, wl, world, rank, local):
     return out
 
 
+def run_route_stage(args, wl):
+    """moe_route alone on the workload's x and router weights: K steps, one line."""
+    import numpy as np
+    import torch
+
+    import moe_inputs as mi
+    import sparse_mixture_experts_19_b200 as moe
+    from sparse_mixture_experts_19_b200 import build as moe_build
+
+    moe_build.build()
+    moe.load()
+    inp = mi.make_inputs(wl, router_only=True)
+
+    def to_dev(a):
+        if a is None:
+            return None
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.cuda()
+
+    x, rw, rb = to_dev(inp["x"]), to_dev(inp["router_w"]), to_dev(inp["router_b"])
+    cfg = moe.config(wl.T, wl.H, wl.I, wl.E, wl.k, wl.I_shared, wl.capacity_factor, wl.dtype)
+    ws = moe.workspace(cfg)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        moe.moe_route(cfg, x, rw, rb, idx, w, ws)
+    torch.cuda.synchronize()
+    moe.moe_trace_begin(8 * args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        moe.moe_route(cfg, x, rw, rb, idx, w, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    trace = moe.moe_trace_end(8 * args.steps)
+    ms = e0.elapsed_time(e1) / args.steps
+    kern = {}
+    for name, t in trace:
+        kern.setdefault(name, []).append(t)
+    return {"stage": "route", "config": config_of(wl), "ms_per_call": ms, "tokens_per_s": wl.T / (ms / 1e3),
+            "x_bytes_per_s": wl.T * wl.H * (2 if wl.dtype == "bf16" else 4) / (ms / 1e3),
+            "kernels_ms_per_call": {k: sum(v) / len(v) for k, v in kern.items()}}
+
+
 def main():
     args = parse_args()
     wl = workload(args)
+    if args.stage == "route":
+        print(json.dumps(run_route_stage(args, wl)), flush=True)
+        return
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         out = run_reference(args, wl, world, rank)

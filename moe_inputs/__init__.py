@@ -169,21 +169,26 @@ SMALL = {
 }
 
 
-def make_inputs(w: Workload) -> dict:
-    """All inputs of workload w as numpy arrays (bf16 as uint16 bits)."""
+def make_inputs(w: Workload, router_only: bool = False) -> dict:
+    """All inputs of workload w as numpy arrays (bf16 as uint16 bits).
+
+    router_only: only x, router_w and router_b (expert weights are None)."""
     s, dt = w.seed, w.dtype
     out = {
         "x": normal(s, STREAM_X, (w.T, w.H), 1.0, dt),
         "router_w": normal(s, STREAM_ROUTER_W, (w.E, w.H), 1.0 / math.sqrt(w.H), dt),
-        "w_gate": normal(s, STREAM_W_GATE, (w.E, w.I, w.H), 1.0 / math.sqrt(w.H), dt),
-        "w_up": normal(s, STREAM_W_UP, (w.E, w.I, w.H), 1.0 / math.sqrt(w.H), dt),
-        "w_down": normal(s, STREAM_W_DOWN, (w.E, w.H, w.I), 1.0 / math.sqrt(w.I), dt),
+        "w_gate": None, "w_up": None, "w_down": None,
         "router_b": None,
         "ws_gate": None, "ws_up": None, "ws_down": None,
     }
     if w.has_bias:
         rank = permutation(s, STREAM_ZIPF_RANK, w.E).astype(np.float64) + 1.0
         out["router_b"] = (-w.zipf_s * np.log(rank)).astype(np.float32)
+    if router_only:
+        return out
+    out["w_gate"] = normal(s, STREAM_W_GATE, (w.E, w.I, w.H), 1.0 / math.sqrt(w.H), dt)
+    out["w_up"] = normal(s, STREAM_W_UP, (w.E, w.I, w.H), 1.0 / math.sqrt(w.H), dt)
+    out["w_down"] = normal(s, STREAM_W_DOWN, (w.E, w.H, w.I), 1.0 / math.sqrt(w.I), dt)
     if w.I_shared > 0:
         Is = w.I_shared
         out["ws_gate"] = normal(s, STREAM_WS_GATE, (Is, w.H), 1.0 / math.sqrt(w.H), dt)

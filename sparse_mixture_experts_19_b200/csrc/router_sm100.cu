@@ -238,31 +238,38 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
             int pe = -1;
 #pragma unroll
             for (int j = 0; j <= KMAX; ++j) {
-                float bv = -INFINITY;
-                int be = 0x7fffffff;
+                // four independent running maxima (elements i % 4), merged at
+                // the end; each keeps the lower index on ties because it
+                // visits its elements in ascending index order
+                float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                int be[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
                 if (j < kk) {
-                    for (int c0 = 0; c0 < E; c0 += 32) {
-                        float v[32];
-                        tmem_ld32(tq + c0, v);
+                    for (int c0 = 0; c0 < E; c0 += 64) {
+                        float v[64];
+                        tmem_ld64(tq + c0, v);  // columns past E (up to the allocation) are ignored
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
+                        for (int i = 0; i < 64; ++i) {
                             const int e = c0 + i;
                             if (j == 0) amax = fmaxf(amax, (e < E) ? fabsf(v[i]) : 0.f);
                             const float cv = v[i] + bs[e < E ? e : 0];
-                            // after the previous pick, and strictly better than the best so far
-                            // (scanning in ascending index keeps the lower index on ties)
                             const bool after = (cv < pv) || (cv == pv && e > pe);
-                            if (e < E && after && cv > bv) {
-                                bv = cv;
-                                be = e;
+                            if (e < E && after && cv > bv[i & 3]) {
+                                bv[i & 3] = cv;
+                                be[i & 3] = e;
                             }
                         }
                     }
-                    pv = bv;
-                    pe = be;
+#pragma unroll
+                    for (int c = 1; c < 4; ++c)
+                        if (ranks_before(bv[c], be[c], bv[0], be[0])) {
+                            bv[0] = bv[c];
+                            be[0] = be[c];
+                        }
+                    pv = bv[0];
+                    pe = be[0];
                 }
-                tv[j] = bv;
-                te[j] = be;
+                tv[j] = bv[0];
+                te[j] = be[0];
             }
 
             // certainty of the decision
@@ -420,7 +427,9 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     if (p.T == 0) return cudaSuccess;
     const int E = (int)p.E;
     const int Npad = E <= 16 ? 16 : (E + 15) / 16 * 16;
-    uint32_t cols = 32;
+    // accumulator width: a power of two >= Npad and >= 64, so that the
+    // epilogue's 64-column TMEM reads stay inside the accumulator
+    uint32_t cols = 64;
     while ((int)cols < Npad) cols <<= 1;
     CUtensorMap mx, mw;
     if (!make_map_bf16(&mx, x, p.H, p.T, 1, kBK, kBM) || !make_map_bf16(&mw, router_w, p.H, E, 1, kBK, Npad))
