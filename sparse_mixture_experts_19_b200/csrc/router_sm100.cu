@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     uint8_t* tail = smem + stages * stage_bytes;
     int2* qp = reinterpret_cast<int2*>(tail);                   // [kQueue] (row, expert)
     double* qs = reinterpret_cast<double*>(qp + kQueue);       // [kQueue] exact scores
-    uint64_t* full = reinterpret_cast<uint64_t*>(qs + kQueue);  // [stages]
+    uint8_t* misc = reinterpret_cast<uint8_t*>(qs + kQueue);   // 1024-aligned, 256 bytes
+    uint64_t* full = reinterpret_cast<uint64_t*>(misc);        // [stages]
     uint64_t* empty = full + kMaxStages;
     uint64_t* tfull = empty + kMaxStages;
     uint64_t* tempty = tfull + 2;
@@ -129,10 +130,12 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     int* qn = reinterpret_cast<int*>(tmem_holder + 2);
-    float* bs = reinterpret_cast<float*>(tmem_holder + 4);  // [E]
+    float* bs = reinterpret_cast<float*>(misc + 256);  // [E rounded up to 64], 16-byte aligned
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    for (int e = threadIdx.x; e < E; e += kThreads) bs[e] = bias ? bias[e] : 0.f;
+    const bool has_bias = bias != nullptr;
+    const int E64 = (E + 63) / 64 * 64;
+    for (int e = threadIdx.x; e < E64; e += kThreads) bs[e] = (bias && e < E) ? bias[e] : 0.f;
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
@@ -247,11 +250,28 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                     for (int c0 = 0; c0 < E; c0 += 64) {
                         float v[64];
                         tmem_ld64(tq + c0, v);  // columns past E (up to the allocation) are ignored
+                        if (j == 0) {
+                            // round 0: magnitude of the raw sums, then the bias is added
+                            // once and the biased scores are written back to TMEM for
+                            // the later rounds and the band pass
+#pragma unroll
+                            for (int i = 0; i < 64; ++i) amax = fmaxf(amax, (c0 + i < E) ? fabsf(v[i]) : 0.f);
+                            if (has_bias) {
+#pragma unroll
+                                for (int i = 0; i < 64; i += 4) {
+                                    const float4 b4 = *reinterpret_cast<const float4*>(bs + c0 + i);
+                                    v[i] += b4.x;
+                                    v[i + 1] += b4.y;
+                                    v[i + 2] += b4.z;
+                                    v[i + 3] += b4.w;
+                                }
+                                tmem_st64(tq + c0, v);
+                            }
+                        }
 #pragma unroll
                         for (int i = 0; i < 64; ++i) {
                             const int e = c0 + i;
-                            if (j == 0) amax = fmaxf(amax, (e < E) ? fabsf(v[i]) : 0.f);
-                            const float cv = v[i] + bs[e < E ? e : 0];
+                            const float cv = v[i];
                             const bool after = (cv < pv) || (cv == pv && e > pe);
                             if (e < E && after && cv > bv[i & 3]) {
                                 bv[i & 3] = cv;
@@ -321,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                         for (int i = 0; i < 32; ++i) {
                             const int e = c0 + i;
                             if (!stop && e >= cursor && e < E) {
-                                const float sv = v[i] + bs[e];
+                                const float sv = v[i];  // biased already (round 0)
                                 if (sv >= band_lo && sv <= band_hi) {
                                     const int slot = atomicAdd(qn, 1);
                                     if (slot < kQueue) {
@@ -435,7 +455,8 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     if (!make_map_bf16(&mx, x, p.H, p.T, 1, kBK, kBM) || !make_map_bf16(&mw, router_w, p.H, E, 1, kBK, Npad))
         return cudaErrorInvalidValue;
     const int stage_bytes = kABytes + Npad * kBK * 2;
-    const size_t fixed = 1024 + (size_t)kQueue * 16 + 8 * (2 * kMaxStages + 5) + 16 + sizeof(float) * E;
+    // alignment slack + queue + barrier block (168 B used of 256) + bias
+    const size_t fixed = 1024 + (size_t)kQueue * 16 + 256 + sizeof(float) * ((E + 63) / 64 * 64);
     int stages = (int)((227 * 1024 - fixed) / stage_bytes);
     stages = stages > kMaxStages ? kMaxStages : stages;
     const size_t smem = (size_t)stages * stage_bytes + fixed;
