@@ -151,9 +151,14 @@ def traffic_for(kernel: str, wl):
     d = json.load(open(path)).get(kernel)
     if not d or d.get("workload") != wl.name or d.get("T") != wl.T:
         return None
-    src = os.path.join(ROOT, d["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
-        return None
+    h = hashlib.sha256()
+    for rel in d["sources"]:
+        src = os.path.join(ROOT, rel)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    if h.hexdigest() != d["sources_sha256"]:
+        return None  # the kernel changed since the counters were taken
     return float(d["dram_bytes_per_launch"])
 
 
