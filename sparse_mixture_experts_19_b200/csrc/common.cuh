@@ -35,6 +35,7 @@ struct Plan {
     int32_t* dropped;     // [E]
     int32_t* offsets;     // [E + 2]: routed rows, offsets[E+1] = offsets[E] + shared rows
     int32_t* mtile_prefix;  // [E + 1]: prefix over experts of ceil(kept rows / 128)
+    int32_t* mpair_prefix;  // [E + 1]: prefix over experts of ceil(kept rows / 256)
     int32_t* perm_rows;   // [S]
     int32_t* row_of;      // [S]
     void* xperm;          // [S, H] layer dtype: x rows in grouped order

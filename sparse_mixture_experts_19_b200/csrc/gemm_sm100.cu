@@ -133,6 +133,76 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Drain one accumulator: this thread owns row r of the tile (TMEM lane
+// quadrant q).  gate/up: h = silu(G) * U in bf16; down: mode 1 weighted bf16
+// rows, mode 0 unweighted float32 rows.  tcgen05.ld is warp-collective, so
+// every lane loads and only rows < ti.rows store.
+template <bool kGateUp, int BN>
+__device__ __forceinline__ void epilogue_tile(const TileInfo& ti, const GemmArgs& a, uint32_t acc_base, int q,
+                                              int r) {
+    const uint32_t tq = acc_base + ((uint32_t)(q * 32) << 16);
+    const bool valid = r < ti.rows;
+    if (kGateUp) {
+        bf16* dst = ti.shared ? a.hs + (int64_t)(ti.arow + r) * a.Ns : a.h + (ti.row0 + r) * (int64_t)a.N;
+#pragma unroll 1
+        for (int j0 = 0; j0 < BN; j0 += 32) {
+            float g[32], u[32];
+            tmem_ld32(tq + j0, g);
+            tmem_ld32(tq + BN + j0, u);
+            if (valid) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int n = ti.n0 + j0 + v * 8;
+                    if (n < ti.N) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(silu_f32(g[v * 8 + 0]) * u[v * 8 + 0], silu_f32(g[v * 8 + 1]) * u[v * 8 + 1]);
+                        pk.y = pack_bf16x2(silu_f32(g[v * 8 + 2]) * u[v * 8 + 2], silu_f32(g[v * 8 + 3]) * u[v * 8 + 3]);
+                        pk.z = pack_bf16x2(silu_f32(g[v * 8 + 4]) * u[v * 8 + 4], silu_f32(g[v * 8 + 5]) * u[v * 8 + 5]);
+                        pk.w = pack_bf16x2(silu_f32(g[v * 8 + 6]) * u[v * 8 + 6], silu_f32(g[v * 8 + 7]) * u[v * 8 + 7]);
+                        *reinterpret_cast<uint4*>(dst + n) = pk;
+                    }
+                }
+            }
+        }
+    } else {
+        // output row: grouped row, or S + token for the shared expert
+        const int64_t orow = ti.shared ? a.S + ti.arow + r : ti.row0 + r;
+        float w = 1.f;
+        if (valid && a.mode == 1 && !ti.shared) w = a.topk_w[a.perm_rows[ti.row0 + r]];
+#pragma unroll 1
+        for (int j0 = 0; j0 < BN; j0 += 32) {
+            float v[32];
+            tmem_ld32(tq + j0, v);
+            if (valid) {
+                if (a.mode == 1) {
+                    bf16* dst = a.rows + orow * (int64_t)ti.N;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = ti.n0 + j0 + i * 8;
+                        if (n < ti.N) {
+                            uint4 pk;
+                            pk.x = pack_bf16x2(w * v[i * 8 + 0], w * v[i * 8 + 1]);
+                            pk.y = pack_bf16x2(w * v[i * 8 + 2], w * v[i * 8 + 3]);
+                            pk.z = pack_bf16x2(w * v[i * 8 + 4], w * v[i * 8 + 5]);
+                            pk.w = pack_bf16x2(w * v[i * 8 + 6], w * v[i * 8 + 7]);
+                            *reinterpret_cast<uint4*>(dst + n) = pk;
+                        }
+                    }
+                } else {
+                    float* dst = a.out + orow * (int64_t)ti.N;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int n = ti.n0 + j0 + i * 4;
+                        if (n < ti.N)
+                            *reinterpret_cast<float4*>(dst + n) =
+                                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                }
+            }
+        }
+    }
+}
+
 template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
@@ -272,68 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
             tc_fence_after();
-            const bool valid = r < ti.rows;
-            const uint32_t tq = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
-            if (kGateUp) {
-                bf16* dst = ti.shared ? a.hs + (int64_t)(ti.arow + r) * a.Ns
-                                      : a.h + (ti.row0 + r) * (int64_t)a.N;
-#pragma unroll 1
-                for (int j0 = 0; j0 < BN; j0 += 32) {
-                    float g[32], u[32];
-                    tmem_ld32(tq + j0, g);
-                    tmem_ld32(tq + BN + j0, u);
-                    if (valid) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const int n = ti.n0 + j0 + v * 8;
-                            if (n < ti.N) {
-                                uint4 pk;
-                                pk.x = pack_bf16x2(silu_f32(g[v * 8 + 0]) * u[v * 8 + 0], silu_f32(g[v * 8 + 1]) * u[v * 8 + 1]);
-                                pk.y = pack_bf16x2(silu_f32(g[v * 8 + 2]) * u[v * 8 + 2], silu_f32(g[v * 8 + 3]) * u[v * 8 + 3]);
-                                pk.z = pack_bf16x2(silu_f32(g[v * 8 + 4]) * u[v * 8 + 4], silu_f32(g[v * 8 + 5]) * u[v * 8 + 5]);
-                                pk.w = pack_bf16x2(silu_f32(g[v * 8 + 6]) * u[v * 8 + 6], silu_f32(g[v * 8 + 7]) * u[v * 8 + 7]);
-                                *reinterpret_cast<uint4*>(dst + n) = pk;
-                            }
-                        }
-                    }
-                }
-            } else {
-                // output row: grouped row, or S + token for the shared expert
-                const int64_t orow = ti.shared ? a.S + ti.arow + r : ti.row0 + r;
-                float w = 1.f;
-                if (valid && a.mode == 1 && !ti.shared) w = a.topk_w[a.perm_rows[ti.row0 + r]];
-#pragma unroll 1
-                for (int j0 = 0; j0 < BN; j0 += 32) {
-                    float v[32];
-                    tmem_ld32(tq + j0, v);
-                    if (valid) {
-                        if (a.mode == 1) {
-                            bf16* dst = a.rows + orow * (int64_t)ti.N;
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int n = ti.n0 + j0 + i * 8;
-                                if (n < ti.N) {
-                                    uint4 pk;
-                                    pk.x = pack_bf16x2(w * v[i * 8 + 0], w * v[i * 8 + 1]);
-                                    pk.y = pack_bf16x2(w * v[i * 8 + 2], w * v[i * 8 + 3]);
-                                    pk.z = pack_bf16x2(w * v[i * 8 + 4], w * v[i * 8 + 5]);
-                                    pk.w = pack_bf16x2(w * v[i * 8 + 6], w * v[i * 8 + 7]);
-                                    *reinterpret_cast<uint4*>(dst + n) = pk;
-                                }
-                            }
-                        } else {
-                            float* dst = a.out + orow * (int64_t)ti.N;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int n = ti.n0 + j0 + i * 4;
-                                if (n < ti.N)
-                                    *reinterpret_cast<float4*>(dst + n) =
-                                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                            }
-                        }
-                    }
-                }
-            }
+            epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r);
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
         }
@@ -343,6 +352,214 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ----------------------------------------------------------- CTA pairs
+// The same grouped GEMM on CTA pairs (clusters of 2): a tile is 256 rows x
+// BN of one group.  Each CTA stages its own 128 rows of A and 128 rows of B
+// (gate/up: CTA0 the gate rows, CTA1 the matching up rows; down: the two
+// halves of the 256 output columns), so a stage is 32 KB per CTA instead of
+// 48 KB and the shared-memory traffic per CTA drops by a third.  The leader
+// (rank 0) issues M = 256, N = 256 MMAs that read both CTAs' stages and write
+// each CTA's 128-row half of the accumulator into that CTA's TMEM, so both
+// CTAs drain their own half with the single-CTA epilogue.
+constexpr int kPStages = 6;
+constexpr int kPABytes = kBM * kBK * 2;         // 16 KB: this CTA's 128 rows of A
+constexpr int kPBBytes = (kBRows / 2) * kBK * 2;  // 16 KB: this CTA's half of B
+constexpr int kPStageBytes = kPABytes + kPBBytes;
+constexpr uint32_t kPIdesc = idesc_bf16(2 * kBM, kBRows);
+
+struct PairTables {
+    int32_t off[kMaxExperts + 2];
+    int32_t mpp[kMaxExperts + 1];  // prefix of 256-row pair tiles
+};
+
+// Pair tile t -> this CTA's (rank) half: rows row0 .. row0 + rows - 1 (rows may
+// be <= 0 when the group ends inside the pair's first half).
+__device__ __forceinline__ void decode_pair(int64_t t, const PairTables& tb, const Sched& sc, const GemmArgs& a,
+                                            int BN, uint32_t rank, TileInfo& ti) {
+    if (t < sc.routed_tiles) {
+        const int q = (int)(t / sc.nb_r);
+        int lo = 0, hi = sc.E - 1;  // largest g with mpp[g] <= q
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (tb.mpp[mid] <= q)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int g = lo;
+        const int mt = tb.mpp[g + 1] - tb.mpp[g];
+        const int64_t local = t - (int64_t)tb.mpp[g] * sc.nb_r;
+        const int nbi = (int)(local / mt), mb = (int)(local % mt);
+        ti.shared = false;
+        ti.g = ti.e = g;
+        ti.row0 = tb.off[g] + (int64_t)mb * (2 * kBM) + rank * kBM;
+        ti.arow = (int)ti.row0;
+        const int64_t left = tb.off[g + 1] - ti.row0;
+        ti.rows = left < kBM ? (int)left : kBM;
+        ti.n0 = nbi * BN;
+        ti.N = a.N;
+        ti.K = a.K;
+    } else {
+        const int64_t local = t - sc.routed_tiles;
+        const int nbi = (int)(local / sc.mt_s), mb = (int)(local % sc.mt_s);
+        ti.shared = true;
+        ti.g = sc.E;
+        ti.e = 0;
+        ti.arow = mb * (2 * kBM) + (int)rank * kBM;
+        ti.row0 = tb.off[sc.E] + ti.arow;
+        ti.rows = min(kBM, a.T - ti.arow);
+        ti.n0 = nbi * BN;
+        ti.N = a.Ns;
+        ti.K = a.Ks;
+    }
+}
+
+template <bool kGateUp>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+    const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+    const __grid_constant__ CUtensorMap tmBs0, const __grid_constant__ CUtensorMap tmBs1,
+    const GemmArgs a) {
+    constexpr int BN = kGateUp ? kBRows / 2 : kBRows;  // output columns per tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);  // used in the leader
+    uint64_t* empty = full + kPStages;
+    uint64_t* tfull = empty + kPStages;
+    uint64_t* tempty = tfull + 2;  // used in the leader: 4 epilogue warps x 2 CTAs
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    PairTables* tb = reinterpret_cast<PairTables*>(smem + kPStages * kPStageBytes + 256);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = (rank == 0);
+    for (int i = threadIdx.x; i < a.E + 2; i += kThreads) tb->off[i] = a.offsets[i];
+    for (int i = threadIdx.x; i < a.E + 1; i += kThreads) tb->mpp[i] = a.mtile_prefix[i];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 2 * (kEpiThreads / 32));
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    // both CTAs' barriers are initialised before any cross-CTA signal
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    Sched sc;
+    sc.E = a.E;
+    sc.nb_r = (a.N + BN - 1) / BN;
+    sc.nb_s = a.has_shared ? (a.Ns + BN - 1) / BN : 0;
+    sc.mt_s = a.has_shared ? (a.T + 2 * kBM - 1) / (2 * kBM) : 0;
+    sc.routed_tiles = (int64_t)tb->mpp[a.E] * sc.nb_r;
+    sc.total = sc.routed_tiles + (int64_t)sc.mt_s * sc.nb_s;
+    const int64_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t t = pair; t < sc.total && !*abort_flag; t += npairs) {
+                TileInfo ti;
+                decode_pair(t, *tb, sc, a, BN, rank, ti);
+                const CUtensorMap* mA = ti.shared ? &tmAs : &tmA;
+                const CUtensorMap* mB = kGateUp ? (ti.shared ? (rank ? &tmBs1 : &tmBs0) : (rank ? &tmB1 : &tmB0))
+                                                : (ti.shared ? &tmBs0 : &tmB0);
+                const int bcol = kGateUp ? ti.n0 : ti.n0 + (int)rank * (kBRows / 2);
+                const int nkb = (ti.K + kBK - 1) / kBK;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kPStages;
+                    const uint32_t ph = (it / kPStages) & 1;
+                    if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, a.flags)) break;
+                    uint8_t* sa = smem + s * kPStageBytes;
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * kPStageBytes);
+                    tma_load_3d_pair(sa, mA, &full[s], kb * kBK, ti.arow, 0);
+                    tma_load_3d_pair(sa + kPABytes, mB, &full[s], kb * kBK, bcol, ti.e);
+                }
+            }
+            // copies of both CTAs complete on the leader's barriers
+            if (leader)
+                for (uint32_t j = (it > (uint32_t)kPStages ? it - kPStages : 0); j < it; ++j)
+                    drain_wait(&full[j % kPStages], (j / kPStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && leader) {
+            uint32_t it = 0, tc = 0;
+            for (int64_t t = pair; t < sc.total && !*abort_flag; t += npairs, ++tc) {
+                TileInfo ti;
+                decode_pair(t, *tb, sc, a, BN, rank, ti);
+                const int nkb = (ti.K + kBK - 1) / kBK;
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!wait_or_abort(&tempty[acc], aph ^ 1, abort_flag, a.flags)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * kAccCols;
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kPStages;
+                    const uint32_t ph = (it / kPStages) & 1;
+                    if (!wait_or_abort(&full[s], ph, abort_flag, a.flags)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + s * kPStageBytes);
+                    const uint32_t b0 = a0 + kPABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_bf16_pair(d, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), kPIdesc,
+                                      (kb | kk) != 0);
+                    mma_commit_pair(&empty[s], 0x3);  // frees the stage in both CTAs
+                }
+                if (!ok) break;
+                mma_commit_pair(&tfull[acc], 0x3);  // both halves of the accumulator ready
+            }
+            mma_commit_pair(drain, 0x1);
+            drain_wait(drain, 0);
+        }
+    } else {
+        // ------------------------------------------------ epilogue warps 2..5 (both CTAs)
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        uint32_t tc = 0;
+        for (int64_t t = pair; t < sc.total; t += npairs, ++tc) {
+            TileInfo ti;
+            decode_pair(t, *tb, sc, a, BN, rank, ti);
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
+            tc_fence_after();
+            epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(&tempty[acc], 0);  // the leader's barrier
+        }
+    }
+
+    if (*abort_flag && !leader) {
+        // aborted: this CTA's copies complete on the leader's barriers; give
+        // any still in flight time to land before shared memory is released
+        for (int i = 0; i < 2000; ++i) __nanosleep(100);
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
 // ------------------------------------------------------------------ host side
@@ -362,6 +579,31 @@ cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const Ge
                                                                          maps[4], maps[5], args);
     return cudaGetLastError();
 }
+
+constexpr size_t kPSmemBytes = kPStages * kPStageBytes + 1024 + 256 + sizeof(PairTables);
+
+template <bool kGateUp>
+cudaError_t launch_grouped_pair(const Plan& p, const CUtensorMap (&maps)[6], const GemmArgs& args,
+                                cudaStream_t st) {
+    constexpr int BN = kGateUp ? kBRows / 2 : kBRows;
+    cudaError_t e = ensure_smem_attr(grouped_gemm_pair_kernel<kGateUp>, kPSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int64_t nb_r = (args.N + BN - 1) / BN;
+    const int64_t nb_s = args.has_shared ? (args.Ns + BN - 1) / BN : 0;
+    const int64_t ub = ((p.S + 2 * kBM - 1) / (2 * kBM) + p.E) * nb_r + ((p.T + 2 * kBM - 1) / (2 * kBM)) * nb_s;
+    const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, ub));
+    grouped_gemm_pair_kernel<kGateUp><<<(unsigned)(2 * pairs), kThreads, kPSmemBytes, st>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], args);
+    return cudaGetLastError();
+}
+
+// CTA pairs where they measured faster on B200: the down GEMM with a short
+// reduction (I <= 1024) and groups large enough (>= 512 kept rows per routed
+// expert on average) that 256-row tiles waste little.  Elsewhere single CTAs
+// were as fast or faster: in a pair each SM's tensor core still reads all of
+// B (its half from its own shared memory, the other half from the peer's),
+// so shared-memory traffic drops only by about a sixth.
+bool use_pairs(const Plan& p, bool gate_up) { return !gate_up && p.I <= 1024 && p.S >= 512 * p.E; }
 
 GemmArgs base_args(const Plan& p) {
     GemmArgs a{};
@@ -402,8 +644,10 @@ cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate
     a.K = a.Ks = (int)p.H;
     a.h = h;
     a.hs = hs;
+    const bool pairs = use_pairs(p, true);
+    if (pairs) a.mtile_prefix = p.mpair_prefix;
     trace_before("gateup_sm100", st);
-    cudaError_t e = launch_grouped<true>(p, m, a, st);
+    cudaError_t e = pairs ? launch_grouped_pair<true>(p, m, a, st) : launch_grouped<true>(p, m, a, st);
     trace_after(st);
     return e;
 }
@@ -414,9 +658,12 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     const bf16* h = (const bf16*)p.h;
     const bf16* hs = h + p.S * p.I;
     CUtensorMap m[6];
-    bool ok = make_map_bf16(&m[0], h, p.I, p.S, 1, kBK, kBM) && make_map_bf16(&m[2], w_down, p.I, p.H, p.E, kBK, kBRows);
+    // a CTA pair stages half of the 256 output columns per CTA
+    const bool pairs = use_pairs(p, false);
+    const uint32_t brows = pairs ? kBRows / 2 : kBRows;
+    bool ok = make_map_bf16(&m[0], h, p.I, p.S, 1, kBK, kBM) && make_map_bf16(&m[2], w_down, p.I, p.H, p.E, kBK, brows);
     if (ok && p.Is > 0)
-        ok = make_map_bf16(&m[1], hs, p.Is, p.T, 1, kBK, kBM) && make_map_bf16(&m[4], ws_down, p.Is, p.H, 1, kBK, kBRows);
+        ok = make_map_bf16(&m[1], hs, p.Is, p.T, 1, kBK, kBM) && make_map_bf16(&m[4], ws_down, p.Is, p.H, 1, kBK, brows);
     else {
         m[1] = m[0];
         m[4] = m[2];
@@ -433,8 +680,9 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     a.out = mode == 0 ? (float*)out : nullptr;
     a.rows = mode == 1 ? (bf16*)out : nullptr;
     a.mode = mode;
+    if (pairs) a.mtile_prefix = p.mpair_prefix;
     trace_before(mode ? "down_sm100_weighted" : "down_sm100", st);
-    cudaError_t e = launch_grouped<false>(p, m, a, st);
+    cudaError_t e = pairs ? launch_grouped_pair<false>(p, m, a, st) : launch_grouped<false>(p, m, a, st);
     trace_after(st);
     return e;
 }

@@ -119,6 +119,7 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->dropped = (int32_t*)take(sizeof(int32_t) * p->E);
     p->offsets = (int32_t*)take(sizeof(int32_t) * (p->E + 2));
     p->mtile_prefix = (int32_t*)take(sizeof(int32_t) * (p->E + 1));
+    p->mpair_prefix = (int32_t*)take(sizeof(int32_t) * (p->E + 1));
     p->perm_rows = (int32_t*)take(sizeof(int32_t) * p->S);
     p->row_of = (int32_t*)take(sizeof(int32_t) * p->S);
     p->xperm = take(elt * p->S * p->H);

@@ -64,20 +64,27 @@ __device__ __forceinline__ int32_t block_scan_256(int32_t v, int32_t* sm) {
     return r;
 }
 
-// m-tiles of kGemmTileRows rows per expert -> exclusive prefix mtile_prefix[0..E].
-__device__ __forceinline__ void write_mtile_prefix(int32_t kept, int E, int32_t* sm,
-                                                   int32_t* mtile_prefix) {
+// Tiles of `rows_per_tile` rows per expert -> exclusive prefix prefix[0..E].
+__device__ __forceinline__ void write_tile_prefix(int32_t kept, int E, int32_t* sm, int rows_per_tile,
+                                                  int32_t* prefix) {
     const int e = threadIdx.x;
-    int32_t mt = (e < E) ? (kept + kGemmTileRows - 1) / kGemmTileRows : 0;
+    int32_t mt = (e < E) ? (kept + rows_per_tile - 1) / rows_per_tile : 0;
     int32_t incl = block_scan_256(mt, sm);
-    if (e < E) mtile_prefix[e] = incl - mt;
-    if (e == E - 1) mtile_prefix[E] = incl;
+    if (e < E) prefix[e] = incl - mt;
+    if (e == E - 1) prefix[E] = incl;
+}
+
+// Both tile prefixes of the grouped GEMMs: 128-row tiles and 256-row CTA-pair tiles.
+__device__ __forceinline__ void write_mtile_prefix(int32_t kept, int E, int32_t* sm, int32_t* mtile_prefix,
+                                                   int32_t* mpair_prefix) {
+    write_tile_prefix(kept, E, sm, kGemmTileRows, mtile_prefix);
+    write_tile_prefix(kept, E, sm, 2 * kGemmTileRows, mpair_prefix);
 }
 
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(
     int32_t* __restrict__ hist, int64_t nchunks, int E, int64_t cap, int32_t* __restrict__ counts,
     int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
-    int32_t* __restrict__ mtile_prefix, int32_t shared_rows) {
+    int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix, int32_t shared_rows) {
     __shared__ int32_t kept_s[kScanThreads];
     const int e = threadIdx.x;
     int32_t total = 0;
@@ -114,7 +121,7 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(
         offsets_ws[E + 1] = R + shared_rows;
         offsets_out[E] = R;
     }
-    write_mtile_prefix(e < E ? kept : 0, E, kept_s, mtile_prefix);
+    write_mtile_prefix(e < E ? kept : 0, E, kept_s, mtile_prefix, mpair_prefix);
 }
 
 __global__ void __launch_bounds__(kScatterWarps * 32) permute_scatter_kernel(
@@ -164,12 +171,12 @@ __global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_
 
 __global__ void __launch_bounds__(kScanThreads) offsets_from_user_kernel(
     const int32_t* __restrict__ user, int E, int32_t shared_rows, int32_t* __restrict__ ws_off,
-    int32_t* __restrict__ mtile_prefix) {
+    int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix) {
     __shared__ int32_t sm[kScanThreads];
     const int e = threadIdx.x;
     if (e <= E) ws_off[e] = user[e];
     if (e == 0) ws_off[E + 1] = user[E] + shared_rows;
-    write_mtile_prefix(e < E ? user[e + 1] - user[e] : 0, E, sm, mtile_prefix);
+    write_mtile_prefix(e < E ? user[e + 1] - user[e] : 0, E, sm, mtile_prefix, mpair_prefix);
 }
 
 }  // namespace
@@ -178,7 +185,7 @@ cudaError_t launch_offsets_from_user(const Plan& p, const int32_t* offsets, cuda
     trace_before("offsets_from_user", st);
     offsets_from_user_kernel<<<1, kScanThreads, 0, st>>>(offsets, (int)p.E,
                                                          (int32_t)(p.Is > 0 ? p.T : 0), p.offsets,
-                                                         p.mtile_prefix);
+                                                         p.mtile_prefix, p.mpair_prefix);
     trace_after(st);
     return cudaGetLastError();
 }
@@ -198,6 +205,7 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
             e1 = cudaMemsetAsync(p.offsets + p.E, 0, sizeof(int32_t) * 2, st);
         }
         if (e1 == cudaSuccess) e1 = cudaMemsetAsync(p.mtile_prefix, 0, sizeof(int32_t) * (p.E + 1), st);
+        if (e1 == cudaSuccess) e1 = cudaMemsetAsync(p.mpair_prefix, 0, sizeof(int32_t) * (p.E + 1), st);
         return e1;
     }
     const int E = (int)p.E;
@@ -208,7 +216,7 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
     trace_before("permute_scan", st);
     permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
         p.chunk_base, p.nchunks, E, p.cap, counts, dropped, offsets, p.offsets, p.mtile_prefix,
-        (int32_t)(p.Is > 0 ? p.T : 0));
+        p.mpair_prefix, (int32_t)(p.Is > 0 ? p.T : 0));
     trace_after(st);
     trace_before("permute_scatter", st);
     unsigned blocks = (unsigned)((p.nchunks + kScatterWarps - 1) / kScatterWarps);
@@ -234,7 +242,7 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
 namespace {
 
 constexpr int64_t kNoAllocChunks = kNoAllocMaxSlots / kPermuteChunk;
-constexpr int64_t kNoAllocInts = kNoAllocChunks * kMaxExperts + 2 * (kMaxExperts + 2) + 64;
+constexpr int64_t kNoAllocInts = kNoAllocChunks * kMaxExperts + 3 * (kMaxExperts + 2) + 64;
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocInts];
 
@@ -273,7 +281,8 @@ cudaError_t launch_permute_noalloc(const Plan& sizes, const int32_t* topk_idx, i
     p.chunk_base = scratch;                                 // [kNoAllocChunks * E]
     p.offsets = scratch + kNoAllocChunks * kMaxExperts;     // [E + 2]
     p.mtile_prefix = p.offsets + (kMaxExperts + 2);         // [E + 1]
-    p.flags = p.offsets + 2 * (kMaxExperts + 2);            // flag word, cleared per call
+    p.mpair_prefix = p.offsets + 2 * (kMaxExperts + 2);     // [E + 1]
+    p.flags = p.offsets + 3 * (kMaxExperts + 2);            // flag word, cleared per call
     e = cudaMemsetAsync(p.flags, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return e;
     return launch_permute(p, topk_idx, counts, offsets, perm_rows, row_of, dropped, st);

@@ -103,6 +103,25 @@ def test_layer_tensor_core_router(gpu_lib, wl):
     check_layer(gpu_lib, wl)
 
 
+# The down GEMM runs on CTA pairs (256-row tiles) when I <= 1024 and the
+# routed groups average at least 512 kept rows (T*k >= 512*E), else on single
+# CTAs.  These cases take the pair path at sizes the oracle evaluates in full: ragged
+# groups (odd numbers of 128-row halves), a shared expert, capacity drops and
+# an output width that is not a multiple of 256.
+PAIRS = [
+    mi.Workload("pairs_basic", T=2300, H=512, I=384, E=4, k=2),
+    mi.Workload("pairs_shared_ragged", T=1337, H=520, I=200, E=2, k=1, I_shared=136),
+    mi.Workload("pairs_capacity", T=2100, H=256, I=256, E=4, k=2, capacity_factor=1.1),
+    mi.Workload("pairs_zipf_k4", T=1600, H=384, I=128, E=8, k=4, zipf_s=1.1),
+]
+
+
+@pytest.mark.parametrize("wl", PAIRS, ids=[w.name for w in PAIRS])
+def test_layer_cta_pairs(gpu_lib, wl):
+    assert wl.T * wl.k >= 512 * wl.E and wl.I <= 1024
+    check_layer(gpu_lib, wl)
+
+
 def test_all_tokens_to_one_expert(gpu_lib):
     """A router bias that sends every token to experts 0 and 1."""
     wl = mi.Workload("skew", T=400, H=128, I=64, E=8, k=2, zipf_s=0.0)
@@ -140,7 +159,8 @@ def stage_setup(moe, wl):
 
 
 @pytest.mark.parametrize("wl", [mi.SMALL["fine_grained_e256_layer"], mi.SMALL["qwen3_30b_a3b_layer"],
-                                mi.TINY, TC_ROUTER[0]], ids=["fine_small", "qwen3_small", "tiny", "tc_router"])
+                                mi.TINY, TC_ROUTER[0], PAIRS[1]],
+                         ids=["fine_small", "qwen3_small", "tiny", "tc_router", "pairs"])
 def test_stages_route_permute_ffn_combine(gpu_lib, wl):
     moe = gpu_lib
     inp, d, cfg, ws = stage_setup(moe, wl)
