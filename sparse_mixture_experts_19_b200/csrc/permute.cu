@@ -169,6 +169,81 @@ __global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_
         perm_rows[r] = -1;
 }
 
+// All of the grouping in one CTA when the slots fit one chunk (S <= 2048):
+// histogram, capacity cut and scans (phase 2 as in permute_scan_kernel with a
+// single chunk), then warp 0 scatters the slots in order while the other
+// warps mark the unused tail of perm_rows.  Same outputs, one launch.
+__global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
+    const int32_t* __restrict__ idx, int S, int E, int64_t cap, int32_t* __restrict__ counts,
+    int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
+    int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix, int32_t shared_rows,
+    int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of, int32_t* __restrict__ flags) {
+    __shared__ int32_t hist[kScanThreads];
+    __shared__ int32_t sm[kScanThreads];
+    __shared__ int32_t off[kScanThreads + 1];
+    const int e = threadIdx.x;
+    hist[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int s = threadIdx.x; s < S; s += kScanThreads) {
+        const int ex = idx[s];
+        if (ex >= 0 && ex < E)
+            atomicAdd(&hist[ex], 1);
+        else
+            bad = true;
+    }
+    if (bad) set_flag(flags, MOE_DEVFLAG_BAD_EXPERT_INDEX);
+    __syncthreads();
+    const int32_t total = (e < E) ? hist[e] : 0;
+    const int32_t kept = (cap > 0 && total > cap) ? (int32_t)cap : total;
+    if (e < E) {
+        counts[e] = total;
+        dropped[e] = total - kept;
+    }
+    const int32_t incl = block_scan_256(kept, sm);
+    if (e < E) {
+        off[e] = incl - kept;
+        offsets_ws[e] = incl - kept;
+        offsets_out[e] = incl - kept;
+    }
+    if (e == E - 1) {
+        off[E] = incl;
+        offsets_ws[E] = incl;
+        offsets_ws[E + 1] = incl + shared_rows;
+        offsets_out[E] = incl;
+    }
+    write_mtile_prefix(kept, E, sm, mtile_prefix, mpair_prefix);
+    hist[e] = 0;  // running count of each expert's rows in slot order
+    __syncthreads();
+    const int R = off[E];
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const uint32_t lt = (1u << lane) - 1u;
+        for (int sb = 0; sb < S; sb += 32) {
+            const int s = sb + lane;
+            const int ex = (s < S) ? idx[s] : -1;
+            const bool valid = (ex >= 0 && ex < E);
+            const uint32_t peers = __match_any_sync(0xffffffffu, valid ? ex : -1);
+            int32_t rank = 0;
+            if (valid) rank = hist[ex] + __popc(peers & lt);
+            __syncwarp();
+            if (valid && (peers & lt) == 0) hist[ex] += __popc(peers);
+            __syncwarp();
+            if (s < S) {
+                if (valid && (cap <= 0 || rank < cap)) {
+                    const int32_t row = off[ex] + rank;
+                    perm_rows[row] = s;
+                    row_of[s] = row;
+                } else {
+                    row_of[s] = -1;
+                }
+            }
+        }
+    } else {
+        for (int r = R + (int)threadIdx.x - 32; r < S; r += kScanThreads - 32) perm_rows[r] = -1;
+    }
+}
+
 __global__ void __launch_bounds__(kScanThreads) offsets_from_user_kernel(
     const int32_t* __restrict__ user, int E, int32_t shared_rows, int32_t* __restrict__ ws_off,
     int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix) {
@@ -209,6 +284,14 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
         return e1;
     }
     const int E = (int)p.E;
+    if (p.nchunks == 1) {
+        trace_before("permute_small", st);
+        permute_small_kernel<<<1, kScanThreads, 0, st>>>(topk_idx, (int)p.S, E, p.cap, counts, dropped, offsets,
+                                                         p.offsets, p.mtile_prefix, p.mpair_prefix,
+                                                         (int32_t)(p.Is > 0 ? p.T : 0), perm_rows, row_of, p.flags);
+        trace_after(st);
+        return cudaGetLastError();
+    }
     trace_before("permute_hist", st);
     permute_hist_kernel<<<(unsigned)p.nchunks, kHistThreads, 0, st>>>(topk_idx, p.S, E,
                                                                        p.chunk_base, p.flags);

@@ -5,18 +5,18 @@
 //
 // With few tokens the router is a matrix-vector product per token: the
 // weights (E x H) stay in L2 and every SM can work on its own token.  One CTA
-// per token: its 8 warps split the experts, the 32 lanes of a warp split H in
-// 16-byte chunks, and each score is accumulated in fp64 (every product of two
-// bf16 or float32 values is exact in fp64, so the scores are the exact sums up
-// to fp64 rounding and the selection matches an fp64 reference except for
-// ties closer than that).  Warp 0 then picks the k best by (score desc,
+// per token: its 32 warps split the experts, the 32 lanes of a warp split H in
+// 16-byte chunks (four in flight per lane), and each score is accumulated in
+// fp64 (every product of two bf16 or float32 values is exact in fp64, so the
+// scores are the exact sums up to fp64 rounding and the selection matches an
+// fp64 reference except for ties closer than that).  Warp 0 then picks the k best by (score desc,
 // index asc) with warp arg-max rounds and writes the softmax of those k.
 #include "common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 32;
 
 template <typename TIn>
 __device__ __forceinline__ void widen16(const uint4& q, double* out) {
@@ -48,25 +48,26 @@ __global__ void __launch_bounds__(kWarps * 32) router_decode_kernel(
 
     for (int e = warp; e < E; e += kWarps) {
         const uint4* wrow = reinterpret_cast<const uint4*>(wr + (int64_t)e * H);
-        double acc[2] = {0.0, 0.0};
-        for (int c = lane; c < nch; c += 64) {
-            uint4 xa = xr[c], wa = wrow[c];
-            uint4 xb = make_uint4(0, 0, 0, 0), wb = make_uint4(0, 0, 0, 0);
-            if (c + 32 < nch) {
-                xb = xr[c + 32];
-                wb = wrow[c + 32];
+        // four 16-byte chunks per lane in flight, four accumulators
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int c = lane; c < nch; c += 128) {
+            uint4 xq[4], wq[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int cu = c + 32 * u;
+                xq[u] = cu < nch ? xr[cu] : make_uint4(0, 0, 0, 0);
+                wq[u] = cu < nch ? wrow[cu] : make_uint4(0, 0, 0, 0);
             }
-            double fx[V], fw[V];
-            widen16<TIn>(xa, fx);
-            widen16<TIn>(wa, fw);
 #pragma unroll
-            for (int i = 0; i < V; ++i) acc[0] = fma(fx[i], fw[i], acc[0]);
-            widen16<TIn>(xb, fx);
-            widen16<TIn>(wb, fw);
+            for (int u = 0; u < 4; ++u) {
+                double fx[V], fw[V];
+                widen16<TIn>(xq[u], fx);
+                widen16<TIn>(wq[u], fw);
 #pragma unroll
-            for (int i = 0; i < V; ++i) acc[1] = fma(fx[i], fw[i], acc[1]);
+                for (int i = 0; i < V; ++i) acc[u] = fma(fx[i], fw[i], acc[u]);
+            }
         }
-        double s = acc[0] + acc[1];
+        double s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (lane == 0) sc[e] = s + (b ? (double)b[e] : 0.0);
