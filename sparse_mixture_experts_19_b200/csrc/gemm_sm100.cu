@@ -18,9 +18,12 @@
 //
 // Groups: 0..E-1 routed experts (rows offsets[g]..offsets[g+1] of the
 // grouped activations), group E the shared expert (token rows of x / hs).
-// A tile is 128 rows x BN columns of one group; tiles of one expert are
-// ordered m-fastest inside each weight column block so CTAs running side by
-// side share the same weight slice through L2.
+// A tile is 128 rows x BN columns of one group.  Tiles of one group run in
+// bands of gm row tiles: a band visits every weight column block, m-fastest
+// inside each block, before the next band starts.  CTAs running side by side
+// then share one weight slice through L2, and the band's activation rows
+// (gm x 128 x K, about 32 MB) stay in L2 across the column blocks instead of
+// being read from HBM once per block when a group has many rows.
 //
 // Persistent CTA per SM, 192 threads: warp 0 issues TMA loads into a 4-stage
 // shared-memory ring, warp 1 issues tcgen05.mma (one thread) and owns the
@@ -77,8 +80,28 @@ struct Tables {
 
 struct Sched {
     int E, nb_r, nb_s, mt_s;
+    int gm_r, gm_s;  // row tiles per band (routed, shared)
     int64_t routed_tiles, total;
 };
+
+// Row tiles per band: as many 128-row A tiles of length K as fit in about
+// 32 MB of L2 (at least 8).
+__host__ __device__ __forceinline__ int band_tiles(int K, int rows_per_tile) {
+    const int64_t per = (int64_t)rows_per_tile * (K > 0 ? K : 1) * 2;
+    const int64_t g = (32ll << 20) / per;
+    return g < 8 ? 8 : (g > (1 << 20) ? (1 << 20) : (int)g);
+}
+
+// Position `local` of a group's tile list (mt row tiles x nb column blocks,
+// bands of gm row tiles) -> (column block, row tile).
+__device__ __forceinline__ void band_order(int64_t local, int mt, int nb, int gm, int& nbi, int& mb) {
+    const int64_t band = local / ((int64_t)gm * nb);
+    const int64_t rem = local - band * gm * nb;
+    const int first = (int)band * gm;
+    const int width = min(gm, mt - first);
+    nbi = (int)(rem / width);
+    mb = first + (int)(rem % width);
+}
 
 struct TileInfo {
     bool shared;
@@ -103,7 +126,8 @@ __device__ __forceinline__ void decode_tile(int64_t t, const Tables& tb, const S
         const int g = lo;
         const int mt = tb.mtp[g + 1] - tb.mtp[g];
         const int64_t local = t - (int64_t)tb.mtp[g] * sc.nb_r;
-        const int nbi = (int)(local / mt), mb = (int)(local % mt);
+        int nbi, mb;
+        band_order(local, mt, sc.nb_r, sc.gm_r, nbi, mb);
         ti.shared = false;
         ti.g = ti.e = g;
         ti.row0 = tb.off[g] + (int64_t)mb * kBM;
@@ -115,7 +139,8 @@ __device__ __forceinline__ void decode_tile(int64_t t, const Tables& tb, const S
         ti.K = a.K;
     } else {
         const int64_t local = t - sc.routed_tiles;
-        const int nbi = (int)(local / sc.mt_s), mb = (int)(local % sc.mt_s);
+        int nbi, mb;
+        band_order(local, sc.mt_s, sc.nb_s, sc.gm_s, nbi, mb);
         ti.shared = true;
         ti.g = sc.E;
         ti.e = 0;
@@ -256,6 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
     sc.nb_r = (a.N + BN - 1) / BN;
     sc.nb_s = a.has_shared ? (a.Ns + BN - 1) / BN : 0;
     sc.mt_s = a.has_shared ? (a.T + kBM - 1) / kBM : 0;
+    sc.gm_r = band_tiles(a.K, kBM);
+    sc.gm_s = band_tiles(a.Ks, kBM);
     sc.routed_tiles = (int64_t)tb->mtp[a.E] * sc.nb_r;
     sc.total = sc.routed_tiles + (int64_t)sc.mt_s * sc.nb_s;
 
@@ -391,7 +418,8 @@ __device__ __forceinline__ void decode_pair(int64_t t, const PairTables& tb, con
         const int g = lo;
         const int mt = tb.mpp[g + 1] - tb.mpp[g];
         const int64_t local = t - (int64_t)tb.mpp[g] * sc.nb_r;
-        const int nbi = (int)(local / mt), mb = (int)(local % mt);
+        int nbi, mb;
+        band_order(local, mt, sc.nb_r, sc.gm_r, nbi, mb);
         ti.shared = false;
         ti.g = ti.e = g;
         ti.row0 = tb.off[g] + (int64_t)mb * (2 * kBM) + rank * kBM;
@@ -403,7 +431,8 @@ __device__ __forceinline__ void decode_pair(int64_t t, const PairTables& tb, con
         ti.K = a.K;
     } else {
         const int64_t local = t - sc.routed_tiles;
-        const int nbi = (int)(local / sc.mt_s), mb = (int)(local % sc.mt_s);
+        int nbi, mb;
+        band_order(local, sc.mt_s, sc.nb_s, sc.gm_s, nbi, mb);
         ti.shared = true;
         ti.g = sc.E;
         ti.e = 0;
@@ -467,6 +496,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
     sc.nb_r = (a.N + BN - 1) / BN;
     sc.nb_s = a.has_shared ? (a.Ns + BN - 1) / BN : 0;
     sc.mt_s = a.has_shared ? (a.T + 2 * kBM - 1) / (2 * kBM) : 0;
+    sc.gm_r = band_tiles(a.K, 2 * kBM);
+    sc.gm_s = band_tiles(a.Ks, 2 * kBM);
     sc.routed_tiles = (int64_t)tb->mpp[a.E] * sc.nb_r;
     sc.total = sc.routed_tiles + (int64_t)sc.mt_s * sc.nb_s;
     const int64_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
