@@ -198,7 +198,13 @@ moe_status_t moe_combine(const moe_config_t* cfg, const float* expert_out, const
  * rounded once to the layer dtype.
  *   y [T,H] (layer dtype).  Optional outputs (NULL to skip): topk_idx_out
  *   [T,top_k] int32, counts_out [E] and dropped_out [E] int32.
- * y is bit-reproducible for given inputs (no atomics, fixed summation order).
+ * With T*top_k <= 8 (bf16) no rows are grouped: two weight-streaming
+ * kernels read each selected expert's weight rows once and sum each
+ * token's k weighted FFN outputs (then the shared expert's) in float32 in
+ * slot order, rounded once; the routed outputs are not rounded to bf16
+ * before that sum.
+ * y is bit-reproducible for given inputs (fixed summation order; the only
+ * atomics are arrival counters that pick which warp does a fixed-order sum).
  */
 moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* router_w,
                          const float* router_b, const void* w_gate, const void* w_up,

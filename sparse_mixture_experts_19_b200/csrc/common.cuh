@@ -17,6 +17,7 @@ constexpr int kPermuteChunk = 2048;  // slots per histogram chunk in moe_permute
 constexpr int kWsAlign = 256;
 constexpr int kGemmTileRows = 128;  // rows per tile of the tcgen05 grouped GEMMs
 constexpr int64_t kNoAllocMaxSlots = 1 << 20;  // T*k limit of moe_permute_noalloc
+constexpr int kDecodeMaxSlots = 8;             // T*k limit of the decode FFN kernels
 
 // Everything the kernels of one call need, carved out of the caller's workspace.
 struct Plan {
@@ -41,6 +42,8 @@ struct Plan {
     void* xperm;          // [S, H] layer dtype: x rows in grouped order
     void* h;              // [S, I] + [T, Is] layer dtype: SwiGLU activations
     void* rows;           // [S + T, H] layer dtype: routing-weighted expert output rows
+    float* dec_part;      // decode FFN (S <= kDecodeMaxSlots): [H, S + T] partial dot products
+    int32_t* dec_cnt;     // decode FFN: [H] arrivals per output column
     size_t bytes;         // total workspace bytes
 };
 
@@ -72,6 +75,13 @@ cudaError_t launch_router_decode(const Plan& p, const void* x, const void* route
 // Scores of T*E*H at most this many multiply-adds go to the per-token router
 // (its weight traffic, T*E*H*2 bytes from L2, stays small).
 constexpr int64_t kDecodeRouterMaxMacs = int64_t(1) << 26;
+// Decode FFN (bf16, T*k <= kDecodeMaxSlots): expert FFNs and the weighted
+// combine as two weight-streaming kernels, y written directly; also writes
+// counts and dropped.
+bool decode_ffn_eligible(const Plan& p);
+cudaError_t launch_decode_ffn(const Plan& p, const void* x, const int32_t* topk_idx, const void* w_gate,
+                              const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                              const void* ws_down, void* y, int32_t* counts, int32_t* dropped, cudaStream_t st);
 cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
                            int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
                            int32_t* dropped, cudaStream_t st);

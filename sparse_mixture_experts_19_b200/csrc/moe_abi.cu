@@ -125,6 +125,9 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->xperm = take(elt * p->S * p->H);
     p->h = take(elt * (p->S * p->I + p->T * p->Is));
     p->rows = take(elt * (p->S + (p->Is ? p->T : 0)) * p->H);
+    const int64_t dec_cols = p->S <= kDecodeMaxSlots ? p->S + (p->Is ? p->T : 0) : 0;
+    p->dec_part = (float*)take(sizeof(float) * p->H * dec_cols);
+    p->dec_cnt = (int32_t*)take(dec_cols ? sizeof(int32_t) * p->H : 0);
     p->bytes = off;
 }
 
@@ -346,6 +349,12 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
     CUDA_TRY(run_router(p, x, router_w, router_b, idx, p.topk_w, st), "router");
+    if (decode_ffn_eligible(p)) {
+        // few slots: weight-streaming FFN kernels, no grouped rows
+        CUDA_TRY(launch_decode_ffn(p, x, idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, counts, dropped, st),
+                 "decode_ffn");
+        return MOE_OK;
+    }
     CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
     if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.rows, st)) != MOE_OK)
         return s;

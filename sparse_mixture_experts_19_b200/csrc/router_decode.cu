@@ -1,54 +1,75 @@
-// Router for few tokens (decode): exact fp64 scores, warp top-k, softmax.
+// Router for few tokens (decode): exact scores, warp top-k, softmax.
 //
 // "MoE稀疏架构是什么？从原理到落地的系统解读", section 三.1 (a small linear
 // router scores every expert) and section 四 (top-k, softmax over the k).
 //
-// With few tokens the router is a matrix-vector product per token: the
-// weights (E x H) stay in L2 and every SM can work on its own token.  One CTA
-// per token: its 32 warps split the experts, the 32 lanes of a warp split H in
-// 16-byte chunks (four in flight per lane), and each score is accumulated in
-// fp64 (every product of two bf16 or float32 values is exact in fp64, so the
-// scores are the exact sums up to fp64 rounding and the selection matches an
-// fp64 reference except for ties closer than that).  Warp 0 then picks the k best by (score desc,
-// index asc) with warp arg-max rounds and writes the softmax of those k.
+// With few tokens the router is a matrix-vector product per token.  Each
+// token gets a thread-block cluster of C CTAs (C <= 8); CTA r scores experts
+// [r*epc, (r+1)*epc) with one warp per expert at a time, the 32 lanes of a
+// warp splitting H in 16-byte chunks (four in flight per lane).  Scores are
+// exact up to fp64 rounding: for bf16 inputs each product of two bf16 values
+// is exact in float32 (8-bit by 8-bit significands, for |product| in
+// [2^-126, 2^128)) and is summed in fp64; float32 inputs are multiplied in
+// fp64.  So the selection matches an fp64 reference except for ties closer
+// than that.  After a cluster barrier, warp 0 of CTA 0 gathers all E scores
+// through distributed shared memory, picks the k best by (score desc, index
+// asc) with warp arg-max rounds and writes the softmax of those k; a second
+// cluster barrier keeps the other CTAs' shared memory alive until then.
+#include <algorithm>
+
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kWarps = 32;
+using namespace sm100;
 
-template <typename TIn>
-__device__ __forceinline__ void widen16(const uint4& q, double* out) {
-    if constexpr (sizeof(TIn) == 2) {
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+constexpr int kWarps = 8;
+constexpr int kMaxCluster = 8;
+constexpr int kExpertsPerWarpRound = kWarps;
+
+__device__ __forceinline__ double ld_dsmem_f64(uint32_t addr) {
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// x . w over one 16-byte chunk, added to acc (fp64).
+__device__ __forceinline__ void chunk_dot(const uint4& xq, const uint4& wq, double& acc, __nv_bfloat16) {
+    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xq);
+    const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&wq);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float2 f = __bfloat1622float2(p[i]);
-            out[2 * i] = f.x;
-            out[2 * i + 1] = f.y;
-        }
-    } else {
-        const float* p = reinterpret_cast<const float*>(&q);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) out[i] = p[i];
+    for (int i = 0; i < 4; ++i) {
+        const float2 xf = __bfloat1622float2(xp[i]);
+        const float2 wf = __bfloat1622float2(wp[i]);
+        // exact float32 products, summed in fp64
+        acc += (double)__fmul_rn(xf.x, wf.x);
+        acc += (double)__fmul_rn(xf.y, wf.y);
     }
+}
+__device__ __forceinline__ void chunk_dot(const uint4& xq, const uint4& wq, double& acc, float) {
+    const float* xp = reinterpret_cast<const float*>(&xq);
+    const float* wp = reinterpret_cast<const float*>(&wq);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc = fma((double)xp[i], (double)wp[i], acc);
 }
 
 template <typename TIn>
 __global__ void __launch_bounds__(kWarps * 32) router_decode_kernel(
-    int T, int H, int E, int k, const TIn* __restrict__ x, const TIn* __restrict__ wr,
+    int T, int H, int E, int k, int C, int epc, const TIn* __restrict__ x, const TIn* __restrict__ wr,
     const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     constexpr int V = 16 / sizeof(TIn);  // elements per 16-byte chunk
-    __shared__ double sc[kMaxExperts];
-    const int t = blockIdx.x;
+    __shared__ double sc[kMaxExperts];   // this CTA's scores; CTA 0 gathers all E here
+    const int t = blockIdx.x / C;  // clusters of C consecutive CTAs along x, one per token
+    const uint32_t rank = cluster_ctarank();
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int nch = H / V;
     const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
+    const int e0 = (int)rank * epc, e1 = min(E, e0 + epc);
 
-    for (int e = warp; e < E; e += kWarps) {
+    for (int e = e0 + warp; e < e1; e += kExpertsPerWarpRound) {
         const uint4* wrow = reinterpret_cast<const uint4*>(wr + (int64_t)e * H);
-        // four 16-byte chunks per lane in flight, four accumulators
         double acc[4] = {0.0, 0.0, 0.0, 0.0};
         for (int c = lane; c < nch; c += 128) {
             uint4 xq[4], wq[4];
@@ -59,62 +80,86 @@ __global__ void __launch_bounds__(kWarps * 32) router_decode_kernel(
                 wq[u] = cu < nch ? wrow[cu] : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                double fx[V], fw[V];
-                widen16<TIn>(xq[u], fx);
-                widen16<TIn>(wq[u], fw);
-#pragma unroll
-                for (int i = 0; i < V; ++i) acc[u] = fma(fx[i], fw[i], acc[u]);
-            }
+            for (int u = 0; u < 4; ++u) chunk_dot(xq[u], wq[u], acc[u], TIn());
         }
         double s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) sc[e] = s + (b ? (double)b[e] : 0.0);
+        if (lane == 0) sc[e - e0] = s + (b ? (double)b[e] : 0.0);
     }
-    __syncthreads();
-    if (warp != 0) return;
-
-    // k rounds of warp arg-max; round j takes the best ranking after pick j-1
-    double pv = INFINITY;
-    int pe = -1;
-    double sel_v[kMaxTopK];
-    int sel_e[kMaxTopK];
-    for (int j = 0; j < k; ++j) {
-        double bv = -INFINITY;
-        int be = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            const double v = sc[e];
-            const bool after = (v < pv) || (v == pv && e > pe);
-            if (after && (v > bv || (v == bv && e < be))) {
-                bv = v;
-                be = e;
-            }
+    cluster_sync();
+    if (rank == 0 && warp == 0) {
+        // gather the other CTAs' scores behind this CTA's own (same offsets)
+        for (int e = epc + lane; e < E; e += 32) {
+            const uint32_t r = (uint32_t)(e / epc);
+            sc[e] = ld_dsmem_f64(mapa_shared(smem_u32(&sc[e - (int)r * epc]), r));
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (ov > bv || (ov == bv && oe < be)) {
-                bv = ov;
-                be = oe;
-            }
-        }
-        sel_v[j] = bv;
-        sel_e[j] = be;
-        pv = bv;
-        pe = be;
-    }
-    if (lane == 0) {
-        // softmax over the k selected, differences taken in fp64
-        float z = 0.f;
-        for (int j = 0; j < k; ++j) z += expf((float)(sel_v[j] - sel_v[0]));
-        const float inv = 1.0f / z;
+        __syncwarp();
+        // k rounds of warp arg-max; round j takes the best ranking after pick j-1
+        double pv = INFINITY;
+        int pe = -1;
+        double sel_v[kMaxTopK];
+        int sel_e[kMaxTopK];
         for (int j = 0; j < k; ++j) {
-            topk_idx[(int64_t)t * k + j] = sel_e[j];
-            topk_w[(int64_t)t * k + j] = expf((float)(sel_v[j] - sel_v[0])) * inv;
+            double bv = -INFINITY;
+            int be = 0x7fffffff;
+            for (int e = lane; e < E; e += 32) {
+                const double v = sc[e];
+                const bool after = (v < pv) || (v == pv && e > pe);
+                if (after && (v > bv || (v == bv && e < be))) {
+                    bv = v;
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (ov > bv || (ov == bv && oe < be)) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            sel_v[j] = bv;
+            sel_e[j] = be;
+            pv = bv;
+            pe = be;
+        }
+        if (lane == 0) {
+            // softmax over the k selected, differences taken in fp64
+            float z = 0.f;
+            for (int j = 0; j < k; ++j) z += expf((float)(sel_v[j] - sel_v[0]));
+            const float inv = 1.0f / z;
+            for (int j = 0; j < k; ++j) {
+                topk_idx[(int64_t)t * k + j] = sel_e[j];
+                topk_w[(int64_t)t * k + j] = expf((float)(sel_v[j] - sel_v[0])) * inv;
+            }
         }
     }
+    cluster_sync();  // CTA 0 has read every CTA's scores
+}
+
+template <typename TIn>
+cudaError_t launch_typed(const Plan& p, const void* x, const void* router_w, const float* router_b,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+    // C CTAs per token, each scoring epc experts (at most 8 per warp round)
+    const int E = (int)p.E;
+    const int C = std::min(kMaxCluster, (E + kExpertsPerWarpRound - 1) / kExpertsPerWarpRound);
+    const int epc = (E + C - 1) / C;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(C * p.T), 1, 1);
+    cfg.blockDim = dim3(kWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, router_decode_kernel<TIn>, (int)p.T, (int)p.H, E, (int)p.k, C, epc,
+                              (const TIn*)x, (const TIn*)router_w, router_b, topk_idx, topk_w);
 }
 
 }  // namespace
@@ -123,15 +168,10 @@ cudaError_t launch_router_decode(const Plan& p, const void* x, const void* route
                                  int32_t* topk_idx, float* topk_w, cudaStream_t st) {
     if (p.T == 0) return cudaSuccess;
     trace_before("router_decode", st);
-    if (p.bf16)
-        router_decode_kernel<bf16><<<(unsigned)p.T, kWarps * 32, 0, st>>>(
-            (int)p.T, (int)p.H, (int)p.E, (int)p.k, (const bf16*)x, (const bf16*)router_w, router_b, topk_idx,
-            topk_w);
-    else
-        router_decode_kernel<float><<<(unsigned)p.T, kWarps * 32, 0, st>>>(
-            (int)p.T, (int)p.H, (int)p.E, (int)p.k, (const float*)x, (const float*)router_w, router_b,
-            topk_idx, topk_w);
+    cudaError_t e = p.bf16 ? launch_typed<bf16>(p, x, router_w, router_b, topk_idx, topk_w, st)
+                           : launch_typed<float>(p, x, router_w, router_b, topk_idx, topk_w, st);
     trace_after(st);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -74,6 +74,43 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return false;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps until it completes or about hint_ns pass, instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// wait_or_abort for roles that may wait long while other warps of the SM
+// compute: sleeps in try_wait (hint 20 us) so waiting costs no issue slots,
+// and gives up after about 2 s of global time.
+__device__ __forceinline__ bool wait_sleep_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                    int32_t* flags, int32_t timeout_bit = 0x2) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > 2000000000ull) break;
+    }
+    *abort_flag = 1;
+    atomicOr(flags, timeout_bit);
+    return false;
+}
+
 // Unbounded-by-abort but still bounded wait used to drain in-flight work.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar, parity); ++i) {
@@ -94,6 +131,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// 1-D bulk copy global -> shared of `bytes` bytes (a multiple of 16; both
+// addresses 16-byte aligned), counted on bar's transaction bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
 // -------------------------------------------------------------- tcgen05

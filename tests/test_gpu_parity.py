@@ -122,15 +122,40 @@ def test_layer_cta_pairs(gpu_lib, wl):
     check_layer(gpu_lib, wl)
 
 
-def test_all_tokens_to_one_expert(gpu_lib):
-    """A router bias that sends every token to experts 0 and 1."""
-    wl = mi.Workload("skew", T=400, H=128, I=64, E=8, k=2, zipf_s=0.0)
+# At most 8 routed slots (T*k <= 8, bf16) the layer runs on the two
+# weight-streaming decode kernels instead of grouping rows for the tile
+# GEMMs.  These cases cover that path's branches: capacity drops, a shared
+# expert wider than the routed ones, many slots of one expert (two passes of
+# 4 token vectors over a weight row), 256 experts, widths that are not
+# multiples of 256 columns, and a wide H (few ring slots per SM).
+DECODE = [
+    mi.Workload("decode_shared_cap", T=4, H=264, I=200, E=4, k=2, I_shared=72, capacity_factor=0.5),
+    mi.Workload("decode_shared_wider", T=3, H=136, I=64, E=4, k=2, I_shared=200),
+    mi.Workload("decode_one_expert_8_slots", T=8, H=128, I=72, E=1, k=1),
+    mi.Workload("decode_e256_zipf", T=1, H=512, I=64, E=256, k=8, zipf_s=1.1),
+    mi.Workload("decode_wide_h", T=2, H=7168, I=512, E=8, k=4, I_shared=512),
+]
+
+
+@pytest.mark.parametrize("wl", DECODE, ids=[w.name for w in DECODE])
+def test_layer_decode_path(gpu_lib, wl):
+    assert wl.T * wl.k <= 8 and wl.dtype == "bf16"
+    r = check_layer(gpu_lib, wl)
+    if wl.capacity_factor > 0:
+        assert r["dropped"] > 0
+
+
+@pytest.mark.parametrize("T", [400, 4])
+def test_all_tokens_to_one_expert(gpu_lib, T):
+    """A router bias that sends every token to experts 0 and 1 (T = 4: the
+    decode path, 4 slots per expert)."""
+    wl = mi.Workload("skew", T=T, H=128, I=64, E=8, k=2, zipf_s=0.0)
     inp = mi.make_inputs(wl)
     inp["router_b"] = np.array([40.0, 30.0] + [-40.0] * 6, np.float32)
     d = to_device(inp, wl.dtype)
     y, idx_g, counts_g, _ = run_forward(gpu_lib, wl, d)
     assert np.all(np.sort(idx_g, 1) == [0, 1])
-    assert counts_g.tolist() == [400, 400] + [0] * 6
+    assert counts_g.tolist() == [T, T] + [0] * 6
     logits, _, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], 2, "bf16")
     yhat, _, _ = oracle_given_selection(wl, inp, logits, idx_g, np.arange(wl.T))
     assert rowwise_rel_err(host_f64(y), yhat) <= TOL["bf16"]
