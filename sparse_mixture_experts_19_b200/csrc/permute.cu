@@ -169,32 +169,47 @@ __global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_
         perm_rows[r] = -1;
 }
 
-// All of the grouping in one CTA when the slots fit one chunk (S <= 2048):
-// histogram, capacity cut and scans (phase 2 as in permute_scan_kernel with a
-// single chunk), then warp 0 scatters the slots in order while the other
-// warps mark the unused tail of perm_rows.  Same outputs, one launch.
+// All of the grouping in one CTA when the slots fit one chunk (S <= 2048).
+// Each of the 8 warps owns a contiguous segment of slots: it counts its
+// segment per expert (warp match, no atomics), the counts give the totals,
+// capacity cut and scans (phase 2 as in permute_scan_kernel with a single
+// chunk) and each warp's first rank per expert (earlier segments' counts),
+// then every warp scatters its segment in slot order while the threads past
+// the kept rows mark the unused tail of perm_rows.  Same outputs, one launch.
+constexpr int kSmallWarps = kScanThreads / 32;
+
 __global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
     const int32_t* __restrict__ idx, int S, int E, int64_t cap, int32_t* __restrict__ counts,
     int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
     int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix, int32_t shared_rows,
     int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of, int32_t* __restrict__ flags) {
-    __shared__ int32_t hist[kScanThreads];
+    __shared__ int32_t wcount[kSmallWarps][kScanThreads];  // per warp segment, per expert
     __shared__ int32_t sm[kScanThreads];
     __shared__ int32_t off[kScanThreads + 1];
-    const int e = threadIdx.x;
-    hist[e] = 0;
+    const int e = threadIdx.x, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int w = 0; w < kSmallWarps; ++w) wcount[w][e] = 0;
     __syncthreads();
+    const int seg = ((S + kSmallWarps - 1) / kSmallWarps + 31) / 32 * 32;
+    const int s0 = min(S, warp * seg), s1 = min(S, s0 + seg);
+    const uint32_t lt = (1u << lane) - 1u;
     bool bad = false;
-    for (int s = threadIdx.x; s < S; s += kScanThreads) {
-        const int ex = idx[s];
-        if (ex >= 0 && ex < E)
-            atomicAdd(&hist[ex], 1);
-        else
-            bad = true;
+    for (int sb = s0; sb < s1; sb += 32) {
+        const int s = sb + lane;
+        const int ex = (s < s1) ? idx[s] : -1;
+        const bool valid = (ex >= 0 && ex < E);
+        if (s < s1 && !valid) bad = true;
+        const uint32_t peers = __match_any_sync(0xffffffffu, valid ? ex : -1);
+        if (valid && (peers & lt) == 0) wcount[warp][ex] += __popc(peers);
+        __syncwarp();
     }
     if (bad) set_flag(flags, MOE_DEVFLAG_BAD_EXPERT_INDEX);
     __syncthreads();
-    const int32_t total = (e < E) ? hist[e] : 0;
+    int32_t total = 0;
+    for (int w = 0; w < kSmallWarps; ++w) {
+        const int32_t c = (e < E) ? wcount[w][e] : 0;
+        wcount[w][e] = total;  // first rank of warp w's segment in expert e
+        total += c;
+    }
     const int32_t kept = (cap > 0 && total > cap) ? (int32_t)cap : total;
     if (e < E) {
         counts[e] = total;
@@ -212,36 +227,29 @@ __global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
         offsets_ws[E + 1] = incl + shared_rows;
         offsets_out[E] = incl;
     }
-    write_mtile_prefix(kept, E, sm, mtile_prefix, mpair_prefix);
-    hist[e] = 0;  // running count of each expert's rows in slot order
-    __syncthreads();
+    write_mtile_prefix(kept, E, sm, mtile_prefix, mpair_prefix);  // ends with a barrier
     const int R = off[E];
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        const uint32_t lt = (1u << lane) - 1u;
-        for (int sb = 0; sb < S; sb += 32) {
-            const int s = sb + lane;
-            const int ex = (s < S) ? idx[s] : -1;
-            const bool valid = (ex >= 0 && ex < E);
-            const uint32_t peers = __match_any_sync(0xffffffffu, valid ? ex : -1);
-            int32_t rank = 0;
-            if (valid) rank = hist[ex] + __popc(peers & lt);
-            __syncwarp();
-            if (valid && (peers & lt) == 0) hist[ex] += __popc(peers);
-            __syncwarp();
-            if (s < S) {
-                if (valid && (cap <= 0 || rank < cap)) {
-                    const int32_t row = off[ex] + rank;
-                    perm_rows[row] = s;
-                    row_of[s] = row;
-                } else {
-                    row_of[s] = -1;
-                }
+    for (int sb = s0; sb < s1; sb += 32) {
+        const int s = sb + lane;
+        const int ex = (s < s1) ? idx[s] : -1;
+        const bool valid = (ex >= 0 && ex < E);
+        const uint32_t peers = __match_any_sync(0xffffffffu, valid ? ex : -1);
+        int32_t rank = 0;
+        if (valid) rank = wcount[warp][ex] + __popc(peers & lt);
+        __syncwarp();
+        if (valid && (peers & lt) == 0) wcount[warp][ex] += __popc(peers);
+        __syncwarp();
+        if (s < s1) {
+            if (valid && (cap <= 0 || rank < cap)) {
+                const int32_t row = off[ex] + rank;
+                perm_rows[row] = s;
+                row_of[s] = row;
+            } else {
+                row_of[s] = -1;
             }
         }
-    } else {
-        for (int r = R + (int)threadIdx.x - 32; r < S; r += kScanThreads - 32) perm_rows[r] = -1;
     }
+    for (int r = R + (int)threadIdx.x; r < S; r += kScanThreads) perm_rows[r] = -1;
 }
 
 __global__ void __launch_bounds__(kScanThreads) offsets_from_user_kernel(
