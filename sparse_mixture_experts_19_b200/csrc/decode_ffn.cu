@@ -168,14 +168,22 @@ __device__ __forceinline__ void widen8(const uint4& q, float2 (&f)[4]) {
     for (int i = 0; i < 4; ++i) f[i] = __bfloat1622float2(p[i]);
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
 // d[r][n] = sum_c W_r[c] * v_n[c] over K8 16-byte chunks, for NW weight rows
-// in shared memory (row r at w + r*K8) and NV vectors; float32 (each lane
-// keeps even and odd elements in the two halves of an f32x2 accumulator),
-// summed over the warp: every lane ends with the totals.  The loop has no
-// branches, so the loads of several iterations are in flight together.
-template <int NW, int NV>
-__device__ __forceinline__ void dots(const uint4* __restrict__ w, int K8, const uint4* const (&v)[NV],
-                                     float (&d)[NW][kDecBatch]) {
+// in shared memory (row r at shared address w + r*K8*16) and NV vectors, in
+// shared memory (kVecSmem: shared addresses vs[n]) or global memory (vg[n]);
+// float32 (each lane keeps even and odd elements in the two halves of an
+// f32x2 accumulator), summed over the warp: every lane ends with the totals.
+// The loop has no branches, so the loads of several iterations are in flight
+// together.
+template <int NW, int NV, bool kVecSmem>
+__device__ __forceinline__ void dots(uint32_t w, int K8, const uint32_t (&vs)[kDecBatch],
+                                     const uint4* const (&vg)[kDecBatch], float (&d)[NW][kDecBatch]) {
     const int lane = threadIdx.x & 31;
     float2 acc[NW][NV];
 #pragma unroll
@@ -186,9 +194,9 @@ __device__ __forceinline__ void dots(const uint4* __restrict__ w, int K8, const 
     for (int c = lane; c < K8; c += 32) {
         uint4 wq[NW], xq[NV];
 #pragma unroll
-        for (int r = 0; r < NW; ++r) wq[r] = w[r * K8 + c];
+        for (int r = 0; r < NW; ++r) wq[r] = lds128(w + (uint32_t)(r * K8 + c) * 16u);
 #pragma unroll
-        for (int n = 0; n < NV; ++n) xq[n] = v[n][c];
+        for (int n = 0; n < NV; ++n) xq[n] = kVecSmem ? lds128(vs[n] + (uint32_t)c * 16u) : __ldg(vg[n] + c);
         float2 wf[NW][4];
 #pragma unroll
         for (int r = 0; r < NW; ++r) widen8(wq[r], wf[r]);
@@ -213,39 +221,33 @@ __device__ __forceinline__ void dots(const uint4* __restrict__ w, int K8, const 
         }
 }
 
-// dots<NW, nv> for the nv (1..4) vectors at base + off[n] bytes, with the
-// vectors' address space (shared or global) known to the compiler in each
-// instantiation.
-template <int NW>
-__device__ __forceinline__ void dots_at(const uint4* w, int K8, const uint8_t* base, const int64_t (&off)[kDecBatch],
-                                        int nv, float (&d)[NW][kDecBatch]) {
+template <int NW, bool kVecSmem>
+__device__ __forceinline__ void dots_n(uint32_t w, int K8, const uint32_t (&vs)[kDecBatch],
+                                       const uint4* const (&vg)[kDecBatch], int nv, float (&d)[NW][kDecBatch]) {
     switch (nv) {
-        case 1: {
-            const uint4* v[1] = {reinterpret_cast<const uint4*>(base + off[0])};
-            dots<NW, 1>(w, K8, v, d);
-            break;
-        }
-        case 2: {
-            const uint4* v[2] = {reinterpret_cast<const uint4*>(base + off[0]),
-                                 reinterpret_cast<const uint4*>(base + off[1])};
-            dots<NW, 2>(w, K8, v, d);
-            break;
-        }
-        case 3: {
-            const uint4* v[3] = {reinterpret_cast<const uint4*>(base + off[0]),
-                                 reinterpret_cast<const uint4*>(base + off[1]),
-                                 reinterpret_cast<const uint4*>(base + off[2])};
-            dots<NW, 3>(w, K8, v, d);
-            break;
-        }
-        default: {
-            const uint4* v[4] = {
-                reinterpret_cast<const uint4*>(base + off[0]), reinterpret_cast<const uint4*>(base + off[1]),
-                reinterpret_cast<const uint4*>(base + off[2]), reinterpret_cast<const uint4*>(base + off[3])};
-            dots<NW, 4>(w, K8, v, d);
-            break;
-        }
+        case 1: dots<NW, 1, kVecSmem>(w, K8, vs, vg, d); break;
+        case 2: dots<NW, 2, kVecSmem>(w, K8, vs, vg, d); break;
+        case 3: dots<NW, 3, kVecSmem>(w, K8, vs, vg, d); break;
+        default: dots<NW, 4, kVecSmem>(w, K8, vs, vg, d); break;
     }
+}
+
+// dots for nv (1..4) vectors at byte offsets off[n]: from the shared-memory
+// vector area (smem_base, a shared address) or from global memory (gbase).
+template <int NW>
+__device__ __forceinline__ void dots_at(uint32_t w, int K8, bool in_smem, uint32_t smem_base, const uint8_t* gbase,
+                                        const int64_t (&off)[kDecBatch], int nv, float (&d)[NW][kDecBatch]) {
+    uint32_t vs[kDecBatch];
+    const uint4* vg[kDecBatch];
+#pragma unroll
+    for (int n = 0; n < kDecBatch; ++n) {
+        vs[n] = smem_base + (uint32_t)off[n];
+        vg[n] = reinterpret_cast<const uint4*>(gbase + off[n]);
+    }
+    if (in_smem)
+        dots_n<NW, true>(w, K8, vs, vg, nv, d);
+    else
+        dots_n<NW, false>(w, K8, vs, vg, nv, d);
 }
 
 // Shared-memory offsets for the vectors of the groups in [ga, gb] (in order,
@@ -359,23 +361,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gateup_kernel(const Dec
         while (q >= pl.gpre[g + 1]) ++g;
         const int i = (int)(q - pl.gpre[g]);
         const bool shared = pl.gexp[g] == a.E;
-        const uint4* wrow = reinterpret_cast<const uint4*>(ring + (size_t)r * slot_bytes);
+        const uint32_t wrow = smem_u32(ring + (size_t)r * slot_bytes);
+        const bool in_smem = pl.voff[g] >= 0;
         for (int b = 0; b < pl.gcnt[g]; b += kDecBatch) {
             const int nv = min(kDecBatch, pl.gcnt[g] - b);
             int64_t off[kDecBatch];  // byte offsets of the vectors in vec, or in x
             float d[2][kDecBatch];
-            if (pl.voff[g] >= 0) {
 #pragma unroll
-                for (int n = 0; n < kDecBatch; ++n) off[n] = pl.voff[g] + (int64_t)(b + min(n, nv - 1)) * row_bytes;
-                dots_at<2>(wrow, K8, vec, off, nv, d);
-            } else {
-#pragma unroll
-                for (int n = 0; n < kDecBatch; ++n) {
-                    const int id = pl.gvec[g][b + min(n, nv - 1)];
-                    off[n] = (shared ? id : id / a.k) * (int64_t)row_bytes;
-                }
-                dots_at<2>(wrow, K8, reinterpret_cast<const uint8_t*>(a.x), off, nv, d);
+            for (int n = 0; n < kDecBatch; ++n) {
+                const int nn = b + min(n, nv - 1);
+                const int id = pl.gvec[g][nn];
+                off[n] = in_smem ? pl.voff[g] + (int64_t)nn * row_bytes : (shared ? id : id / a.k) * (int64_t)row_bytes;
             }
+            dots_at<2>(wrow, K8, in_smem, smem_u32(vec), reinterpret_cast<const uint8_t*>(a.x), off, nv, d);
 #pragma unroll
             for (int n = 0; n < kDecBatch; ++n) {
                 if (lane == n && n < nv) {
@@ -461,20 +459,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_down_kernel(const DecAr
         const int g = (int)(q / npair);
         const bool shared = pl.gexp[g] == a.E;
         const int K = shared ? a.Is : a.I;
-        const uint4* wrow = reinterpret_cast<const uint4*>(ring + (size_t)r * slot_bytes);
+        const uint32_t wrow = smem_u32(ring + (size_t)r * slot_bytes);
+        const bool in_smem = pl.voff[g] >= 0;
         for (int b = 0; b < pl.gcnt[g]; b += kDecBatch) {
             const int nv = min(kDecBatch, pl.gcnt[g] - b);
             int64_t off[kDecBatch];  // byte offsets of the vectors in vec, or in h / hs
             float d[kDecDownRows][kDecBatch];
-            if (pl.voff[g] >= 0) {
 #pragma unroll
-                for (int n = 0; n < kDecBatch; ++n) off[n] = pl.voff[g] + (int64_t)(b + min(n, nv - 1)) * K * 2;
-                dots_at<kDecDownRows>(wrow, K / 8, vec, off, nv, d);
-            } else {
-#pragma unroll
-                for (int n = 0; n < kDecBatch; ++n) off[n] = (int64_t)pl.gvec[g][b + min(n, nv - 1)] * K * 2;
-                dots_at<kDecDownRows>(wrow, K / 8, reinterpret_cast<const uint8_t*>(shared ? a.hs : a.h), off, nv, d);
+            for (int n = 0; n < kDecBatch; ++n) {
+                const int nn = b + min(n, nv - 1);
+                off[n] = in_smem ? pl.voff[g] + (int64_t)nn * K * 2 : (int64_t)pl.gvec[g][nn] * K * 2;
             }
+            dots_at<kDecDownRows>(wrow, K / 8, in_smem, smem_u32(vec),
+                                  reinterpret_cast<const uint8_t*>(shared ? a.hs : a.h), off, nv, d);
 #pragma unroll
             for (int n = 0; n < kDecBatch; ++n) {
                 if (lane == n && n < nv) {
