@@ -4,16 +4,19 @@
 // (grouped_mm sorts tokens by expert id and groups them); "MoE稀疏架构是什么？
 // 从原理到落地的系统解读", section 三.2 (capacity-limited token dropping).
 //
-// Three passes over the T*k slot ids, all bit-reproducible:
+// Passes over the T*k slot ids (chunks of 2048), all bit-reproducible:
 //   1. chunk histogram: hist[c][e] = pairs of expert e in slot chunk c;
-//   2. one block per layer: exclusive scan of hist over chunks (in place), so
-//      base[c][e] = pairs of e in earlier chunks; counts, capacity cut,
-//      dropped, and the exclusive scan over experts -> offsets;
-//   3. stable scatter: each chunk walks its slots in order, 32 at a time,
-//      ranking equal experts inside a warp with __match_any_sync, so the
-//      rank of a pair is the number of earlier slots of the same expert.
-//      Slot order is token-major, hence ranks follow ascending token order,
-//      and a pair is kept iff its rank < C.
+//   2a. one block per expert: exclusive scan of hist[.][e] over the chunks
+//      (in place), so base[c][e] = pairs of e in earlier chunks; the total
+//      is counts[e];
+//   2b. one block: capacity cut, dropped, and the exclusive scan over
+//      experts -> offsets (and the GEMM schedulers' tile prefixes);
+//   3. stable scatter: one block per chunk, each of its 8 warps walking a
+//      256-slot segment in order, 32 slots at a time, ranking equal experts
+//      inside a warp with __match_any_sync and across the block's warps
+//      with per-warp counts; the rank of a pair is the number of earlier
+//      slots of the same expert.  Slot order is token-major, hence ranks
+//      follow ascending token order, and a pair is kept iff its rank < C.
 #include <mutex>
 
 #include "common.cuh"
@@ -23,7 +26,9 @@ namespace {
 
 constexpr int kHistThreads = 256;
 constexpr int kScanThreads = 256;  // >= kMaxExperts
-constexpr int kScatterWarps = 4;
+constexpr int kScatterWarps = 8;                          // warps per chunk in the scatter
+constexpr int kScatterSeg = kPermuteChunk / kScatterWarps;  // slots per warp segment
+constexpr int kChunkScanThreads = 1024;
 
 __global__ void __launch_bounds__(kHistThreads) permute_hist_kernel(
     const int32_t* __restrict__ idx, int64_t S, int E, int32_t* __restrict__ hist,
@@ -81,76 +86,113 @@ __device__ __forceinline__ void write_mtile_prefix(int32_t kept, int E, int32_t*
     write_tile_prefix(kept, E, sm, 2 * kGemmTileRows, mpair_prefix);
 }
 
-__global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(
-    int32_t* __restrict__ hist, int64_t nchunks, int E, int64_t cap, int32_t* __restrict__ counts,
-    int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
-    int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix, int32_t shared_rows) {
-    __shared__ int32_t kept_s[kScanThreads];
-    const int e = threadIdx.x;
-    int32_t total = 0;
-    if (e < E) {
-        for (int64_t c = 0; c < nchunks; ++c) {
-            int32_t v = hist[c * E + e];
-            hist[c * E + e] = total;
-            total += v;
+// 2a. Block e: exclusive scan of hist[.][e] over the chunks, in place, in
+// tiles of 1024 chunks with a carry; counts[e] = the total.
+__global__ void __launch_bounds__(kChunkScanThreads) permute_scan_chunks_kernel(int32_t* __restrict__ hist,
+                                                                                int64_t nchunks, int E,
+                                                                                int32_t* __restrict__ counts) {
+    __shared__ int32_t wsum[kChunkScanThreads / 32];
+    const int e = blockIdx.x, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    int32_t carry = 0;
+    for (int64_t c0 = 0; c0 < nchunks; c0 += kChunkScanThreads) {
+        const int64_t c = c0 + threadIdx.x;
+        const int32_t v = c < nchunks ? hist[c * E + e] : 0;
+        int32_t x = v;  // inclusive warp scan
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
         }
-    }
-    int32_t kept = (cap > 0 && total > cap) ? (int32_t)cap : total;
-    if (e < E) {
-        counts[e] = total;
-        dropped[e] = total - kept;
-    }
-    kept_s[e] = (e < E) ? kept : 0;
-    __syncthreads();
-    // inclusive Hillis-Steele scan over the (at most 256) experts
-    for (int o = 1; o < kScanThreads; o <<= 1) {
-        int32_t v = (e >= o) ? kept_s[e - o] : 0;
+        if (lane == 31) wsum[warp] = x;
         __syncthreads();
-        kept_s[e] += v;
+        if (warp == 0) {
+            int32_t w = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            wsum[lane] = w;  // inclusive over warps
+        }
         __syncthreads();
+        const int32_t incl = x + (warp > 0 ? wsum[warp - 1] : 0);
+        if (c < nchunks) hist[c * E + e] = carry + incl - v;
+        carry += wsum[kChunkScanThreads / 32 - 1];
+        __syncthreads();  // wsum is rewritten by the next tile
     }
-    // offsets_ws [E+2] feeds the GEMMs; offsets_out [E+1] is the caller's copy
-    if (e < E) {
-        int32_t excl = kept_s[e] - kept;
-        offsets_ws[e] = excl;
-        offsets_out[e] = excl;
-    }
-    if (e == 0) {
-        int32_t R = kept_s[E - 1];
-        offsets_ws[E] = R;
-        offsets_ws[E + 1] = R + shared_rows;
-        offsets_out[E] = R;
-    }
-    write_mtile_prefix(e < E ? kept : 0, E, kept_s, mtile_prefix, mpair_prefix);
+    if (threadIdx.x == 0) counts[e] = carry;
 }
 
+// 2b. One block: per-expert totals -> capacity cut, dropped, offsets, and
+// the tile prefixes of the grouped GEMMs.
+__global__ void __launch_bounds__(kScanThreads) permute_scan_experts_kernel(
+    const int32_t* __restrict__ counts, int E, int64_t cap, int32_t* __restrict__ dropped, int32_t* offsets_out,
+    int32_t* offsets_ws, int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix,
+    int32_t shared_rows) {
+    __shared__ int32_t sm[kScanThreads];
+    const int e = threadIdx.x;
+    const int32_t total = (e < E) ? counts[e] : 0;
+    const int32_t kept = (cap > 0 && total > cap) ? (int32_t)cap : total;
+    if (e < E) dropped[e] = total - kept;
+    const int32_t incl = block_scan_256(kept, sm);
+    // offsets_ws [E+2] feeds the GEMMs; offsets_out [E+1] is the caller's copy
+    if (e < E) {
+        offsets_ws[e] = incl - kept;
+        offsets_out[e] = incl - kept;
+    }
+    if (e == E - 1) {
+        offsets_ws[E] = incl;
+        offsets_ws[E + 1] = incl + shared_rows;
+        offsets_out[E] = incl;
+    }
+    write_mtile_prefix(kept, E, sm, mtile_prefix, mpair_prefix);
+}
+
+// 3. Block c scatters chunk c: warp w ranks the slots of its segment
+// [c*2048 + w*256, +256) from base[c][e] plus the earlier warps' counts.
 __global__ void __launch_bounds__(kScatterWarps * 32) permute_scatter_kernel(
-    const int32_t* __restrict__ idx, int64_t S, int E, int64_t cap,
-    const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
-    int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of) {
+    const int32_t* __restrict__ idx, int64_t S, int E, int64_t cap, const int32_t* __restrict__ base,
+    const int32_t* __restrict__ offsets, int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of) {
     __shared__ int32_t run[kScatterWarps][kMaxExperts];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t c = (int64_t)blockIdx.x * kScatterWarps + warp;
-    const int64_t s0 = c * kPermuteChunk;
-    if (s0 >= S) return;
-    for (int e = lane; e < E; e += 32) run[warp][e] = base[c * E + e];
-    __syncwarp();
-    const int64_t s1 = min(S, s0 + kPermuteChunk);
+    const int64_t c = blockIdx.x;
+    const int64_t cs1 = min(S, (c + 1) * kPermuteChunk);
+    const int64_t s0 = min(cs1, c * kPermuteChunk + (int64_t)warp * kScatterSeg);
+    const int64_t s1 = min(cs1, s0 + kScatterSeg);
+    for (int i = threadIdx.x; i < kScatterWarps * kMaxExperts; i += blockDim.x) (&run[0][0])[i] = 0;
+    __syncthreads();
     const uint32_t lt = (1u << lane) - 1u;
-    for (int64_t sb = s0; sb < s1; sb += 32) {
-        int64_t s = sb + lane;
-        int e = (s < s1) ? idx[s] : -1;
-        bool valid = (e >= 0 && e < E);
-        int key = valid ? e : -1;
-        uint32_t peers = __match_any_sync(0xffffffffu, key);
-        int32_t rank = 0;
-        if (valid) rank = run[warp][e] + __popc(peers & lt);
+    for (int64_t sb = s0; sb < s1; sb += 32) {  // counts of this warp's segment
+        const int64_t s = sb + lane;
+        const int ex = (s < s1) ? idx[s] : -1;
+        const bool valid = (ex >= 0 && ex < E);
+        const uint32_t peers = __match_any_sync(0xffffffffu, valid ? ex : -1);
+        if (valid && (peers & lt) == 0) run[warp][ex] += __popc(peers);
         __syncwarp();
-        if (valid && (peers & lt) == 0) run[warp][e] += __popc(peers);  // lowest peer updates
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {  // first rank of each warp's segment
+        int32_t r = base[c * E + e];
+        for (int w = 0; w < kScatterWarps; ++w) {
+            const int32_t n = run[w][e];
+            run[w][e] = r;
+            r += n;
+        }
+    }
+    __syncthreads();
+    for (int64_t sb = s0; sb < s1; sb += 32) {
+        const int64_t s = sb + lane;
+        const int ex = (s < s1) ? idx[s] : -1;
+        const bool valid = (ex >= 0 && ex < E);
+        const uint32_t peers = __match_any_sync(0xffffffffu, valid ? ex : -1);
+        int32_t rank = 0;
+        if (valid) rank = run[warp][ex] + __popc(peers & lt);
+        __syncwarp();
+        if (valid && (peers & lt) == 0) run[warp][ex] += __popc(peers);  // lowest peer updates
         __syncwarp();
         if (s < s1) {
             if (valid && (cap <= 0 || rank < cap)) {
-                int32_t row = offsets[e] + rank;
+                const int32_t row = offsets[ex] + rank;
                 perm_rows[row] = (int32_t)s;
                 row_of[s] = row;
             } else {
@@ -160,7 +202,6 @@ __global__ void __launch_bounds__(kScatterWarps * 32) permute_scatter_kernel(
     }
 }
 
-// perm_rows entries at and past R are set to -1.
 __global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_t S,
                                          const int32_t* __restrict__ offsets, int E) {
     const int64_t R = offsets[E];
@@ -172,7 +213,7 @@ __global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_
 // All of the grouping in one CTA when the slots fit one chunk (S <= 2048).
 // Each of the 8 warps owns a contiguous segment of slots: it counts its
 // segment per expert (warp match, no atomics), the counts give the totals,
-// capacity cut and scans (phase 2 as in permute_scan_kernel with a single
+// capacity cut and scans (as permute_scan_experts_kernel, with a single
 // chunk) and each warp's first rank per expert (earlier segments' counts),
 // then every warp scatters its segment in slot order while the threads past
 // the kept rows mark the unused tail of perm_rows.  Same outputs, one launch.
@@ -304,15 +345,18 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
     permute_hist_kernel<<<(unsigned)p.nchunks, kHistThreads, 0, st>>>(topk_idx, p.S, E,
                                                                        p.chunk_base, p.flags);
     trace_after(st);
+    trace_before("permute_scan_chunks", st);
+    permute_scan_chunks_kernel<<<(unsigned)E, kChunkScanThreads, 0, st>>>(p.chunk_base, p.nchunks, E, counts);
+    trace_after(st);
     trace_before("permute_scan", st);
-    permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
-        p.chunk_base, p.nchunks, E, p.cap, counts, dropped, offsets, p.offsets, p.mtile_prefix,
-        p.mpair_prefix, (int32_t)(p.Is > 0 ? p.T : 0));
+    permute_scan_experts_kernel<<<1, kScanThreads, 0, st>>>(counts, E, p.cap, dropped, offsets, p.offsets,
+                                                            p.mtile_prefix, p.mpair_prefix,
+                                                            (int32_t)(p.Is > 0 ? p.T : 0));
     trace_after(st);
     trace_before("permute_scatter", st);
-    unsigned blocks = (unsigned)((p.nchunks + kScatterWarps - 1) / kScatterWarps);
-    permute_scatter_kernel<<<blocks, kScatterWarps * 32, 0, st>>>(
-        topk_idx, p.S, E, p.cap, p.chunk_base, p.offsets, perm_rows, row_of);
+    permute_scatter_kernel<<<(unsigned)p.nchunks, kScatterWarps * 32, 0, st>>>(topk_idx, p.S, E, p.cap,
+                                                                                p.chunk_base, p.offsets,
+                                                                                perm_rows, row_of);
     trace_after(st);
     trace_before("permute_fill_tail", st);
     permute_fill_tail_kernel<<<64, 256, 0, st>>>(perm_rows, p.S, p.offsets, E);
