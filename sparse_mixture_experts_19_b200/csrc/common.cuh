@@ -91,6 +91,9 @@ cudaError_t launch_permute_noalloc(const Plan& sizes, const int32_t* topk_idx, i
                                    int32_t* dropped, cudaStream_t st);
 // plan offsets [E+2] from a caller's offsets [E+1] (appends the shared rows).
 cudaError_t launch_offsets_from_user(const Plan& p, const int32_t* offsets, cudaStream_t st);
+// xperm rows built token by token from row_of [T, k] (x read once).
+cudaError_t launch_scatter_x_rows(const Plan& p, const void* x, const int32_t* row_of, void* xperm,
+                                  cudaStream_t st);
 cudaError_t launch_gather_rows(const Plan& p, const void* x, const int32_t* perm_rows,
                                const int32_t* offsets, void* xperm, cudaStream_t st);
 // Grouped expert GEMMs for all groups (routed + shared):

@@ -153,6 +153,31 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* _
     }
 }
 
+// The same rows built token by token: xperm[row_of[t,j]] = x[t] for each kept
+// slot (t, j).  One warp per token; each 16-byte chunk of x[t] is read once and
+// stored k times (consecutive lanes: consecutive chunks of a row).  Reading x
+// once matters when x is larger than L2: the row-by-row gather reads every x
+// row k times, once per expert group sweeping the tokens.
+__global__ void scatter_x_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ row_of,
+                                      int64_t T, int k, int64_t row_chunks, uint4* __restrict__ xperm) {
+    const int lane = threadIdx.x % 32;
+    for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; t < T;
+         t += (int64_t)gridDim.x * blockDim.x / 32) {
+        const int32_t my_row = lane < k ? row_of[t * k + lane] : -1;  // k <= 32
+        const uint4* src = x + t * row_chunks;
+        // every lane takes the same iterations (the shuffles need the whole warp)
+        for (int64_t c0 = 0; c0 < row_chunks; c0 += 32) {
+            const int64_t c = c0 + lane;
+            const bool in = c < row_chunks;
+            const uint4 v = in ? src[c] : make_uint4(0, 0, 0, 0);
+            for (int j = 0; j < k; ++j) {
+                const int32_t r = __shfl_sync(0xffffffffu, my_row, j);
+                if (in && r >= 0) xperm[r * row_chunks + c] = v;
+            }
+        }
+    }
+}
+
 // y[t] = sum_j rows[row_of[t,j]] (+ rows[S + t]); one thread per 16-byte chunk
 // of a token's row, float32 sum in slot order, one rounding at the end.
 template <typename TV>
@@ -227,6 +252,17 @@ cudaError_t launch_gather_rows(const Plan& p, const void* x, const int32_t* perm
     trace_before("gather_rows", st);
     gather_rows_kernel<<<grid_for(p.S * 32, 256), 256, 0, st>>>(
         (const uint4*)x, perm_rows, offsets, (int)p.E, (int)p.k, chunks, (uint4*)xperm);
+    trace_after(st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_x_rows(const Plan& p, const void* x, const int32_t* row_of, void* xperm,
+                                  cudaStream_t st) {
+    if (p.S == 0) return cudaSuccess;
+    const int64_t chunks = p.H * (p.bf16 ? 2 : 4) / 16;
+    trace_before("gather_rows", st);
+    scatter_x_rows_kernel<<<grid_for(p.T * 32, 256), 256, 0, st>>>((const uint4*)x, row_of, p.T, (int)p.k, chunks,
+                                                                   (uint4*)xperm);
     trace_after(st);
     return cudaGetLastError();
 }

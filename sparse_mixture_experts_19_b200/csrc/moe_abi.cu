@@ -181,10 +181,15 @@ static cudaError_t run_router(const Plan& p, const void* x, const void* router_w
 }
 
 // The grouped FFN of moe_forward / moe_grouped_ffn, after routing and grouping.
+// row_of (slot -> grouped row, or -1) when known: the x rows are then built
+// token by token, reading x once; else row by row from perm_rows.
 static moe_status_t run_ffn(const Plan& p, const void* x, const void* w_gate, const void* w_up,
                             const void* w_down, const void* ws_gate, const void* ws_up,
-                            const void* ws_down, int mode, void* out, cudaStream_t st) {
-    CUDA_TRY(launch_gather_rows(p, x, p.perm_rows, p.offsets, p.xperm, st), "gather_rows");
+                            const void* ws_down, int mode, void* out, const int32_t* row_of, cudaStream_t st) {
+    if (row_of)
+        CUDA_TRY(launch_scatter_x_rows(p, x, row_of, p.xperm, st), "gather_rows");
+    else
+        CUDA_TRY(launch_gather_rows(p, x, p.perm_rows, p.offsets, p.xperm, st), "gather_rows");
     if (p.bf16) {
         // bf16: tensor cores (tcgen05 + TMEM + TMA)
         CUDA_TRY(launch_gateup_sm100(p, x, w_gate, w_up, ws_gate, ws_up, st), "gateup");
@@ -301,7 +306,7 @@ moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const int32
     CUDA_TRY(launch_offsets_from_user(p, offsets, st), "offsets");
     CUDA_TRY(cudaMemcpyAsync(p.perm_rows, perm_rows, sizeof(int32_t) * p.S, cudaMemcpyDeviceToDevice, st),
              "perm_rows copy");
-    return run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 0, expert_out, st);
+    return run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 0, expert_out, nullptr, st);
 }
 
 moe_status_t moe_combine(const moe_config_t* cfg, const float* expert_out, const int32_t* row_of,
@@ -356,7 +361,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
         return MOE_OK;
     }
     CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
-    if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.rows, st)) != MOE_OK)
+    if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.rows, p.row_of, st)) != MOE_OK)
         return s;
     CUDA_TRY(launch_combine_rows(p, p.rows, p.row_of, y, st), "combine_rows");
     return MOE_OK;
