@@ -195,14 +195,14 @@ __device__ __forceinline__ void epilogue_tile(const TileInfo& ti, const GemmArgs
         float w = 1.f;
         if (valid && a.mode == 1 && !ti.shared) w = a.topk_w[a.perm_rows[ti.row0 + r]];
 #pragma unroll 1
-        for (int j0 = 0; j0 < BN; j0 += 32) {
-            float v[32];
-            tmem_ld32(tq + j0, v);
+        for (int j0 = 0; j0 < BN; j0 += 64) {
+            float v[64];
+            tmem_ld64(tq + j0, v);  // 64 columns per TMEM round trip
             if (valid) {
                 if (a.mode == 1) {
                     bf16* dst = a.rows + orow * (int64_t)ti.N;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < 8; ++i) {
                         const int n = ti.n0 + j0 + i * 8;
                         if (n < ti.N) {
                             uint4 pk;
@@ -216,7 +216,7 @@ __device__ __forceinline__ void epilogue_tile(const TileInfo& ti, const GemmArgs
                 } else {
                     float* dst = a.out + orow * (int64_t)ti.N;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
+                    for (int i = 0; i < 16; ++i) {
                         const int n = ti.n0 + j0 + i * 4;
                         if (n < ti.N)
                             *reinterpret_cast<float4*>(dst + n) =
