@@ -26,8 +26,9 @@
 //                  h[slot][i] = bf16(silu(x . W_g[e][i]) * (x . W_u[e][i])).
 //   decode_down:   stage (group, hrow pair) = rows W_d[e][hrow], W_d[e][hrow+1]
 //                  (one contiguous copy); the dot products with the group's h
-//                  rows go to a float32 buffer [H, S + T], and the warp whose
-//                  stage is the pair's last to arrive (a counter per pair)
+//                  rows go to a float32 buffer [H, S + T]; after its last
+//                  stage each warp counts its stages' arrivals per pair, and
+//                  the warp bringing a pair's count to the number of experts
 //                  writes
 //                  y[t][hrow] = bf16(sum over j in slot order of
 //                  w[t,j] * d(t,j), plus the shared expert's d(t)).
@@ -45,8 +46,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kDecMaxGroups = kDecodeMaxSlots + 1;  // distinct routed experts + shared
-constexpr int kDecWarps = 8;                        // compute warps (warp 0 streams)
-constexpr int kDecThreads = 32 * (kDecWarps + 1);
+constexpr int kDecProducers = 4;                    // warps 0-3 stream (lane 0 of each)
+constexpr int kDecWarps = 8;                        // compute warps 4-11
+constexpr int kDecThreads = 32 * (kDecProducers + kDecWarps);
 constexpr int kDecSmemBytes = 220 * 1024;  // vectors + ring
 constexpr int kDecVecRows = 4;             // token vectors staged in shared memory per CTA
 constexpr int kDecMaxStages = 32;          // ring slots at most
@@ -54,10 +56,13 @@ constexpr int kDecBatch = 4;               // token vectors per pass over a weig
 constexpr int kDecDownRows = 2;            // W_d rows per down stage
 
 // Ring geometry: W compute warps (1, 2, 4 or 8), each owning Rw consecutive
-// slots.  Stage l goes to warp l % W, which takes its stages in order; its
-// j-th stage (j = l / W) uses slot j % Rw of its run.
+// slots.  Stage l goes to compute warp l % W, which takes its stages in
+// order; its j-th stage (j = l / W) uses slot j % Rw of its run.  Producer
+// p < NP = min(4, W) issues the stages l = p mod NP, so each compute warp's
+// slots are always filled, in order, by the same producer thread.
 struct Ring {
     int W, Rw;
+    __device__ __forceinline__ int producers() const { return W < kDecProducers ? W : kDecProducers; }
     __device__ __forceinline__ int slot(int l) const { return (l % W) * Rw + (l / W) % Rw; }
     __device__ __forceinline__ uint32_t parity(int l) const { return ((l / W) / Rw) & 1; }
 };
@@ -149,7 +154,7 @@ __device__ __forceinline__ void init_ring(const Ring& rg, uint64_t* full, uint64
     }
 }
 
-// Barrier of the 8 compute warps only (warp 0 keeps streaming).
+// Barrier of the 8 compute warps only (the producer warps keep streaming).
 __device__ __forceinline__ void compute_warps_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecWarps) : "memory");
 }
@@ -159,7 +164,7 @@ __device__ __forceinline__ void compute_warps_sync() {
 __device__ __forceinline__ void copy_to_smem(uint8_t* dst, const void* src, int64_t bytes) {
     const uint4* s = reinterpret_cast<const uint4*>(src);
     uint4* d = reinterpret_cast<uint4*>(dst);
-    for (int64_t i = threadIdx.x - 32; i < bytes / 16; i += 32 * kDecWarps) d[i] = s[i];
+    for (int64_t i = threadIdx.x - 32 * kDecProducers; i < bytes / 16; i += 32 * kDecWarps) d[i] = s[i];
 }
 
 __device__ __forceinline__ void widen8(const uint4& q, float2 (&f)[4]) {
@@ -272,10 +277,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
-// Producer's exit: no bulk copy may still be in flight (bounded waits on the
-// phases of the last W*Rw stages issued).
-__device__ __forceinline__ void drain_ring(uint64_t* full, int issued, const Ring& rg) {
-    for (int l = std::max(0, issued - rg.W * rg.Rw); l < issued; ++l) drain_wait(&full[rg.slot(l)], rg.parity(l));
+// Producer p's exit: none of its bulk copies may still be in flight (bounded
+// waits on the phases of its stages among the last W*Rw before `end`, the
+// stage it stopped at).
+__device__ __forceinline__ void drain_ring(uint64_t* full, int p, int end, const Ring& rg) {
+    const int np = rg.producers();
+    for (int l = p; l < end; l += np)
+        if (l >= end - rg.W * rg.Rw) drain_wait(&full[rg.slot(l)], rg.parity(l));
 }
 
 __global__ void __launch_bounds__(kDecThreads, 1) decode_gateup_kernel(const DecArgs a, const Ring rg) {
@@ -320,10 +328,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gateup_kernel(const Dec
     __syncthreads();
     volatile int* abort_flag = &abort_s;
 
-    if (warp == 0) {
-        if (lane == 0) {
-            int g = 0, l = 0;
-            for (; l < nq; ++l) {
+    if (warp < kDecProducers) {
+        if (lane == 0 && warp < rg.producers()) {
+            int g = 0, l = warp;
+            for (; l < nq; l += rg.producers()) {
                 const int r = rg.slot(l);
                 if (!wait_sleep_or_abort(&empty[r], rg.parity(l) ^ 1, abort_flag, a.flags)) break;
                 const int64_t q = q0 + l;
@@ -337,7 +345,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gateup_kernel(const Dec
                 bulk_load(dst, rgate, row_bytes, &full[r]);
                 bulk_load(dst + row_bytes, rup, row_bytes, &full[r]);
             }
-            drain_ring(full, l, rg);
+            drain_ring(full, warp, min(l, nq), rg);
         }
         return;
     }
@@ -352,9 +360,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gateup_kernel(const Dec
         }
     }
     compute_warps_sync();
-    if (warp > rg.W) return;
+    const int cw = warp - kDecProducers;  // compute warp 0..7
+    if (cw >= rg.W) return;
     int g = 0;
-    for (int l = warp - 1; l < nq; l += rg.W) {
+    for (int l = cw; l < nq; l += rg.W) {
         const int r = rg.slot(l);
         if (!warp_wait(&full[r], rg.parity(l), abort_flag, a.flags)) break;
         const int64_t q = q0 + l;
@@ -421,10 +430,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_down_kernel(const DecAr
     volatile int* abort_flag = &abort_s;
     const uint32_t slot_bytes = 2u * kDecDownRows * (uint32_t)max(a.I, a.Is);
 
-    if (warp == 0) {
-        if (lane == 0) {
-            int l = 0;
-            for (; l < nq; ++l) {
+    if (warp < kDecProducers) {
+        if (lane == 0 && warp < rg.producers()) {
+            int l = warp;
+            for (; l < nq; l += rg.producers()) {
                 const int r = rg.slot(l);
                 if (!wait_sleep_or_abort(&empty[r], rg.parity(l) ^ 1, abort_flag, a.flags)) break;
                 const int64_t q = q0 + l, hrow = (q % npair) * kDecDownRows;
@@ -435,7 +444,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_down_kernel(const DecAr
                 mbar_arrive_expect_tx(&full[r], bytes);
                 bulk_load(ring + (size_t)r * slot_bytes, src, bytes, &full[r]);
             }
-            drain_ring(full, l, rg);
+            drain_ring(full, warp, min(l, nq), rg);
         }
         return;
     }
@@ -451,8 +460,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_down_kernel(const DecAr
         }
     }
     compute_warps_sync();
-    if (warp > rg.W) return;
-    for (int l = warp - 1; l < nq; l += rg.W) {
+    const int cw = warp - kDecProducers;  // compute warp 0..7
+    if (cw >= rg.W) return;
+    int done = cw;  // first stage of this warp not completed
+    for (int l = cw; l < nq; l += rg.W) {
         const int r = rg.slot(l);
         if (!warp_wait(&full[r], rg.parity(l), abort_flag, a.flags)) break;
         const int64_t q = q0 + l, pair = q % npair, hrow = pair * kDecDownRows;
@@ -478,18 +489,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_down_kernel(const DecAr
                     const int col = shared ? a.S + pl.gvec[g][b + n] : pl.gvec[g][b + n];
 #pragma unroll
                     for (int rr = 0; rr < kDecDownRows; ++rr) a.part[(hrow + rr) * a.P + col] = d[rr][n];
-                    __threadfence();
                 }
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[r]);  // the ring slot is free
-        // The stage that brings the pair's arrivals to ng sums the pair.
+        if (lane == 0) mbar_arrive(&empty[r]);  // the dot products are done: the ring slot is free
+        done = l + rg.W;
+    }
+    // Arrivals after the warp's last stage, behind one fence: the counters
+    // only pick which stage's warp sums a pair (the one bringing its arrivals
+    // to ng), so they need not delay the streaming loop.
+    __threadfence();  // this warp's partials, before its arrivals
+    __syncwarp();
+    for (int l = cw; l < done; l += rg.W) {
+        const int64_t q = q0 + l, pair = q % npair, hrow = pair * kDecDownRows;
         int last = 0;
         if (lane == 0) last = atomicAdd(&a.cnt[pair], 1) == ng - 1;
         last = __shfl_sync(0xffffffffu, last, 0);
         if (last) {
-            __syncwarp();
             __threadfence();
             for (int q2 = lane; q2 < a.T * kDecDownRows; q2 += 32) {
                 const int t = q2 / kDecDownRows;
