@@ -78,6 +78,10 @@ struct Tables {
     int32_t mtp[kMaxExperts + 1];
 };
 
+// Epilogue staging buffers (4 warps x kEpiStageBytes) after the ring, the
+// barriers (256 B) and the tables, 128-byte aligned.
+constexpr size_t kEpiStageOff = (kStages * kStageBytes + 256 + sizeof(Tables) + 127) / 128 * 128;
+
 struct Sched {
     int E, nb_r, nb_s, mt_s;
     int gm_r, gm_s;  // row tiles per band (routed, shared)
@@ -153,6 +157,46 @@ __device__ __forceinline__ void decode_tile(int64_t t, const Tables& tb, const S
     }
 }
 
+// Coalesced epilogue stores (down GEMM).  Each epilogue warp owns a 4 KB shared-memory
+// buffer holding its 32 rows x 64 bf16 columns (128 B per row), with 16-byte
+// chunk c of row r at r*128 + ((c ^ (r % 8)) * 16): the row-wise writes (lane
+// = row) and the column-wise reads (8 lanes per row) are both free of bank
+// conflicts.  The global stores then cover 4 rows x 128 B per instruction
+// instead of 32 rows x 16 B.
+constexpr int kEpiStageBytes = 32 * 128;
+
+__device__ __forceinline__ uint32_t stage_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// The warp's staged 32 x 64 chunk -> global: row i of the warp goes to
+// row_ptr(i) (nullptr: row not stored), columns col0 .. col0 + 63, of which
+// only those < N are stored (N a multiple of 8).
+template <typename RowPtr>
+__device__ __forceinline__ void flush_stage(uint32_t stage, int lane, int col0, int N, RowPtr row_ptr) {
+    __syncwarp();
+    const int c = lane & 7;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int rr = i * 4 + (lane >> 3);
+        const uint4 v = ld_shared_v4(stage + stage_off(rr, c));
+        bf16* dst = row_ptr(rr);
+        const int n = col0 + c * 8;
+        if (dst && n < N) *reinterpret_cast<uint4*>(dst + n) = v;
+    }
+    __syncwarp();
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -164,10 +208,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // every lane loads and only rows < ti.rows store.
 template <bool kGateUp, int BN>
 __device__ __forceinline__ void epilogue_tile(const TileInfo& ti, const GemmArgs& a, uint32_t acc_base, int q,
-                                              int r) {
+                                              int r, uint32_t stage) {
     const uint32_t tq = acc_base + ((uint32_t)(q * 32) << 16);
+    const int lane = r & 31;
     const bool valid = r < ti.rows;
     if (kGateUp) {
+        // h rows are stored directly: this kernel is bound by shared-memory
+        // bandwidth, which staging would add to (measured slower)
         bf16* dst = ti.shared ? a.hs + (int64_t)(ti.arow + r) * a.Ns : a.h + (ti.row0 + r) * (int64_t)a.N;
 #pragma unroll 1
         for (int j0 = 0; j0 < BN; j0 += 32) {
@@ -194,26 +241,35 @@ __device__ __forceinline__ void epilogue_tile(const TileInfo& ti, const GemmArgs
         const int64_t orow = ti.shared ? a.S + ti.arow + r : ti.row0 + r;
         float w = 1.f;
         if (valid && a.mode == 1 && !ti.shared) w = a.topk_w[a.perm_rows[ti.row0 + r]];
+        if (a.mode == 1) {
+            auto row_ptr = [&](int i) -> bf16* {
+                const int rr = q * 32 + i;
+                if (rr >= ti.rows) return nullptr;
+                const int64_t orr = ti.shared ? a.S + ti.arow + rr : ti.row0 + rr;
+                return a.rows + orr * (int64_t)ti.N;
+            };
 #pragma unroll 1
-        for (int j0 = 0; j0 < BN; j0 += 64) {
-            float v[64];
-            tmem_ld64(tq + j0, v);  // 64 columns per TMEM round trip
-            if (valid) {
-                if (a.mode == 1) {
-                    bf16* dst = a.rows + orow * (int64_t)ti.N;
+            for (int j0 = 0; j0 < BN; j0 += 64) {
+                float v[64];
+                tmem_ld64(tq + j0, v);  // 64 columns per TMEM round trip
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int n = ti.n0 + j0 + i * 8;
-                        if (n < ti.N) {
-                            uint4 pk;
-                            pk.x = pack_bf16x2(w * v[i * 8 + 0], w * v[i * 8 + 1]);
-                            pk.y = pack_bf16x2(w * v[i * 8 + 2], w * v[i * 8 + 3]);
-                            pk.z = pack_bf16x2(w * v[i * 8 + 4], w * v[i * 8 + 5]);
-                            pk.w = pack_bf16x2(w * v[i * 8 + 6], w * v[i * 8 + 7]);
-                            *reinterpret_cast<uint4*>(dst + n) = pk;
-                        }
-                    }
-                } else {
+                for (int i = 0; i < 8; ++i) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(w * v[i * 8 + 0], w * v[i * 8 + 1]);
+                    pk.y = pack_bf16x2(w * v[i * 8 + 2], w * v[i * 8 + 3]);
+                    pk.z = pack_bf16x2(w * v[i * 8 + 4], w * v[i * 8 + 5]);
+                    pk.w = pack_bf16x2(w * v[i * 8 + 6], w * v[i * 8 + 7]);
+                    st_shared_v4(stage + stage_off(lane, i), pk);
+                }
+                flush_stage(stage, lane, ti.n0 + j0, ti.N, row_ptr);
+            }
+        } else {
+            // unweighted float32 rows (stage API): direct stores
+#pragma unroll 1
+            for (int j0 = 0; j0 < BN; j0 += 64) {
+                float v[64];
+                tmem_ld64(tq + j0, v);
+                if (valid) {
                     float* dst = a.out + orow * (int64_t)ti.N;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -245,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     Tables* tb = reinterpret_cast<Tables*>(smem + kStages * kStageBytes + 256);
+    const uint32_t epi_stage = smem_u32(smem + kEpiStageOff) + (uint32_t)(((threadIdx.x / 32) & 3) * kEpiStageBytes);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     for (int i = threadIdx.x; i < a.E + 2; i += kThreads) tb->off[i] = a.offsets[i];
@@ -369,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
             tc_fence_after();
-            epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r);
+            epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r, epi_stage);
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
         }
@@ -400,6 +457,8 @@ struct PairTables {
     int32_t off[kMaxExperts + 2];
     int32_t mpp[kMaxExperts + 1];  // prefix of 256-row pair tiles
 };
+
+constexpr size_t kPEpiStageOff = (kPStages * kPStageBytes + 256 + sizeof(PairTables) + 127) / 128 * 128;
 
 // Pair tile t -> this CTA's (rank) half: rows row0 .. row0 + rows - 1 (rows may
 // be <= 0 when the group ends inside the pair's first half).
@@ -462,6 +521,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     PairTables* tb = reinterpret_cast<PairTables*>(smem + kPStages * kPStageBytes + 256);
+    const uint32_t epi_stage = smem_u32(smem + kPEpiStageOff) + (uint32_t)(((threadIdx.x / 32) & 3) * kEpiStageBytes);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_ctarank();
@@ -575,7 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
             tc_fence_after();
-            epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r);
+            epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r, epi_stage);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(&tempty[acc], 0);  // the leader's barrier
@@ -594,7 +654,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
 }
 
 // ------------------------------------------------------------------ host side
-constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + 256 + sizeof(Tables);
+constexpr size_t kSmemBytes = kEpiStageOff + 4 * kEpiStageBytes + 1024;
 
 template <bool kGateUp>
 cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const GemmArgs& args,
@@ -611,7 +671,7 @@ cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const Ge
     return cudaGetLastError();
 }
 
-constexpr size_t kPSmemBytes = kPStages * kPStageBytes + 1024 + 256 + sizeof(PairTables);
+constexpr size_t kPSmemBytes = kPEpiStageOff + 4 * kEpiStageBytes + 1024;
 
 template <bool kGateUp>
 cudaError_t launch_grouped_pair(const Plan& p, const CUtensorMap (&maps)[6], const GemmArgs& args,
