@@ -313,17 +313,19 @@ def run_ours(args, wl, world, rank, local):
     except Exception:
         gpu_uuid = None
 
-    # ---- timed region: device time of K steps.  Only the dominant kernel
-    # (the grouped gate/up GEMM) is bracketed by events there, so the step
-    # time is not perturbed; the per-kernel breakdown comes from a second,
-    # fully traced run of the same K steps.  With graphs (default) the K
-    # steps are captured once into a CUDA graph and a run is one replay.
+    # ---- timed region: device time of K steps, with no event inside the
+    # steps.  The dominant kernel's own time (the grouped gate/up GEMM, or the
+    # decode gate/up kernel) comes from a second run of the same K steps in
+    # which only that kernel is bracketed by events, the per-kernel breakdown
+    # from a third, fully traced run.  With graphs (default) the K steps are
+    # captured once into a CUDA graph and a run is one replay.
     use_graph = not args.no_graph
 
-    def run_k_steps(only, sample_clocks):
+    def run_k_steps(trace, sample_clocks, only=None):
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         graph = None
-        moe.moe_trace_begin(64 * args.steps, only)
+        if trace:
+            moe.moe_trace_begin(64 * args.steps, only)
         if use_graph:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, capture_error_mode="thread_local"):
@@ -344,14 +346,15 @@ def run_ours(args, wl, world, rank, local):
         torch.cuda.synchronize(dev)
         if sampler:
             sampler.__exit__(None, None, None)
-        tr = moe.moe_trace_end(64 * args.steps)
+        tr = moe.moe_trace_end(64 * args.steps) if trace else []
         barrier()
         del graph
         return ev0.elapsed_time(ev1), tr, (sampler.summary() if sampler else None)
 
-    ms_local, trace_dom, clk = run_k_steps("gateup", True)
+    ms_local, _, clk = run_k_steps(False, True)              # the timed run: no trace events
     ms = max_over_ranks(ms_local)
-    _, trace, _ = run_k_steps(None, False)
+    _, trace_dom, _ = run_k_steps(True, False, "gateup")     # the dominant kernel alone
+    _, trace, _ = run_k_steps(True, False)                   # every kernel
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host
     x_host = d["x"].cpu().pin_memory()
