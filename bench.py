@@ -286,10 +286,11 @@ def run_ours(args, wl, world, rank, local):
     counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(x_in):
+    def step(x_in, y_out=None):
         # enqueued on the current stream (the capture stream while a graph is recorded)
         moe.moe_forward(cfg, x_in, d["router_w"], d["router_b"], d["w_gate"], d["w_up"], d["w_down"],
-                        d["ws_gate"], d["ws_up"], d["ws_down"], y, None, counts, None, ws)
+                        d["ws_gate"], d["ws_up"], d["ws_down"], y if y_out is None else y_out, None, counts,
+                        None, ws)
 
     def barrier():
         if world > 1:
@@ -357,24 +358,56 @@ def run_ours(args, wl, world, rank, local):
     _, trace, _ = run_k_steps(True, False)                   # every kernel
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host
+    # Every step copies its x from pinned host memory and its y back, as a
+    # serving loop would: the copies run on their own streams, so step i+1's
+    # input copy and step i-1's output copy overlap step i's forward (x and y
+    # double-buffered on the device; the ordering is kept by events).
     x_host = d["x"].cpu().pin_memory()
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    x_dev = torch.empty_like(d["x"])
+    y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(d["x"]) for _ in range(2)]
+    y_dev = [torch.empty_like(y) for _ in range(2)]
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x_dev)
-        y_host.copy_(y, non_blocking=True)
+    def e2e_steps(n):
+        main = torch.cuda.current_stream(dev)
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        start = torch.cuda.Event()
+        start.record(main)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        x_ready = [torch.cuda.Event() for _ in range(2)]
+        x_free = [torch.cuda.Event() for _ in range(2)]
+        y_ready = [torch.cuda.Event() for _ in range(2)]
+        y_free = [torch.cuda.Event() for _ in range(2)]
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(x_free[b])  # forward i-2 has read x_dev[b]
+                x_dev[b].copy_(x_host, non_blocking=True)
+                x_ready[b].record(s_in)
+            main.wait_event(x_ready[b])
+            if i >= 2:
+                main.wait_event(y_free[b])  # y_dev[b] of step i-2 is on the host
+            step(x_dev[b], y_dev[b])
+            x_free[b].record(main)
+            y_ready[b].record(main)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(y_ready[b])
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+                y_free[b].record(s_out)
+        end_in, end_out = torch.cuda.Event(), torch.cuda.Event()
+        end_in.record(s_in)
+        end_out.record(s_out)
+        main.wait_event(end_in)
+        main.wait_event(end_out)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_steps(2)
     torch.cuda.synchronize(dev)
     g2 = None
     if use_graph:
         g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2, capture_error_mode="thread_local"):
-            for _ in range(args.steps):
-                e2e_step()
+            e2e_steps(args.steps)
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -382,8 +415,7 @@ def run_ours(args, wl, world, rank, local):
     if use_graph:
         g2.replay()
     else:
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_steps(args.steps)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -456,7 +488,8 @@ def run_ours(args, wl, world, rank, local):
         "gpu_launches": len(trace),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+                "d2h_bytes_per_step": int(y_host[0].numel() * y_host[0].element_size()),
+                "overlap": "copies on two side streams, x and y double-buffered"},
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
