@@ -501,25 +501,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_down_kernel(const DecAr
     // to ng), so they need not delay the streaming loop.
     __threadfence();  // this warp's partials, before its arrivals
     __syncwarp();
-    for (int l = cw; l < done; l += rg.W) {
+    // 32 stages at a time, one arrival per lane, all in flight together; a
+    // lane whose arrival completes a pair sums that pair's y entries itself.
+    for (int l0 = cw; l0 < done; l0 += 32 * rg.W) {
+        const int l = l0 + lane * rg.W;
+        if (l >= done) continue;
         const int64_t q = q0 + l, pair = q % npair, hrow = pair * kDecDownRows;
-        int last = 0;
-        if (lane == 0) last = atomicAdd(&a.cnt[pair], 1) == ng - 1;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-            __threadfence();
-            for (int q2 = lane; q2 < a.T * kDecDownRows; q2 += 32) {
-                const int t = q2 / kDecDownRows;
-                const int64_t hr = hrow + q2 % kDecDownRows;
-                const float* pr = a.part + hr * a.P;
-                float acc = 0.f;
-                for (int j = 0; j < a.k; ++j) {
-                    const int s = t * a.k + j;
-                    if (pl.kept[s]) acc = fmaf(pl.wslot[s], __ldcg(pr + s), acc);
-                }
-                if (a.Is > 0) acc += __ldcg(pr + a.S + t);
-                a.y[(int64_t)t * a.H + hr] = __float2bfloat16_rn(acc);
+        if (atomicAdd(&a.cnt[pair], 1) != ng - 1) continue;
+        __threadfence();
+        for (int q2 = 0; q2 < a.T * kDecDownRows; ++q2) {
+            const int t = q2 / kDecDownRows;
+            const int64_t hr = hrow + q2 % kDecDownRows;
+            const float* pr = a.part + hr * a.P;
+            float acc = 0.f;
+            for (int j = 0; j < a.k; ++j) {
+                const int s = t * a.k + j;
+                if (pl.kept[s]) acc = fmaf(pl.wslot[s], __ldcg(pr + s), acc);
             }
+            if (a.Is > 0) acc += __ldcg(pr + a.S + t);
+            a.y[(int64_t)t * a.H + hr] = __float2bfloat16_rn(acc);
         }
     }
 }
