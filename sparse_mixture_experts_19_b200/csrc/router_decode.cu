@@ -6,7 +6,7 @@
 // With few tokens the router is a matrix-vector product per token.  Each
 // token gets a thread-block cluster of C CTAs (C <= 8); CTA r scores experts
 // [r*epc, (r+1)*epc) with one warp per expert at a time, the 32 lanes of a
-// warp splitting H in 16-byte chunks (four in flight per lane).  Scores are
+// warp splitting H in 16-byte chunks (twelve in flight per lane).  Scores are
 // exact up to fp64 rounding: for bf16 inputs each product of two bf16 values
 // is exact in float32 (8-bit by 8-bit significands, for |product| in
 // [2^-126, 2^128)) and is summed in fp64; float32 inputs are multiplied in
@@ -28,6 +28,7 @@ using namespace sm100;
 constexpr int kWarps = 8;
 constexpr int kMaxCluster = 8;
 constexpr int kExpertsPerWarpRound = kWarps;
+constexpr int kRound = 12;  // 16-byte chunks per lane in flight
 
 __device__ __forceinline__ double ld_dsmem_f64(uint32_t addr) {
     double v;
@@ -70,17 +71,19 @@ __global__ void __launch_bounds__(kWarps * 32) router_decode_kernel(
 
     for (int e = e0 + warp; e < e1; e += kExpertsPerWarpRound) {
         const uint4* wrow = reinterpret_cast<const uint4*>(wr + (int64_t)e * H);
+        // up to kRound chunks per lane loaded before any is used (one round
+        // of memory latency for H up to 32 * kRound chunks)
         double acc[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int c = lane; c < nch; c += 128) {
-            uint4 xq[4], wq[4];
+        for (int c = lane; c < nch; c += 32 * kRound) {
+            uint4 xq[kRound], wq[kRound];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kRound; ++u) {
                 const int cu = c + 32 * u;
                 xq[u] = cu < nch ? xr[cu] : make_uint4(0, 0, 0, 0);
                 wq[u] = cu < nch ? wrow[cu] : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) chunk_dot(xq[u], wq[u], acc[u], TIn());
+            for (int u = 0; u < kRound; ++u) chunk_dot(xq[u], wq[u], acc[u % 4], TIn());
         }
         double s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
