@@ -9,18 +9,18 @@
 // With one or two slots per expert a 128-row tensor-core tile would be
 // almost all padding, so the layer is written as what it is: one read of the
 // selected experts' weight rows.  Both kernels are persistent (one CTA per
-// SM).  Warp 0 streams whole weight rows (contiguous 2*H or 2*I bytes) into
-// a shared-memory ring with 1-D bulk copies (cp.async.bulk, completion
+// SM).  Warps 0-3 stream whole weight rows (contiguous 2*H or 2*I bytes)
+// into a shared-memory ring with 1-D bulk copies (cp.async.bulk, completion
 // counted on the stage's mbarrier).  W compute warps (8, or fewer when few
-// rows fit) take the stages round-robin, each lane over 16-byte chunks of the
-// row, against the token vectors (x rows, or h rows) of the CTA's experts
-// that the compute warps first copy into shared memory next to the ring
-// (float32 sums in packed f32x2 FMAs).  Each compute warp owns its
-// own run of ring slots, filled in its stage order, so every wait is on the
-// next phase of a slot that warp itself released (an mbarrier parity wait
-// can only tell its phase from the one before).  Each CTA takes a contiguous
-// range of stages: consecutive stages read consecutive DRAM pages and every
-// SM streams the same number of bytes.
+// rows fit) take the stages round-robin, each lane over 16-byte chunks of
+// the row, against the token vectors (x rows, or h rows) of the CTA's
+// experts that the compute warps first copy into shared memory next to the
+// ring (float32 sums in packed f32x2 FMAs).  Each compute warp owns its own
+// run of ring slots, filled in its stage order by one producer, so every
+// wait is on the next phase of a slot that warp itself released (an mbarrier
+// parity wait can only tell its phase from the one before).  Each CTA takes
+// a contiguous range of stages: consecutive stages read consecutive DRAM
+// pages and every SM streams the same number of bytes.
 //
 //   decode_gateup: stage (group, i) = rows W_g[e][i] and W_u[e][i];
 //                  h[slot][i] = bf16(silu(x . W_g[e][i]) * (x . W_u[e][i])).
