@@ -103,7 +103,11 @@ int64_t moe_capacity(const moe_config_t* cfg);
 /*
  * moe_route -- router scores, top-k selection and softmax over the
  * selected scores ("MoE稀疏架构是什么？从原理到落地的系统解读", sections 三.1
- * and 四).  Scores are accumulated in float32 and never rounded to bf16.
+ * and 四).  Scores are never rounded to bf16.  bf16 with T*E*H > 2^26:
+ * float32 tensor-core sums, and the experts near a token's k-th/(k+1)-th
+ * boundary are rescored exactly in fp64 before the choice.  Otherwise
+ * (few tokens): every score exact up to fp64 rounding (bf16 products are
+ * exact in float32).  float32 layer with many tokens: float32 FMAs.
  *   x [T,H], router_w [E,H], router_b [E] float32 or NULL
  *   -> topk_idx [T,top_k] int32: chosen experts, score descending, ties to
  *      the lower index; topk_w [T,top_k] float32: softmax of those scores.
