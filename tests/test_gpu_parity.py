@@ -282,6 +282,24 @@ def test_permute_is_bit_reproducible(gpu_lib):
     assert np.array_equal(res[0][2], ref["perm_rows"])
 
 
+# y is bit-reproducible on every path (fixed summation orders; the decode
+# down kernel's arrival counters only pick which warp sums a pair): three
+# calls on the same inputs give identical bytes.
+REPRO = [
+    mi.Workload("repro_decode_shared", T=2, H=264, I=200, E=8, k=4, I_shared=72),
+    mi.Workload("repro_tile_gemms", T=700, H=256, I=192, E=8, k=2),
+    mi.Workload("repro_cta_pairs_cap", T=2100, H=256, I=256, E=4, k=2, capacity_factor=1.1),
+]
+
+
+@pytest.mark.parametrize("wl", REPRO, ids=[w.name for w in REPRO])
+def test_forward_is_bit_reproducible(gpu_lib, wl):
+    d = to_device(mi.make_inputs(wl), wl.dtype)
+    ys = [run_forward(gpu_lib, wl, d)[0].view(torch.int16).cpu().numpy() for _ in range(3)]
+    for y in ys[1:]:
+        assert np.array_equal(ys[0], y)
+
+
 # ------------------------------------------------------------ full sizes
 
 FULL_SAMPLE = 24
