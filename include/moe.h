@@ -23,6 +23,8 @@
  *
  * Readings where the pages are silent: ties go to the lower expert index;
  * the expert FFN is SwiGLU without biases; capacity C = ceil(cf * T * k / E)
+ * (taken with a relative tolerance of 1e-6, so that the float32 rounding of
+ * cf does not lift an exact integer to the next one)
  * with tokens served in ascending token order, a dropped (token, expert)
  * pair contributes nothing and the token's other weights are not
  * renormalised; a shared expert (I_shared > 0) is always applied with
@@ -215,6 +217,29 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
                          const void* w_down, const void* ws_gate, const void* ws_up,
                          const void* ws_down, void* y, int32_t* topk_idx_out, int32_t* counts_out,
                          int32_t* dropped_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_forward_routed -- the layer after routing, for one shard of a batch's
+ * tokens ("MoE稀疏架构是什么？…", section 三.2: capacity-limited dropping).
+ * Capacity is served in global token order, so a shard's capacity for an
+ * expert is what the earlier shards left of it.
+ *   x [T,H] (this shard's tokens); topk_idx [T,top_k] int32 and topk_w
+ *   [T,top_k] float32 as moe_route produces them; capacity_left [E] int32 or
+ *   NULL.  With capacity_left, a slot of expert e is kept iff fewer than
+ *   capacity_left[e] earlier slots of e in this shard were kept, and
+ *   cfg->capacity_factor is not used.  For shard r of a batch with capacity
+ *   C: capacity_left[e] = max(0, C - sum over shards q < r of counts_q[e]),
+ *   counts_q being shard q's counts (gathered from every shard).  NULL: the
+ *   capacity of cfg applies, as in moe_forward.
+ *   -> y [T,H], and optionally counts_out / dropped_out [E] for this shard.
+ * With capacity_left NULL and the routing of moe_route, y equals
+ * moe_forward's bit for bit.
+ */
+moe_status_t moe_forward_routed(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                const float* topk_w, const int32_t* capacity_left, const void* w_gate,
+                                const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                                const void* ws_down, void* y, int32_t* counts_out, int32_t* dropped_out,
+                                void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Waits for `stream`, then returns the device check flags (MOE_DEVFLAG_*)
  * accumulated in `ws` since the last call and clears them.  Returns

@@ -51,6 +51,7 @@ _SIGS = {
     "moe_grouped_ffn": ([ctypes.POINTER(moe_config_t)] + [_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_combine": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_forward": ([ctypes.POINTER(moe_config_t)] + [_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_forward_routed": ([ctypes.POINTER(moe_config_t)] + [_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_get_device_status": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_size_t, _P,
                                ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
     "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -181,6 +182,29 @@ def moe_forward(cfg, x, router_w, router_b, w_gate, w_up, w_down, ws_gate, ws_up
                               _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y),
                               _ptr(topk_idx_out), _ptr(counts_out), _ptr(dropped_out), p, n,
                               _stream(stream)))
+
+
+def moe_forward_routed(cfg, x, topk_idx, topk_w, capacity_left, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y,
+                       counts_out=None, dropped_out=None, ws=None, stream=None):
+    p, n = _ws(ws)
+    _check(load().moe_forward_routed(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(capacity_left),
+                                     _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up),
+                                     _ptr(ws_down), _ptr(y), _ptr(counts_out), _ptr(dropped_out), p, n,
+                                     _stream(stream)))
+
+
+def shard_capacity_left(counts_per_shard, capacity: int, shard: int):
+    """Capacity left for each expert in token shard `shard` of a batch whose
+    capacity is `capacity` (served in global token order): capacity minus the
+    rows the earlier shards kept, i.e. max(0, C - sum_{q < shard} counts_q[e]).
+
+    counts_per_shard: [n_shards, E] integer array (every shard's counts before
+    the capacity cut, gathered from all shards); returns an int32 array [E]."""
+    import numpy as np
+
+    c = np.asarray(counts_per_shard, dtype=np.int64)
+    before = c[:shard].sum(axis=0) if shard > 0 else np.zeros(c.shape[1], np.int64)
+    return np.maximum(0, int(capacity) - before).astype(np.int32)
 
 
 def moe_get_device_status(cfg, ws, stream=None) -> int:

@@ -23,6 +23,7 @@ constexpr int kDecodeMaxSlots = 8;             // T*k limit of the decode FFN ke
 struct Plan {
     int64_t T, H, I, E, k, Is, S;  // S = T*k slots
     int64_t cap;                   // 0 = unlimited
+    const int32_t* cap_left_arr;   // [E] device or null: capacity left per expert (token shards)
     bool bf16;
     int64_t nchunks;               // ceil(S / kPermuteChunk)
     int64_t h_rows;                // S + (Is ? T : 0)
@@ -57,6 +58,14 @@ template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __f
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-z)); }
 
 __device__ __forceinline__ void set_flag(int32_t* flags, int32_t bit) { atomicOr(flags, bit); }
+
+// Capacity of expert e when cap > 0: the per-expert capacity left for this
+// token shard when given (the batch's capacity minus the rows of e that
+// earlier shards kept; capacity is served in global token order), else cap.
+__device__ __forceinline__ int64_t cap_left(int64_t cap, const int32_t* cap_left_arr, int e) {
+    const int64_t left = cap_left_arr ? (int64_t)cap_left_arr[e] : cap;
+    return left > 0 ? left : 0;
+}
 
 // ---- launchers (defined in the .cu files; return the launch error) ------
 // Router for the float32 layer (CUDA cores, float32 FMAs).

@@ -82,6 +82,7 @@ struct DecArgs {
     int32_t* flags;
     int T, H, I, Is, E, k, S, P;
     int64_t cap;
+    const int32_t* cap_left_arr;  // [E] or null: capacity left per expert (token shards)
     int vec_bytes;  // bytes of shared memory before the ring (multiple of 128)
 };
 
@@ -99,8 +100,8 @@ struct DecPlan {
 };
 
 // Capacity in token order: slot s = t*k + j of expert e is kept while fewer
-// than cap earlier slots of e were kept (a token meets an expert at most
-// once, so slot order is token order).
+// than cap_left(e) earlier slots of e were kept (a token meets an expert at
+// most once, so slot order is token order).
 __device__ void build_plan(const DecArgs& a, DecPlan& pl) {
     const int tid = threadIdx.x;
     if (tid < a.S) {
@@ -125,7 +126,7 @@ __device__ void build_plan(const DecArgs& a, DecPlan& pl) {
                 pl.gcnt[ng] = 0;
                 ++ng;
             }
-            if (a.cap > 0 && pl.gcnt[g] >= a.cap) continue;
+            if (a.cap > 0 && pl.gcnt[g] >= cap_left(a.cap, a.cap_left_arr, e)) continue;
             pl.gvec[g][pl.gcnt[g]++] = s;
             pl.kept[s] = 1;
         }
@@ -300,7 +301,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gateup_kernel(const Dec
         for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
             int c = 0;
             for (int s = 0; s < a.S; ++s) c += pl.e_of[s] == e;
-            const int kept = (a.cap > 0 && c > a.cap) ? (int)a.cap : c;
+            const int64_t cl = a.cap > 0 ? cap_left(a.cap, a.cap_left_arr, e) : 0;
+            const int kept = (a.cap > 0 && c > cl) ? (int)cl : c;
             a.counts[e] = c;
             a.dropped[e] = c - kept;
         }
@@ -598,6 +600,7 @@ cudaError_t launch_decode_ffn(const Plan& p, const void* x, const int32_t* topk_
     a.S = (int)p.S;
     a.P = (int)(p.S + (p.Is ? p.T : 0));
     a.cap = p.cap;
+    a.cap_left_arr = p.cap_left_arr;
     cudaError_t e = ensure_smem_attr(decode_gateup_kernel, kDecSmemBytes);
     if (e == cudaSuccess) e = ensure_smem_attr(decode_down_kernel, kDecSmemBytes);
     if (e != cudaSuccess) return e;

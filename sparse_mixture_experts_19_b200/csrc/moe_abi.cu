@@ -81,9 +81,14 @@ static moe_status_t check_config(const moe_config_t* c) {
     return MOE_OK;
 }
 
+// C = ceil(cf * T * k / E).  cf arrives as float32, whose rounding (about
+// 6e-8 relative) can lift an exact integer just above itself (0.8f * 2400 / 8
+// = 240.0000029): the ceiling is taken after removing a relative 1e-6, far
+// below any fractional part a real configuration produces.
 static int64_t capacity_of(const moe_config_t* c) {
     if (c->capacity_factor <= 0.f) return 0;
-    double C = ceil((double)c->capacity_factor * (double)c->T * (double)c->top_k / (double)c->E);
+    const double v = (double)c->capacity_factor * (double)c->T * (double)c->top_k / (double)c->E;
+    const double C = ceil(v - 1e-6 * (v > 1.0 ? v : 1.0));
     return C < 1.0 ? 1 : (int64_t)C;
 }
 
@@ -99,6 +104,7 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->Is = c->I_shared;
     p->S = p->T * p->k;
     p->cap = capacity_of(c);
+    p->cap_left_arr = nullptr;
     p->bf16 = (c->dtype == MOE_BF16);
     p->nchunks = (p->S + kPermuteChunk - 1) / kPermuteChunk;
     p->h_rows = p->S + (p->Is ? p->T : 0);
@@ -324,6 +330,29 @@ moe_status_t moe_combine(const moe_config_t* cfg, const float* expert_out, const
     return MOE_OK;
 }
 
+}  // extern "C"
+
+// Everything after routing: grouping (with a per-expert capacity for a token
+// shard, when given), the expert FFNs and the combine.
+static moe_status_t forward_after_routing(Plan& p, const void* x, const int32_t* idx, const void* w_gate,
+                                          const void* w_up, const void* w_down, const void* ws_gate,
+                                          const void* ws_up, const void* ws_down, void* y, int32_t* counts,
+                                          int32_t* dropped, cudaStream_t st) {
+    if (decode_ffn_eligible(p)) {
+        // few slots: weight-streaming FFN kernels, no grouped rows
+        CUDA_TRY(launch_decode_ffn(p, x, idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, counts, dropped, st),
+                 "decode_ffn");
+        return MOE_OK;
+    }
+    CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
+    moe_status_t s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.rows, p.row_of, st);
+    if (s != MOE_OK) return s;
+    CUDA_TRY(launch_combine_rows(p, p.rows, p.row_of, y, st), "combine_rows");
+    return MOE_OK;
+}
+
+extern "C" {
+
 moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* router_w,
                          const float* router_b, const void* w_gate, const void* w_up,
                          const void* w_down, const void* ws_gate, const void* ws_up,
@@ -354,17 +383,43 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
     CUDA_TRY(run_router(p, x, router_w, router_b, idx, p.topk_w, st), "router");
-    if (decode_ffn_eligible(p)) {
-        // few slots: weight-streaming FFN kernels, no grouped rows
-        CUDA_TRY(launch_decode_ffn(p, x, idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, counts, dropped, st),
-                 "decode_ffn");
+    return forward_after_routing(p, x, idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, counts, dropped, st);
+}
+
+moe_status_t moe_forward_routed(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                const float* topk_w, const int32_t* capacity_left, const void* w_gate,
+                                const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                                const void* ws_down, void* y, int32_t* counts_out, int32_t* dropped_out,
+                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    OPTIONAL_PTR(capacity_left);
+    OPTIONAL_PTR(counts_out);
+    OPTIONAL_PTR(dropped_out);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (p.T == 0) {
+        if (counts_out) CUDA_TRY(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * p.E, st), "memset");
+        if (dropped_out) CUDA_TRY(cudaMemsetAsync(dropped_out, 0, sizeof(int32_t) * p.E, st), "memset");
         return MOE_OK;
     }
-    CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
-    if ((s = run_ffn(p, x, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, 1, p.rows, p.row_of, st)) != MOE_OK)
-        return s;
-    CUDA_TRY(launch_combine_rows(p, p.rows, p.row_of, y, st), "combine_rows");
-    return MOE_OK;
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    REQUIRE_PTR(w_gate);
+    REQUIRE_PTR(w_up);
+    REQUIRE_PTR(w_down);
+    REQUIRE_PTR(y);
+    if ((s = check_shared(p, ws_gate, ws_up, ws_down)) != MOE_OK) return s;
+    p.topk_w = const_cast<float*>(topk_w);  // read only on this path
+    if (capacity_left) {
+        p.cap_left_arr = capacity_left;  // the shard's capacities replace cfg's
+        p.cap = INT32_MAX;               // marks the layer as capped
+    }
+    int32_t* counts = counts_out ? counts_out : p.counts;
+    int32_t* dropped = dropped_out ? dropped_out : p.dropped;
+    return forward_after_routing(p, x, topk_idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, counts, dropped,
+                                 st);
 }
 
 moe_status_t moe_get_device_status(const moe_config_t* cfg, void* ws, size_t ws_bytes,

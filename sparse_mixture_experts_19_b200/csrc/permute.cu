@@ -126,13 +126,15 @@ __global__ void __launch_bounds__(kChunkScanThreads) permute_scan_chunks_kernel(
 // 2b. One block: per-expert totals -> capacity cut, dropped, offsets, and
 // the tile prefixes of the grouped GEMMs.
 __global__ void __launch_bounds__(kScanThreads) permute_scan_experts_kernel(
-    const int32_t* __restrict__ counts, int E, int64_t cap, int32_t* __restrict__ dropped, int32_t* offsets_out,
+    const int32_t* __restrict__ counts, int E, int64_t cap, const int32_t* __restrict__ cap_left_arr,
+    int32_t* __restrict__ dropped, int32_t* offsets_out,
     int32_t* offsets_ws, int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix,
     int32_t shared_rows) {
     __shared__ int32_t sm[kScanThreads];
     const int e = threadIdx.x;
     const int32_t total = (e < E) ? counts[e] : 0;
-    const int32_t kept = (cap > 0 && total > cap) ? (int32_t)cap : total;
+    const int64_t cl = (cap > 0 && e < E) ? cap_left(cap, cap_left_arr, e) : 0;
+    const int32_t kept = (cap > 0 && total > cl) ? (int32_t)cl : total;
     if (e < E) dropped[e] = total - kept;
     const int32_t incl = block_scan_256(kept, sm);
     // offsets_ws [E+2] feeds the GEMMs; offsets_out [E+1] is the caller's copy
@@ -151,7 +153,8 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_experts_kernel(
 // 3. Block c scatters chunk c: warp w ranks the slots of its segment
 // [c*2048 + w*256, +256) from base[c][e] plus the earlier warps' counts.
 __global__ void __launch_bounds__(kScatterWarps * 32) permute_scatter_kernel(
-    const int32_t* __restrict__ idx, int64_t S, int E, int64_t cap, const int32_t* __restrict__ base,
+    const int32_t* __restrict__ idx, int64_t S, int E, int64_t cap, const int32_t* __restrict__ cap_left_arr,
+    const int32_t* __restrict__ base,
     const int32_t* __restrict__ offsets, int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of) {
     __shared__ int32_t run[kScatterWarps][kMaxExperts];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) permute_scatter_kernel(
         if (valid && (peers & lt) == 0) run[warp][ex] += __popc(peers);  // lowest peer updates
         __syncwarp();
         if (s < s1) {
-            if (valid && (cap <= 0 || rank < cap)) {
+            if (valid && (cap <= 0 || rank < cap_left(cap, cap_left_arr, ex))) {
                 const int32_t row = offsets[ex] + rank;
                 perm_rows[row] = (int32_t)s;
                 row_of[s] = row;
@@ -220,13 +223,15 @@ __global__ void permute_fill_tail_kernel(int32_t* __restrict__ perm_rows, int64_
 constexpr int kSmallWarps = kScanThreads / 32;
 
 __global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
-    const int32_t* __restrict__ idx, int S, int E, int64_t cap, int32_t* __restrict__ counts,
+    const int32_t* __restrict__ idx, int S, int E, int64_t cap, const int32_t* __restrict__ cap_left_arr,
+    int32_t* __restrict__ counts,
     int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
     int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix, int32_t shared_rows,
     int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of, int32_t* __restrict__ flags) {
     __shared__ int32_t wcount[kSmallWarps][kScanThreads];  // per warp segment, per expert
     __shared__ int32_t sm[kScanThreads];
     __shared__ int32_t off[kScanThreads + 1];
+    __shared__ int32_t capl[kScanThreads];  // capacity left per expert (when cap > 0)
     const int e = threadIdx.x, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     for (int w = 0; w < kSmallWarps; ++w) wcount[w][e] = 0;
     __syncthreads();
@@ -251,10 +256,12 @@ __global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
         wcount[w][e] = total;  // first rank of warp w's segment in expert e
         total += c;
     }
-    const int32_t kept = (cap > 0 && total > cap) ? (int32_t)cap : total;
+    const int64_t cl = (cap > 0 && e < E) ? cap_left(cap, cap_left_arr, e) : 0;
+    const int32_t kept = (cap > 0 && total > cl) ? (int32_t)cl : total;
     if (e < E) {
         counts[e] = total;
         dropped[e] = total - kept;
+        capl[e] = (int32_t)cl;
     }
     const int32_t incl = block_scan_256(kept, sm);
     if (e < E) {
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
         if (valid && (peers & lt) == 0) wcount[warp][ex] += __popc(peers);
         __syncwarp();
         if (s < s1) {
-            if (valid && (cap <= 0 || rank < cap)) {
+            if (valid && (cap <= 0 || rank < capl[ex])) {
                 const int32_t row = off[ex] + rank;
                 perm_rows[row] = s;
                 row_of[s] = row;
@@ -335,7 +342,7 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
     const int E = (int)p.E;
     if (p.nchunks == 1) {
         trace_before("permute_small", st);
-        permute_small_kernel<<<1, kScanThreads, 0, st>>>(topk_idx, (int)p.S, E, p.cap, counts, dropped, offsets,
+        permute_small_kernel<<<1, kScanThreads, 0, st>>>(topk_idx, (int)p.S, E, p.cap, p.cap_left_arr, counts, dropped, offsets,
                                                          p.offsets, p.mtile_prefix, p.mpair_prefix,
                                                          (int32_t)(p.Is > 0 ? p.T : 0), perm_rows, row_of, p.flags);
         trace_after(st);
@@ -349,12 +356,12 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
     permute_scan_chunks_kernel<<<(unsigned)E, kChunkScanThreads, 0, st>>>(p.chunk_base, p.nchunks, E, counts);
     trace_after(st);
     trace_before("permute_scan", st);
-    permute_scan_experts_kernel<<<1, kScanThreads, 0, st>>>(counts, E, p.cap, dropped, offsets, p.offsets,
+    permute_scan_experts_kernel<<<1, kScanThreads, 0, st>>>(counts, E, p.cap, p.cap_left_arr, dropped, offsets, p.offsets,
                                                             p.mtile_prefix, p.mpair_prefix,
                                                             (int32_t)(p.Is > 0 ? p.T : 0));
     trace_after(st);
     trace_before("permute_scatter", st);
-    permute_scatter_kernel<<<(unsigned)p.nchunks, kScatterWarps * 32, 0, st>>>(topk_idx, p.S, E, p.cap,
+    permute_scatter_kernel<<<(unsigned)p.nchunks, kScatterWarps * 32, 0, st>>>(topk_idx, p.S, E, p.cap, p.cap_left_arr,
                                                                                 p.chunk_base, p.offsets,
                                                                                 perm_rows, row_of);
     trace_after(st);
