@@ -126,6 +126,40 @@ def test_stage_calls_validate(lib):
     assert lib.moe_combine(ctypes.byref(c), FAKE, FAKE, FAKE, None, FAKE, need, None) == 1
 
 
+def call_forward_routed(lib, c, ws, ws_bytes, **ptrs):
+    p = dict(x=FAKE, topk_idx=FAKE, topk_w=FAKE, capacity_left=None, w_gate=FAKE, w_up=FAKE, w_down=FAKE,
+             ws_gate=None, ws_up=None, ws_down=None, y=FAKE)
+    p.update(ptrs)
+    return lib.moe_forward_routed(ctypes.byref(c), p["x"], p["topk_idx"], p["topk_w"], p["capacity_left"],
+                                  p["w_gate"], p["w_up"], p["w_down"], p["ws_gate"], p["ws_up"], p["ws_down"],
+                                  p["y"], None, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("field", ["x", "topk_idx", "topk_w", "w_gate", "w_up", "w_down", "y"])
+def test_forward_routed_rejects_null_and_misaligned_pointers(lib, field):
+    c = cfg(capacity_factor=1.0)
+    need = lib.moe_workspace_size(ctypes.byref(c))
+    assert call_forward_routed(lib, c, FAKE, need, **{field: None}) == 1
+    assert field in moe.moe_last_error()
+    assert call_forward_routed(lib, c, FAKE, need, **{field: FAKE + 4}) == 1
+
+
+def test_forward_routed_optional_capacity_must_be_aligned(lib):
+    c = cfg(capacity_factor=1.0)
+    need = lib.moe_workspace_size(ctypes.byref(c))
+    assert call_forward_routed(lib, c, FAKE, need, capacity_left=FAKE + 8) == 1
+    assert "capacity_left" in moe.moe_last_error()
+    assert call_forward_routed(lib, c, FAKE, need - 1) == 3
+    assert call_forward_routed(lib, cfg(T=0), FAKE, need, x=None, y=None) == 0
+
+
+def test_capacity_ceiling_ignores_float32_rounding_of_the_factor(lib):
+    # 0.8 is stored as 0.800000012 in float32; 0.8 * 1200 * 2 / 8 = 240 exactly
+    assert moe.capacity(cfg(T=1200, E=8, top_k=2, capacity_factor=0.8)) == 240
+    assert moe.capacity(cfg(T=1201, E=8, top_k=2, capacity_factor=0.8)) == 241
+    assert moe.capacity(cfg(T=3000, E=128, top_k=8, capacity_factor=1.25)) == 235
+
+
 def test_status_strings(lib):
     for code, name in moe.STATUS.items():
         assert moe.moe_status_string(code) == name
