@@ -8,7 +8,9 @@ both read their inputs from the seeded generator in ``moe_inputs``.
 What it computes, per token (see ``moe_oracle.c`` for the sources):
 score -> top-k (ties to the lower expert index) -> softmax over the k selected
 scores -> capacity drop in token order -> weighted sum of the selected SwiGLU
-experts (+ the always-on shared expert).
+experts (+ the always-on shared expert).  Router statistics for the
+load-balance penalties: per-expert importance (sum over tokens of the softmax
+over all E scores) and the penalties built from it and the top-k counts.
 
 Parity pins of every function here live in ``tests/test_oracle.py``.
 """
@@ -164,3 +166,44 @@ def expert_rows(x, w_gate, w_up, w_down, tokens, experts, dtype: str) -> np.ndar
     xs = np.ascontiguousarray(np.asarray(x)[tokens])
     e = np.asarray(experts, np.int32).reshape(-1, 1)
     return moe_tokens(xs, w_gate, w_up, w_down, e, np.ones(e.shape), dtype)
+
+
+def importance(logits) -> np.ndarray:
+    """Per-expert importance: the sum over tokens of the softmax over ALL E
+    scores of each token (fp64), the router statistic the load-balance
+    penalties start from ("2026年人工智能MoE混合专家模型入门指南", the MoE
+    layer's load-balance loss; "模型的“分工的艺术”：MoE技术如何提升计算效率",
+    section 3.1, mean gate probability per expert = importance / T).  The
+    scores include the router bias."""
+    l = np.asarray(logits, np.float64)
+    p = np.exp(l - l.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return p.sum(axis=0)
+
+
+def balance_losses(importance_e, load_e, T: int) -> dict:
+    """The pages' two load-balance penalties from per-expert statistics (fp64).
+
+    kl  -- "模型的“分工的艺术”...", section 3.1: KL(uniform || mean gate
+           probability), mean probability q_e = importance_e / T, target
+           1/E, log(q_e + 1e-8), and the sum divided by E (the mean over the
+           first and only dimension of the E-vector).
+    std -- "2026年人工智能MoE...", MoE layer: std(importance) + std(load),
+           unbiased standard deviations (divisor E - 1).  load_e is the
+           number of tokens whose selection includes e (top-k counts): the
+           page's literal load, the number of positive dense-softmax
+           probabilities, equals T for every expert.
+    switch -- E * sum_e (load_e / T) * (importance_e / T): fraction of tokens
+           routed to e times its mean gate probability, the Switch-Transformer
+           form (the pages name Switch Transformer's routing in "模型的“分工的
+           艺术”...", section 1.2, without a formula).
+    """
+    imp = np.asarray(importance_e, np.float64)
+    load = np.asarray(load_e, np.float64)
+    E = imp.size
+    q = imp / T
+    target = np.full(E, 1.0 / E)
+    kl = float(np.sum(target * (np.log(target) - np.log(q + 1e-8))) / E)
+    std = float(np.std(imp, ddof=1) + np.std(load, ddof=1))
+    switch = float(E * np.sum((load / T) * (imp / T)))
+    return dict(kl=kl, std=std, switch=switch)

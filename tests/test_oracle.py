@@ -11,6 +11,10 @@ Each test pins one step of the method to an independent fact:
   * brute force over all k-subsets on tiny shapes;
   * invariants: weights sum to 1, counts sum to T*k, capacity bookkeeping,
     unselected experts do not matter, token-permutation invariance;
+  * load-balance statistics: importance against the routing weights at
+    k = E, the logistic closed form and uniform cases; the penalties against
+    transformers' Mixtral load-balancing loss and the torch calls (kl_div,
+    std) the pages' snippets make;
   * hand-built golden fixtures under tests/golden/.
 """
 import itertools
@@ -131,6 +135,85 @@ def test_weights_sum_to_one_and_follow_scores(E, k):
     np.testing.assert_allclose(pk / pk.sum(1, keepdims=True), w, rtol=0, atol=1e-15)
     # the selected probabilities are the k largest of the full softmax
     assert np.all(pk.min(1) >= np.sort(p, 1)[:, -k] - 1e-15)
+
+
+# ------------------------------------------------- load-balance statistics
+
+def test_importance_with_top_k_equal_E_is_the_sum_of_routing_weights():
+    """With k = E the routing weights are the softmax over all E scores, so
+    their per-expert sum over tokens is the importance (and it sums to T)."""
+    wl = small(T=90, H=40, E=16, k=16, dtype="bf16", zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    logits, idx, w = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+    from_route = np.zeros(wl.E)
+    np.add.at(from_route, idx.ravel(), w.ravel())
+    imp = oracle.importance(logits)
+    np.testing.assert_allclose(imp, from_route, rtol=1e-13, atol=0)
+    assert abs(imp.sum() - wl.T) <= 1e-12 * wl.T
+
+
+def test_importance_of_two_experts_is_a_sum_of_logistics():
+    wl = small(T=120, H=32, E=2, k=1)
+    inp = mi.make_inputs(wl)
+    logits, _, _ = oracle.route(inp["x"], inp["router_w"], None, 1, "f32")
+    imp = oracle.importance(logits)
+    ref0 = np.sum(1.0 / (1.0 + np.exp(logits[:, 1] - logits[:, 0])))
+    assert abs(imp[0] - ref0) <= 1e-12 * wl.T
+    assert abs(imp[1] - (wl.T - ref0)) <= 1e-12 * wl.T
+
+
+def test_importance_of_identical_router_rows_is_uniform():
+    wl = small(T=33, H=24, E=8, k=2)
+    inp = mi.make_inputs(wl)
+    rw = np.repeat(inp["router_w"][:1], wl.E, axis=0)
+    logits, _, _ = oracle.route(inp["x"], rw, None, wl.k, "f32")
+    assert np.array_equal(oracle.importance(logits), np.full(wl.E, wl.T / wl.E))
+
+
+def test_importance_follows_a_permutation_of_the_experts():
+    wl = small(T=64, H=32, E=12, k=3, dtype="bf16", zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    perm = np.random.default_rng(3).permutation(wl.E)
+    l1, _, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+    l2, _, _ = oracle.route(inp["x"], inp["router_w"][perm], inp["router_b"][perm], wl.k, wl.dtype)
+    np.testing.assert_allclose(oracle.importance(l2), oracle.importance(l1)[perm], rtol=1e-14, atol=0)
+
+
+def test_switch_loss_matches_transformers_mixtral_load_balancing():
+    from transformers.models.mixtral.modeling_mixtral import load_balancing_loss_func
+    wl = small(T=200, H=48, E=8, k=2, dtype="bf16", zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    logits, idx, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+    counts = oracle.permute(idx, wl.E)["counts"]
+    got = oracle.balance_losses(oracle.importance(logits), counts, wl.T)["switch"]
+    ref = load_balancing_loss_func((torch.from_numpy(logits),), wl.E, wl.k).item()
+    assert abs(got - ref) <= 1e-9 * abs(ref)
+
+
+@pytest.mark.parametrize("case", ["uniform", "collapsed", "random"])
+def test_kl_and_std_losses_match_the_torch_calls_of_the_pages(case):
+    """KL: torch.nn.functional.kl_div(log(q + 1e-8), 1/E, reduction="batchmean")
+    on the mean gate probability q; std: torch.std (unbiased) of importance and
+    load, the calls the pages' snippets make."""
+    E, T = 8, 100
+    if case == "uniform":
+        imp, load = np.full(E, T / E), np.full(E, 25.0)
+    elif case == "collapsed":
+        imp, load = np.eye(E)[0] * T, np.eye(E)[0] * 2 * T
+    else:
+        rng = np.random.default_rng(7)
+        imp = rng.dirichlet(np.ones(E)) * T
+        load = rng.integers(0, 2 * T, E).astype(np.float64)
+    got = oracle.balance_losses(imp, load, T)
+    q = torch.from_numpy(imp / T)
+    kl = torch.nn.functional.kl_div(torch.log(q + 1e-8), torch.full((E,), 1.0 / E, dtype=torch.float64),
+                                    reduction="batchmean").item()
+    std = (torch.std(torch.from_numpy(imp)) + torch.std(torch.from_numpy(load))).item()
+    assert abs(got["kl"] - kl) <= 1e-12 * max(1.0, abs(kl))
+    assert abs(got["std"] - std) <= 1e-12 * max(1.0, abs(std))
+    if case == "uniform":
+        assert got["std"] == 0.0 and abs(got["kl"] + math.log1p(E * 1e-8) / E) < 1e-15
+        assert abs(got["switch"] - 2.0) < 1e-12  # E * sum (2T/E / T)(1/E) = k with k = 2
 
 
 # ---------------------------------------------------------------- grouping
