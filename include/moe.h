@@ -119,6 +119,29 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* route
                        size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_route_importance -- moe_route plus the router statistic that the
+ * load-balance penalties start from ("2026年人工智能MoE混合专家模型入门指南",
+ * the MoE layer's importance = softmax probabilities summed over tokens;
+ * "模型的“分工的艺术”：MoE技术如何提升计算效率", section 3.1, mean gate
+ * probability per expert = importance / T).  topk_idx and topk_w are those
+ * of moe_route, bit for bit.
+ *   importance [E] float32, device, 16-byte aligned, required: ADDED to
+ *   (the caller zeroes it, or keeps summing over batches):
+ *   importance[e] += sum over tokens t of exp(s[t,e] - m_t) / sum_e' exp(s[t,e'] - m_t),
+ *   s the router scores with bias, m_t the token's largest score.  The
+ *   probabilities come from the scores moe_route computes (float32
+ *   tensor-core sums on the tensor-core path; exact scores on the few-token
+ *   path) and are summed with float32 atomic adds, so the order of the sum,
+ *   and its last bits, vary from run to run.  With T = 0 nothing is added.
+ * The top-k counts, the other statistic, come from moe_permute (counts) or
+ * moe_forward (counts_out).  Errors: as moe_route, and importance NULL or
+ * misaligned is MOE_ERR_INVALID_ARG.
+ */
+moe_status_t moe_route_importance(const moe_config_t* cfg, const void* x, const void* router_w,
+                                  const float* router_b, int32_t* topk_idx, float* topk_w, float* importance,
+                                  void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_permute -- group (token, slot) pairs by expert, with capacity drop in
  * token order ("Mixture of Experts (MoEs) in Transformers", section Expert
  * Backend: grouped_mm sorts tokens by expert id; "MoE稀疏架构是什么？…",

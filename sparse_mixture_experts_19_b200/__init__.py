@@ -45,6 +45,8 @@ _SIGS = {
     "moe_workspace_size": ([ctypes.POINTER(moe_config_t)], ctypes.c_size_t),
     "moe_capacity": ([ctypes.POINTER(moe_config_t)], ctypes.c_int64),
     "moe_route": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_route_importance": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+                             ctypes.c_int),
     "moe_permute": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
                     ctypes.c_int),
     "moe_permute_noalloc": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
@@ -144,6 +146,40 @@ def moe_route(cfg, x, router_w, router_b, topk_idx, topk_w, ws, stream=None):
     p, n = _ws(ws)
     _check(load().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(topk_idx),
                             _ptr(topk_w), p, n, _stream(stream)))
+
+
+def moe_route_importance(cfg, x, router_w, router_b, topk_idx, topk_w, importance, ws, stream=None):
+    """moe_route, and the softmax over all E scores of each token added to
+    importance [E] float32 (the caller zeroes it)."""
+    _check(load().moe_route_importance(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b),
+                                       _ptr(topk_idx), _ptr(topk_w), _ptr(importance), *_ws(ws), _stream(stream)))
+
+
+def balance_losses(importance, load, T: int) -> dict:
+    """Load-balance penalties from the per-expert statistics (host arithmetic
+    on E numbers; importance from moe_route_importance, load = the top-k
+    counts from moe_permute or moe_forward):
+      kl     = (1/E) sum_e (1/E) (log(1/E) - log(importance_e / T + 1e-8)),
+               KL from uniform to the mean gate probability
+               ("模型的“分工的艺术”…", section 3.1);
+      std    = std(importance) + std(load), unbiased
+               ("2026年人工智能MoE混合专家模型入门指南", MoE layer; the page's
+               load, a count of positive softmax probabilities, is T for every
+               expert, so the top-k counts stand in for it);
+      switch = E sum_e (load_e / T)(importance_e / T), the Switch-Transformer
+               form."""
+    import numpy as np
+    imp = np.asarray(importance, dtype=np.float64).ravel()
+    ld = np.asarray(load, dtype=np.float64).ravel()
+    E = imp.size
+    if E < 2 or ld.size != E or T <= 0:
+        raise ValueError("need E >= 2 experts, matching lengths and T > 0")
+    mean_prob = imp / T
+    kl = float(np.sum((np.log(1.0 / E) - np.log(mean_prob + 1e-8)) / E) / E)
+    dev_i, dev_l = imp - imp.mean(), ld - ld.mean()
+    std = float(np.sqrt(np.dot(dev_i, dev_i) / (E - 1)) + np.sqrt(np.dot(dev_l, dev_l) / (E - 1)))
+    switch = float(E * np.dot(ld / T, mean_prob))
+    return dict(kl=kl, std=std, switch=switch)
 
 
 def moe_permute(cfg, topk_idx, counts, offsets, perm_rows, row_of, dropped, ws, stream=None):

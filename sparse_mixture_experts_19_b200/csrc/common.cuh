@@ -24,6 +24,7 @@ struct Plan {
     int64_t T, H, I, E, k, Is, S;  // S = T*k slots
     int64_t cap;                   // 0 = unlimited
     const int32_t* cap_left_arr;   // [E] device or null: capacity left per expert (token shards)
+    float* importance;             // [E] device or null: router importance, added to
     bool bf16;
     int64_t nchunks;               // ceil(S / kPermuteChunk)
     int64_t h_rows;                // S + (Is ? T : 0)

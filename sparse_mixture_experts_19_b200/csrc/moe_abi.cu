@@ -105,6 +105,7 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->S = p->T * p->k;
     p->cap = capacity_of(c);
     p->cap_left_arr = nullptr;
+    p->importance = nullptr;
     p->bf16 = (c->dtype == MOE_BF16);
     p->nchunks = (p->S + kPermuteChunk - 1) / kPermuteChunk;
     p->h_rows = p->S + (p->Is ? p->T : 0);
@@ -240,6 +241,25 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* route
     OPTIONAL_PTR(router_b);
     REQUIRE_PTR(topk_idx);
     REQUIRE_PTR(topk_w);
+    cudaStream_t st = (cudaStream_t)stream;
+    CUDA_TRY(run_router(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
+    return MOE_OK;
+}
+
+moe_status_t moe_route_importance(const moe_config_t* cfg, const void* x, const void* router_w,
+                                  const float* router_b, int32_t* topk_idx, float* topk_w, float* importance,
+                                  void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    REQUIRE_PTR(importance);
+    if (p.T == 0) return MOE_OK;
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(router_w);
+    OPTIONAL_PTR(router_b);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    p.importance = importance;
     cudaStream_t st = (cudaStream_t)stream;
     CUDA_TRY(run_router(p, x, router_w, router_b, topk_idx, topk_w, st), "router");
     return MOE_OK;

@@ -15,6 +15,8 @@
 // through distributed shared memory, picks the k best by (score desc, index
 // asc) with warp arg-max rounds and writes the softmax of those k; a second
 // cluster barrier keeps the other CTAs' shared memory alive until then.
+// When asked, the same warp adds the token's softmax over all E scores
+// (fp64, from the exact scores) to the per-expert importance.
 #include <algorithm>
 
 #include "common.cuh"
@@ -59,7 +61,8 @@ __device__ __forceinline__ void chunk_dot(const uint4& xq, const uint4& wq, doub
 template <typename TIn>
 __global__ void __launch_bounds__(kWarps * 32) router_decode_kernel(
     int T, int H, int E, int k, int C, int epc, const TIn* __restrict__ x, const TIn* __restrict__ wr,
-    const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    float* __restrict__ importance) {
     constexpr int V = 16 / sizeof(TIn);  // elements per 16-byte chunk
     __shared__ double sc[kMaxExperts];   // this CTA's scores; CTA 0 gathers all E here
     const int t = blockIdx.x / C;  // clusters of C consecutive CTAs along x, one per token
@@ -138,6 +141,14 @@ __global__ void __launch_bounds__(kWarps * 32) router_decode_kernel(
                 topk_w[(int64_t)t * k + j] = expf((float)(sel_v[j] - sel_v[0])) * inv;
             }
         }
+        if (importance) {
+            // softmax over all E scores, shifted by the largest (sel_v[0])
+            double z = 0.0;
+            for (int e = lane; e < E; e += 32) z += exp(sc[e] - sel_v[0]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            for (int e = lane; e < E; e += 32) atomicAdd(&importance[e], (float)(exp(sc[e] - sel_v[0]) / z));
+        }
     }
     cluster_sync();  // CTA 0 has read every CTA's scores
 }
@@ -162,7 +173,7 @@ cudaError_t launch_typed(const Plan& p, const void* x, const void* router_w, con
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, router_decode_kernel<TIn>, (int)p.T, (int)p.H, E, (int)p.k, C, epc,
-                              (const TIn*)x, (const TIn*)router_w, router_b, topk_idx, topk_w);
+                              (const TIn*)x, (const TIn*)router_w, router_b, topk_idx, topk_w, p.importance);
 }
 
 }  // namespace

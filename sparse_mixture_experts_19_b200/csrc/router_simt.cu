@@ -9,6 +9,9 @@
 // chunks of 32 columns are staged in shared memory as float; each thread owns
 // up to 32 (token, expert) accumulators.  The scores then go to shared memory
 // and each warp selects the top-k of 4 tokens with warp arg-max rounds.
+// When asked, each warp also forms its tokens' softmax over all E scores; the
+// block sums them per expert in shared memory and adds the sums to the
+// importance in global memory.
 #include "common.cuh"
 
 namespace moe {
@@ -34,13 +37,16 @@ __device__ __forceinline__ void warp_argmax(float& v, int& e) {
 template <typename TIn>
 __global__ void __launch_bounds__(kThreads) router_simt_kernel(
     int T, int H, int E, int k, const TIn* __restrict__ x, const TIn* __restrict__ wr,
-    const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    const float* __restrict__ b, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    float* __restrict__ importance) {
     __shared__ float xs[kTB][kHC + 1];
+    __shared__ float imp[kMaxExperts];  // this block's importance, when asked
     // weights chunk [E][kHC+1] during the scores, then scores [kTB][E+1]
     __shared__ float buf[kMaxExperts * (kHC + 1)];
 
     const int tid = threadIdx.x;
     const int t0 = blockIdx.x * kTB;
+    for (int e = tid; e < kMaxExperts; e += kThreads) imp[e] = 0.f;  // ordered by the loop's barriers
     const int P = kTB * E;  // (token, expert) pairs of this block
 
     float acc[kTB * kMaxExperts / kThreads];
@@ -118,6 +124,19 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(
                 topk_w[(int64_t)t * k + j] = expf(sel_v[j] - m) * inv;
             }
         }
+        if (importance) {
+            // softmax over all E scores, shifted by the largest (sel_v[0])
+            float z = 0.f;
+            for (int e = lane; e < E; e += 32) z += expf(l[e] - sel_v[0]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            const float inv = 1.0f / z;
+            for (int e = lane; e < E; e += 32) atomicAdd(&imp[e], expf(l[e] - sel_v[0]) * inv);
+        }
+    }
+    if (importance) {
+        __syncthreads();
+        for (int e = tid; e < E; e += kThreads) atomicAdd(&importance[e], imp[e]);
     }
 }
 
@@ -131,7 +150,7 @@ cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_
     trace_before("router_simt", st);
     router_simt_kernel<float><<<grid, kThreads, 0, st>>>((int)p.T, (int)p.H, (int)p.E, (int)p.k,
                                                          (const float*)x, (const float*)router_w,
-                                                         router_b, topk_idx, topk_w);
+                                                         router_b, topk_idx, topk_w, p.importance);
     trace_after(st);
     return cudaGetLastError();
 }

@@ -22,6 +22,12 @@
 // fp64 (bf16 products are exact) by warp-cooperative dot products, and its
 // selection is completed from those exact scores.  Experts above the band
 // are certainly selected, experts below it certainly not.
+//
+// Importance (optional).  Before the accumulator is handed back, each thread
+// forms its token's softmax over all E float32 scores, each warp sums the 32
+// tokens' probabilities per expert by a reduce-scatter over its lanes (lane l
+// ends with expert c0 + l of a 32-column block) and adds the sums to the
+// importance in global memory: one atomic add per expert, warp and tile.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
@@ -106,6 +112,23 @@ __device__ __forceinline__ bool epilogue_any(bool pred) {
 
 __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Column sums of a warp's 32 x 32 values (v[i] of lane l is row l, column i):
+// five exchange steps, each halving the columns a lane keeps; afterwards v[0]
+// of lane l holds the sum of column l over all 32 lanes.
+__device__ __forceinline__ float warp_column_sum32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float send = upper ? v[i] : v[i + o];
+            const float keep = upper ? v[i + o] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
 // KMAX: capacity of the per-thread selection (k <= KMAX).  KMAX = kMaxTopK
 // serves only k == E (every expert selected), where no decision is uncertain.
 template <int KMAX>
@@ -113,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int H, int E,
     int Npad, int k, int stages, uint32_t acc_cols, const float* __restrict__ bias,
     const bf16* __restrict__ x_rows, const bf16* __restrict__ wr_rows, int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_w, int32_t* flags) {
+    float* __restrict__ topk_w, float* __restrict__ importance, int32_t* flags) {
     constexpr bool kDense = (KMAX == kMaxTopK);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -384,6 +407,28 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                         }
                     }
             }
+            if (importance) {
+                // token's softmax over all E scores (TMEM holds them biased),
+                // shifted by the largest (tv[0]); rows past T add nothing
+                __syncwarp();
+                const float m = tv[0];
+                float z = 0.f;
+                for (int c0 = 0; c0 < E; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tq + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) z += (c0 + i < E) ? expf(v[i] - m) : 0.f;
+                }
+                const float inv = 1.0f / z;
+                for (int c0 = 0; c0 < E; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tq + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = (t < T && c0 + i < E) ? expf(v[i] - m) * inv : 0.f;
+                    const float colsum = warp_column_sum32(v, lane);
+                    if (c0 + lane < E) atomicAdd(&importance[c0 + lane], colsum);
+                }
+            }
             // the accumulator is no longer needed: hand it back to the MMA warp
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
@@ -469,13 +514,14 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
         if (e == cudaSuccess)
             router_sm100_kernel<8><<<grid, kThreads, smem, st>>>(mx, mw, (int)p.T, (int)p.H, E, Npad, (int)p.k,
                                                                stages, cols, router_b, (const bf16*)x,
-                                                               (const bf16*)router_w, topk_idx, topk_w, p.flags);
+                                                               (const bf16*)router_w, topk_idx, topk_w,
+                                                               p.importance, p.flags);
     } else {
         e = ensure_smem_attr(router_sm100_kernel<kMaxTopK>, smem);
         if (e == cudaSuccess)
             router_sm100_kernel<kMaxTopK><<<grid, kThreads, smem, st>>>(
                 mx, mw, (int)p.T, (int)p.H, E, Npad, (int)p.k, stages, cols, router_b, (const bf16*)x,
-                (const bf16*)router_w, topk_idx, topk_w, p.flags);
+                (const bf16*)router_w, topk_idx, topk_w, p.importance, p.flags);
     }
     trace_after(st);
     return e != cudaSuccess ? e : cudaGetLastError();

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import sparse_mixture_experts_19_b200 as moe
@@ -124,6 +125,39 @@ def test_stage_calls_validate(lib):
     assert lib.moe_grouped_ffn(ctypes.byref(c), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, None, FAKE,
                                FAKE, need, None) == 1
     assert lib.moe_combine(ctypes.byref(c), FAKE, FAKE, FAKE, None, FAKE, need, None) == 1
+
+
+def test_route_importance_validates(lib):
+    c = cfg(T=300, E=16, top_k=4)
+    need = lib.moe_workspace_size(ctypes.byref(c))
+
+    def call(**kw):
+        p = dict(x=FAKE, router_w=FAKE, router_b=None, topk_idx=FAKE, topk_w=FAKE, importance=FAKE)
+        p.update(kw)
+        return lib.moe_route_importance(ctypes.byref(c), p["x"], p["router_w"], p["router_b"],
+                                        p["topk_idx"], p["topk_w"], p["importance"], FAKE, need, None)
+
+    assert call(importance=None) == 1 and "importance" in moe.moe_last_error()
+    assert call(importance=FAKE + 4) == 1
+    for field in ("x", "router_w", "topk_idx", "topk_w"):
+        assert call(**{field: None}) == 1 and field in moe.moe_last_error()
+    assert call(router_b=FAKE + 8) == 1
+    c0 = cfg(T=0, E=16, top_k=4)
+    assert lib.moe_route_importance(ctypes.byref(c0), None, None, None, None, None, FAKE, FAKE, need, None) == 0
+
+
+def test_balance_losses_host_helper_matches_oracle():
+    import oracle
+    rng = np.random.default_rng(11)
+    for E, T in ((2, 10), (8, 1000), (256, 16384)):
+        imp = rng.dirichlet(np.ones(E)) * T
+        load = rng.integers(0, 8 * T // E + 1, E)
+        got = moe.balance_losses(imp, load, T)
+        ref = oracle.balance_losses(imp, load, T)
+        for key in ("kl", "std", "switch"):
+            assert abs(got[key] - ref[key]) <= 1e-12 * max(1.0, abs(ref[key])), (E, key)
+    with pytest.raises(ValueError):
+        moe.balance_losses(np.ones(1), np.ones(1), 4)
 
 
 def call_forward_routed(lib, c, ws, ws_bytes, **ptrs):
