@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", choices=["forward", "route"], default="forward",
                     help="route: time moe_route alone (only x and the router weights are allocated)")
+    ap.add_argument("--importance", action="store_true",
+                    help="with --stage route: also time moe_route_importance (router importance as a side output)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step from the host instead of replaying a CUDA graph of the K steps")
     return ap.parse_args()
@@ -523,24 +525,34 @@ def run_route_stage(args, wl):
     ws = moe.workspace(cfg)
     idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
     w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
-    for _ in range(args.warmup):
-        moe.moe_route(cfg, x, rw, rb, idx, w, ws)
-    torch.cuda.synchronize()
-    moe.moe_trace_begin(8 * args.steps)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        moe.moe_route(cfg, x, rw, rb, idx, w, ws)
-    e1.record()
-    torch.cuda.synchronize()
-    trace = moe.moe_trace_end(8 * args.steps)
-    ms = e0.elapsed_time(e1) / args.steps
-    kern = {}
-    for name, t in trace:
-        kern.setdefault(name, []).append(t)
-    return {"stage": "route", "config": config_of(wl), "ms_per_call": ms, "tokens_per_s": wl.T / (ms / 1e3),
-            "x_bytes_per_s": wl.T * wl.H * (2 if wl.dtype == "bf16" else 4) / (ms / 1e3),
-            "kernels_ms_per_call": {k: sum(v) / len(v) for k, v in kern.items()}}
+    imp = torch.zeros(wl.E, dtype=torch.float32, device="cuda")
+
+    def timed(call):
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        moe.moe_trace_begin(8 * args.steps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        trace = moe.moe_trace_end(8 * args.steps)
+        kern = {}
+        for name, t in trace:
+            kern.setdefault(name, []).append(t)
+        return e0.elapsed_time(e1) / args.steps, {k: sum(v) / len(v) for k, v in kern.items()}
+
+    ms, kern = timed(lambda: moe.moe_route(cfg, x, rw, rb, idx, w, ws))
+    out = {"stage": "route", "config": config_of(wl), "ms_per_call": ms, "tokens_per_s": wl.T / (ms / 1e3),
+           "x_bytes_per_s": wl.T * wl.H * (2 if wl.dtype == "bf16" else 4) / (ms / 1e3),
+           "kernels_ms_per_call": kern}
+    if args.importance:
+        ms_i, kern_i = timed(lambda: moe.moe_route_importance(cfg, x, rw, rb, idx, w, imp, ws))
+        out["importance"] = {"ms_per_call": ms_i, "kernels_ms_per_call": kern_i,
+                             "sum_over_calls_per_T": float(imp.sum().item()) / wl.T}
+    return out
 
 
 def main():
