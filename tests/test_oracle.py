@@ -179,6 +179,24 @@ def test_importance_follows_a_permutation_of_the_experts():
     np.testing.assert_allclose(oracle.importance(l2), oracle.importance(l1)[perm], rtol=1e-14, atol=0)
 
 
+def test_importance_and_penalties_golden():
+    g = json.load(open(os.path.join(GOLDEN, "importance_bias_only.json")))
+    for case in g["cases"]:
+        b = np.array(case["bias"], np.float32)
+        E, T, k = len(b), case["T"], case["k"]
+        x = np.zeros((T, 8), np.float32)
+        rw = mi.normal(0, 99, (E, 8), 1.0, "f32")
+        logits, idx, _ = oracle.route(x, rw, b, k, "f32")
+        imp = oracle.importance(logits)
+        np.testing.assert_allclose(imp, case["importance"], rtol=1e-7, atol=0)
+        if case["load"] is not None:
+            load = oracle.permute(idx, E)["counts"]
+            assert load.tolist() == case["load"]
+            got = oracle.balance_losses(imp, load, T)
+            for key in ("kl", "std", "switch"):
+                assert abs(got[key] - case[key]) <= 1e-6 * abs(case[key]), key
+
+
 def test_switch_loss_matches_transformers_mixtral_load_balancing():
     from transformers.models.mixtral.modeling_mixtral import load_balancing_loss_func
     wl = small(T=200, H=48, E=8, k=2, dtype="bf16", zipf_s=1.1)
