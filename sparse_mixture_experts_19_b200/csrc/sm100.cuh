@@ -2,8 +2,12 @@
 // tensor loads, and the 5th-generation tensor core (tcgen05) with its tensor
 // memory (TMEM).  Only the forms used by the kernels of this library.
 //
-// Conventions: one CTA is its own cluster (no clusters, no multicast);
-// operands are K-major bf16 tiles in shared memory with the 128-byte swizzle
+// Conventions: a CTA is its own cluster, except in the CTA-pair GEMM
+// (clusters of 2, cta_group::2; a tcgen05.commit multicast to both CTAs
+// signals MMA completion) and the few-token router (clusters of up to 8
+// sharing scores through distributed shared memory); no TMA or bulk load
+// uses cluster multicast.
+// Operands are K-major bf16 tiles in shared memory with the 128-byte swizzle
 // (8 rows x 128 B atoms, 1024-byte aligned); accumulators are float32 in TMEM.
 #pragma once
 
