@@ -34,7 +34,7 @@ def _max_worker(rank, world, port, out):
 def test_reduce_max_and_job_throughput_two_ranks():
     world = 2
     port = free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_max_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
@@ -102,7 +102,7 @@ def test_expert_parallel_partials_sum_to_the_layer_two_ranks():
 
     world = 2
     port = free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_ep_worker, args=(world, port, out), nprocs=world, join=True)
         ys = [out[r] for r in range(world)]

@@ -67,7 +67,7 @@ def _shard_worker(rank, world, port, out):
 def test_shard_capacity_exchange_matches_global_order_two_ranks():
     world = 2
     port = free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
         kept = np.concatenate([out[r] for r in range(world)])
