@@ -213,3 +213,9 @@ def test_product_path_does_not_import_the_oracle():
                 src = open(os.path.join(root, f), encoding="utf-8").read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "moe_oracle" not in src, f
+
+
+def test_missing_library_raises_instead_of_falling_back(tmp_path):
+    with pytest.raises(moe.MoeError) as e:
+        moe.load(str(tmp_path / "libmoe.so"))
+    assert "missing" in str(e.value)
