@@ -41,6 +41,8 @@ STREAM_WS_UP = 7
 STREAM_WS_DOWN = 8
 STREAM_ZIPF_RANK = 9
 STREAM_SAMPLE = 10
+STREAM_MX_GATE, STREAM_MX_UP, STREAM_MX_DOWN = 11, 12, 13        # mxfp4 element codes
+STREAM_MXS_GATE, STREAM_MXS_UP, STREAM_MXS_DOWN = 14, 15, 16     # mxfp4 block scales
 
 
 def build(force: bool = False) -> str:
@@ -63,6 +65,7 @@ def _L():
         _lib.moe_gen_normal_f32.argtypes = [u64, u64, u64, i64, ctypes.c_double, ctypes.c_void_p]
         _lib.moe_gen_normal_bf16.argtypes = [u64, u64, u64, i64, ctypes.c_double, ctypes.c_void_p]
         _lib.moe_gen_permutation.argtypes = [u64, u64, ctypes.c_int32, ctypes.c_void_p]
+        _lib.moe_gen_bytes.argtypes = [u64, u64, u64, i64, ctypes.c_void_p]
         _lib.moe_gen_u64.argtypes = [u64, u64, u64]
         _lib.moe_gen_u64.restype = u64
     return _lib
@@ -89,6 +92,42 @@ def permutation(seed: int, stream: int, n: int) -> np.ndarray:
     out = np.empty(n, dtype=np.int32)
     _L().moe_gen_permutation(seed, stream, n, out.ctypes.data)
     return out
+
+
+def random_bytes(seed: int, stream: int, shape, first: int = 0) -> np.ndarray:
+    """Uniform random bytes [first, first+n) of stream (seed, stream)."""
+    n = int(np.prod(shape)) if len(shape) else 1
+    out = np.empty(shape, dtype=np.uint8)
+    _L().moe_gen_bytes(seed, stream, first, n, out.ctypes.data)
+    return out
+
+
+def mxfp4_weights(seed: int, code_stream: int, scale_stream: int, E: int, rows: int, cols: int,
+                  fan_in: int) -> tuple:
+    """Synthetic mxfp4 expert weights [E, rows, cols] (blocks of 32 along
+    cols): uniformly random 4-bit element codes, two per byte, and one scale
+    byte per block, drawn from the three exponents around the one that gives
+    weights of RMS about 1/sqrt(fan_in) (uniform codes have an RMS magnitude
+    of about 2.93; scale byte s stands for 2^(s - 127)).  Returns
+    (blocks uint8 [E, rows, cols/32, 16], scales uint8 [E, rows, cols/32])."""
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    nb = cols // 32
+    blocks = random_bytes(seed, code_stream, (E, rows, nb, 16))
+    center = 127 + int(round(math.log2(1.0 / (math.sqrt(fan_in) * 2.926))))
+    scales = (center - 1 + random_bytes(seed, scale_stream, (E, rows, nb)) % 3).astype(np.uint8)
+    return blocks, scales
+
+
+def make_mxfp4_experts(w: "Workload") -> dict:
+    """mxfp4 versions of the routed experts of workload w (gate/up [E, I, H],
+    down [E, H, I]), as (blocks, scales) pairs; H and I multiples of 32."""
+    s = w.seed
+    return {
+        "w_gate": mxfp4_weights(s, STREAM_MX_GATE, STREAM_MXS_GATE, w.E, w.I, w.H, w.H),
+        "w_up": mxfp4_weights(s, STREAM_MX_UP, STREAM_MXS_UP, w.E, w.I, w.H, w.H),
+        "w_down": mxfp4_weights(s, STREAM_MX_DOWN, STREAM_MXS_DOWN, w.E, w.H, w.I, w.I),
+    }
 
 
 def u64(seed: int, stream: int, n: int) -> int:

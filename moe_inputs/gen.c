@@ -99,3 +99,15 @@ void moe_gen_permutation(uint64_t seed, uint64_t stream, int32_t n, int32_t* out
         out[j] = t;
     }
 }
+
+/* out[i] = byte ((first + i) mod 8) of splitmix64 output (first + i) / 8 of
+ * the stream (least significant byte first): uniform random bytes, each a
+ * pure function of (seed, stream, index). */
+void moe_gen_bytes(uint64_t seed, uint64_t stream, uint64_t first, int64_t n, uint8_t* out) {
+    uint64_t key = moe_gen_stream_key(seed, stream);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const uint64_t j = first + (uint64_t)i;
+        out[i] = (uint8_t)(splitmix_at(key, j >> 3) >> (8 * (j & 7)));
+    }
+}

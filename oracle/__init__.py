@@ -11,6 +11,8 @@ scores -> capacity drop in token order -> weighted sum of the selected SwiGLU
 experts (+ the always-on shared expert).  Router statistics for the
 load-balance penalties: per-expert importance (sum over tokens of the softmax
 over all E scores) and the penalties built from it and the top-k counts.
+Expert weights in the MXFP4 microscaling format: dequantization from the
+format's definition and the layer on those weights.
 
 Parity pins of every function here live in ``tests/test_oracle.py``.
 """
@@ -207,3 +209,61 @@ def balance_losses(importance_e, load_e, T: int) -> dict:
     std = float(np.std(imp, ddof=1) + np.std(load, ddof=1))
     switch = float(E * np.sum((load / T) * (imp / T)))
     return dict(kl=kl, std=std, switch=switch)
+
+
+# ------------------------------------------------------------- mxfp4 weights
+# Expert weights in the MXFP4 format of the OCP Microscaling (MX) v1.0
+# specification: blocks of 32 elements along the reduction dimension, each
+# element an FP4 E2M1 number (sign bit, 2 exponent bits with bias 1, 1
+# mantissa bit, subnormal when the exponent field is 0, no inf or NaN) and
+# one E8M0 scale per block (value 2^(s - 127); s = 255 is NaN).  The pages
+# note that native mxfp4 kernels would speed up gpt-oss ("Mixture of Experts
+# (MoEs) in Transformers", section From Dense to Sparse) without giving the
+# format; its storage order is read here as two codes per byte, the element
+# with the lower index in the low nibble.
+
+def e2m1_value(code: int) -> float:
+    """Value of a 4-bit E2M1 code, from its bit fields."""
+    sign = -1.0 if code & 0x8 else 1.0
+    exp = (code >> 1) & 0x3
+    man = code & 0x1
+    if exp == 0:
+        return sign * (man / 2.0)  # subnormal: 2^(1 - bias) * (m / 2), bias 1
+    return sign * 2.0 ** (exp - 1) * (1.0 + man / 2.0)
+
+
+def mxfp4_dequantize(blocks, scales) -> np.ndarray:
+    """float64 weights [..., 32 * nb] from blocks uint8 [..., nb, 16] (two
+    codes per byte) and scales uint8 [..., nb]."""
+    blocks = np.asarray(blocks, np.uint8)
+    scales = np.asarray(scales, np.uint8)
+    table = np.array([e2m1_value(c) for c in range(16)], np.float64)
+    lo = table[blocks & 0x0F]
+    hi = table[blocks >> 4]
+    elems = np.stack([lo, hi], axis=-1).reshape(blocks.shape[:-1] + (32,))  # element 2j low, 2j+1 high
+    scale = np.where(scales == 255, np.nan, np.ldexp(1.0, scales.astype(np.int64) - 127))
+    return (elems * scale[..., None]).reshape(blocks.shape[:-2] + (blocks.shape[-2] * 32,))
+
+
+def moe_tokens_mxfp4(x, mx: dict, topk_idx, topk_w, dtype: str, row_of=None, tokens=None) -> np.ndarray:
+    """moe_tokens with routed experts given as mxfp4 (blocks, scales) pairs
+    under "w_gate", "w_up", "w_down".  The dequantized weights and the
+    activations are exact in float32 (the scales of the inputs used here
+    stay far inside its range), so the fp64 evaluation runs on the exact
+    values."""
+    w = {}
+    for name in ("w_gate", "w_up", "w_down"):
+        d = mxfp4_dequantize(*mx[name])
+        f = d.astype(np.float32)
+        if not np.array_equal(f.astype(np.float64), d):
+            raise ValueError(f"{name}: mxfp4 values outside the float32 range")
+        w[name] = f
+    xs = np.asarray(x)
+    x32 = _bf16_bits_to_f32(xs) if dtype == "bf16" else xs.astype(np.float32)
+    return moe_tokens(x32, w["w_gate"], w["w_up"], w["w_down"], topk_idx, topk_w, "f32", row_of=row_of,
+                      tokens=tokens)
+
+
+def _bf16_bits_to_f32(a) -> np.ndarray:
+    """Exact float32 values of bfloat16 bit patterns (uint16)."""
+    return (np.asarray(a, np.uint16).astype(np.uint32) << 16).view(np.float32)

@@ -54,3 +54,17 @@ def test_sample_tokens():
 def test_workload_capacity():
     assert mi.QWEN3.capacity() == 2560
     assert mi.MIXTRAL.capacity() == 0
+
+
+def test_mxfp4_weights_are_seeded_uniform_codes_with_clustered_scales():
+    b1, s1 = mi.mxfp4_weights(0, mi.STREAM_MX_GATE, mi.STREAM_MXS_GATE, 4, 64, 2880, 2880)
+    b2, s2 = mi.mxfp4_weights(0, mi.STREAM_MX_GATE, mi.STREAM_MXS_GATE, 4, 64, 2880, 2880)
+    assert b1.shape == (4, 64, 90, 16) and s1.shape == (4, 64, 90)
+    assert np.array_equal(b1, b2) and np.array_equal(s1, s2)
+    nib = np.concatenate([(b1 & 0xF).ravel(), (b1 >> 4).ravel()])
+    hist = np.bincount(nib, minlength=16) / nib.size
+    assert np.all(np.abs(hist - 1 / 16) < 0.01)
+    # 2^(s - 127) * RMS(E2M1) ~ 1/sqrt(2880): the center byte is 120
+    assert set(np.unique(s1).tolist()) == {119, 120, 121}
+    # any sub-range regenerates alone
+    assert np.array_equal(mi.random_bytes(0, 11, (100,), first=37), mi.random_bytes(0, 11, (137,))[37:])

@@ -423,3 +423,55 @@ def test_sampled_tokens_equal_full_evaluation():
     tok = mi.sample_tokens(5, wl.T, 9)
     part = oracle.forward(wl, inp, tokens=tok)
     assert np.array_equal(part["y"], full["y"][tok])
+
+
+# ------------------------------------------------------------- mxfp4 weights
+# The FP4 E2M1 value table of the OCP Microscaling v1.0 specification
+# (magnitudes of codes 0..7; codes 8..15 are their negatives).
+E2M1_SPEC = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_codes_match_the_specification_table():
+    spec = E2M1_SPEC + [-v for v in E2M1_SPEC]
+    assert [oracle.e2m1_value(c) for c in range(16)] == spec
+    # all 16 codes through the block path, scale byte 127 = 2^0
+    codes = np.arange(32) % 16
+    blocks = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)[None, :]
+    got = oracle.mxfp4_dequantize(blocks, np.array([127], np.uint8))
+    assert got.tolist() == [spec[c] for c in codes]
+    assert math.copysign(1.0, got[8]) == -1.0  # code 8 is -0
+
+
+def test_mxfp4_scale_bytes_are_powers_of_two():
+    blocks = np.full((255, 1, 16), 0x22, np.uint8)  # every element code 2 = 1.0
+    scales = np.arange(255, dtype=np.uint8)[:, None]
+    got = oracle.mxfp4_dequantize(blocks, scales)
+    for s in range(255):
+        assert np.all(got[s] == math.ldexp(1.0, s - 127)), s
+    nan = oracle.mxfp4_dequantize(blocks[:1], np.array([[255]], np.uint8))
+    assert np.all(np.isnan(nan))
+
+
+def test_mxfp4_nibble_order_and_per_block_scales():
+    """Hand-built row of two blocks: bytes 0x21, 0xF0 in block 0 (scale 2^0)
+    and 0x76 in block 1 (scale 2^1): elements 0.5, 1, 0, -6, ... and 8, 12."""
+    blocks = np.zeros((2, 16), np.uint8)
+    blocks[0, 0], blocks[0, 1], blocks[1, 0] = 0x21, 0xF0, 0x76
+    got = oracle.mxfp4_dequantize(blocks, np.array([127, 128], np.uint8))
+    assert got.shape == (64,)
+    assert got[:4].tolist() == [0.5, 1.0, 0.0, -6.0] and np.all(got[4:32] == 0)
+    assert got[32:34].tolist() == [8.0, 12.0] and np.all(got[34:] == 0)
+
+
+def test_mxfp4_single_expert_is_dense_swiglu_ffn():
+    """E = k = 1 with mxfp4 weights: y = W_d (silu(W_g x) * W_u x) on the
+    dequantized weights, via torch float64."""
+    wl = small(T=12, H=64, I=96, E=1, k=1, dtype="bf16")
+    inp = mi.make_inputs(wl, router_only=True)
+    mx = mi.make_mxfp4_experts(wl)
+    idx = np.zeros((wl.T, 1), np.int32)
+    y = oracle.moe_tokens_mxfp4(inp["x"], mx, idx, np.ones((wl.T, 1)), "bf16")
+    x = torch.from_numpy(f64(inp["x"], "bf16"))
+    g, u, d = (torch.from_numpy(oracle.mxfp4_dequantize(*mx[n])[0]) for n in ("w_gate", "w_up", "w_down"))
+    ref = torch.nn.functional.linear(torch.nn.functional.silu(x @ g.T) * (x @ u.T), d).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-13 * np.abs(ref).max())
