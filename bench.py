@@ -135,6 +135,11 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- roofline
+def layer_flops(wl) -> float:
+    """Algorithmic FLOPs of the expert FFNs, 2*T*k*3*H*I (+ 2*T*3*H*I_s shared)."""
+    return 2.0 * wl.T * wl.k * 3 * wl.H * wl.I + 2.0 * wl.T * 3 * wl.H * wl.I_shared
+
+
 def layer_bytes(wl, active_experts: int) -> float:
     """Algorithmic bytes: weights of the activated experts + x + y + router (+ shared)."""
     elt = 2 if wl.dtype == "bf16" else 4
@@ -452,7 +457,7 @@ def run_ours(args, wl, world, rank, local):
         t_avg = sum(dom_times[dom]) / len(dom_times[dom]) / 1e3
         kept = wl.T * wl.k
         if wl.capacity_factor > 0:
-            kept = int(np.minimum(counts.cpu().numpy(), wl.capacity()).sum())
+            kept = int(np.minimum(counts.cpu().numpy(), moe.capacity(cfg)).sum())
         flops = 2.0 * kept * 2 * wl.H * wl.I + 2.0 * wl.T * 2 * wl.H * wl.I_shared
         achieved = flops / t_avg / 1e12
         # one launch of the kernel lasts milliseconds at most: burst peak
@@ -461,7 +466,7 @@ def run_ours(args, wl, world, rank, local):
                 "frac": achieved / peak, "traffic": traffic_for(dom, wl),
                 "peak_kind": f"{pk_kind} bf16 dense, burst", "launch_ms": t_avg * 1e3,
                 "flops_per_launch": flops, "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
-    F = wl.flops()
+    F = layer_flops(wl)
     B = layer_bytes(wl, active)
     t_roof = max(F / (pk["bf16_tflops"] * 1e12), B / (pk["hbm_gbs"] * 1e9))
     t_roof_sus = max(F / (pk["bf16_tflops_sustained"] * 1e12), B / (pk["hbm_gbs"] * 1e9))

@@ -264,6 +264,56 @@ moe_status_t moe_forward_routed(const moe_config_t* cfg, const void* x, const in
                                 const void* ws_down, void* y, int32_t* counts_out, int32_t* dropped_out,
                                 void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * moe_shard_capacity_left -- per-expert capacity left for one token shard of
+ * a capacity-limited batch ("MoE稀疏架构是什么？…", section 三.2: an expert
+ * takes tokens up to its capacity and drops the rest; capacity is served in
+ * global token order, so a shard gets what the earlier shards left of it).
+ *   cfg describes the WHOLE batch: cfg->T is the tokens of all shards
+ *   together, so C = moe_capacity(cfg), which must be > 0.
+ *   counts_per_shard [n_shards, E] int32, device: every shard's per-expert
+ *   counts before the capacity cut (moe_permute counts, or moe_forward_routed
+ *   counts_out with capacity_left NULL), gathered from all shards, shards in
+ *   token order.
+ *   -> capacity_left [E] int32, device:
+ *      capacity_left[e] = max(0, C - sum over shards q < shard of counts_q[e]),
+ *   the argument moe_forward_routed takes for that shard.  One small kernel
+ *   on `stream`; the counts never leave the device.
+ * Errors: no capacity (cfg->capacity_factor <= 0), n_shards < 1 or shard
+ * outside [0, n_shards) -> MOE_ERR_INVALID_ARG, before anything is enqueued.
+ */
+moe_status_t moe_shard_capacity_left(const moe_config_t* cfg, const int32_t* counts_per_shard, int32_t n_shards,
+                                     int32_t shard, int32_t* capacity_left, moe_stream_t stream);
+
+/* moe_shard_capacity_left on HOST arrays (counts gathered on the host, e.g.
+ * by a CPU process group): same arguments and result, computed on the
+ * calling thread, no CUDA call. */
+moe_status_t moe_shard_capacity_left_host(const moe_config_t* cfg, const int32_t* counts_per_shard,
+                                          int32_t n_shards, int32_t shard, int32_t* capacity_left);
+
+/*
+ * moe_balance_losses -- the load-balance penalties from the two per-expert
+ * router statistics, on HOST arrays (2*E numbers; no CUDA call), in fp64:
+ *   q_e = importance[e] / T (mean gate probability),
+ *   out[0] kl     = (1/E) sum_e (1/E) (log(1/E) - log(q_e + 1e-8)):
+ *                   KL from uniform to the mean gate probability, the batch
+ *                   mean over the E-vector ("模型的“分工的艺术”：MoE技术如何
+ *                   提升计算效率", section 3.1);
+ *   out[1] std    = std(importance) + std(load), unbiased (divisor E - 1)
+ *                   ("2026年人工智能MoE混合专家模型入门指南", the MoE layer's
+ *                   load-balance loss; the page's load, a count of positive
+ *                   dense-softmax probabilities, is T for every expert, so
+ *                   the top-k counts stand in for it);
+ *   out[2] switch = E * sum_e (load[e] / T) * q_e, the Switch-Transformer
+ *                   form (fraction of tokens routed to e times its mean gate
+ *                   probability).
+ *   importance [E] float32 (from moe_route_importance), load [E] int32 (the
+ *   top-k counts from moe_permute or moe_forward), T the tokens they cover.
+ * Errors: E < 2, T <= 0 or a NULL pointer -> MOE_ERR_INVALID_ARG.
+ */
+moe_status_t moe_balance_losses(int32_t E, int64_t T, const float* importance, const int32_t* load,
+                                double* out);
+
 /* Waits for `stream`, then returns the device check flags (MOE_DEVFLAG_*)
  * accumulated in `ws` since the last call and clears them.  Returns
  * MOE_ERR_DEVICE_CHECK if any flag was set, MOE_OK otherwise. */

@@ -171,16 +171,6 @@ class Workload:
     def has_bias(self) -> bool:
         return self.zipf_s > 0
 
-    def capacity(self) -> int:
-        """Per-expert capacity C = ceil(cf * T * k / E); 0 means unlimited."""
-        if self.capacity_factor <= 0:
-            return 0
-        return int(math.ceil(self.capacity_factor * self.T * self.k / self.E))
-
-    def flops(self) -> float:
-        """Algorithmic FLOPs of the expert FFNs, 2*T*k*3*H*I (+ shared)."""
-        return 2.0 * self.T * self.k * 3 * self.H * self.I + 2.0 * self.T * 3 * self.H * self.I_shared
-
 
 # The five workload families (full sizes).
 TINY = Workload("tiny_f32", T=64, H=128, I=256, E=8, k=2, dtype="f32",

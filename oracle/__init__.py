@@ -130,8 +130,28 @@ def moe_tokens(x, w_gate, w_up, w_down, topk_idx, topk_w, dtype: str, row_of=Non
     return y
 
 
+def capacity(cf: float, T: int, k: int, E: int) -> int:
+    """Per-expert capacity C = ceil(cf * T * k / E), 0 meaning unlimited (cf <= 0).
+
+    The pages name the capacity factor without a formula ("MoE稀疏架构是什么？
+    从原理到落地的系统解读", section 三.2; "模型的“分工的艺术”：MoE技术如何提升
+    计算效率", section 3.1); the reading taken is the expected share of an
+    expert, T * k / E slots, scaled by cf and rounded up.  cf is read as the
+    decimal it is written as (the shortest decimal that round-trips the
+    Python float, e.g. 1.25 or 0.8) and the product is formed exactly, so no
+    binary rounding of cf can lift an exact integer to the next one."""
+    from fractions import Fraction
+
+    if cf <= 0:
+        return 0
+    v = Fraction(repr(float(cf))) * int(T) * int(k) / int(E)
+    return int(-((-v.numerator) // v.denominator))  # ceiling of a rational
+
+
 def topk_margin(logits: np.ndarray, k: int) -> np.ndarray:
-    """Gap between the k-th and (k+1)-th largest logit of each token (inf if k == E)."""
+    """Gap between the k-th and (k+1)-th largest logit of each token (inf if k == E):
+    how far the selection of "MoE稀疏架构是什么？…", section 四 (the k best
+    scores) is from changing.  0 for an exact tie across the boundary."""
     T, E = logits.shape
     if k >= E:
         return np.full(T, np.inf)
@@ -146,7 +166,7 @@ def forward(wl, inp: dict, tokens=None) -> dict:
     for ``tokens`` (all tokens if None).
     """
     logits, idx, w = route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
-    perm = permute(idx, wl.E, wl.capacity())
+    perm = permute(idx, wl.E, capacity(wl.capacity_factor, wl.T, wl.k, wl.E))
     y = moe_tokens(inp["x"], inp["w_gate"], inp["w_up"], inp["w_down"], idx, w, wl.dtype,
                    row_of=perm["row_of"], ws_gate=inp["ws_gate"], ws_up=inp["ws_up"],
                    ws_down=inp["ws_down"], tokens=tokens)
@@ -154,8 +174,9 @@ def forward(wl, inp: dict, tokens=None) -> dict:
 
 
 def weights_for(logits: np.ndarray, sel: np.ndarray) -> np.ndarray:
-    """Softmax over the given selection's scores (fp64), the gating step of the
-    method for a selection made elsewhere (a near-tie resolved differently)."""
+    """Softmax over the given selection's scores (fp64), the gating step of
+    "MoE稀疏架构是什么？…", section 四 (softmax over the k chosen scores) for
+    a selection made elsewhere (a near-tie resolved differently)."""
     l = np.take_along_axis(np.asarray(logits, np.float64), np.asarray(sel, np.int64), 1)
     e = np.exp(l - l.max(1, keepdims=True))
     return e / e.sum(1, keepdims=True)
@@ -255,7 +276,9 @@ def moe_tokens_mxfp4(x, mx: dict, topk_idx, topk_w, dtype: str, row_of=None, tok
     for name in ("w_gate", "w_up", "w_down"):
         d = mxfp4_dequantize(*mx[name])
         f = d.astype(np.float32)
-        if not np.array_equal(f.astype(np.float64), d):
+        # a scale byte of 255 is NaN (the specification's E8M0 NaN): it
+        # propagates to every output that reads the block, as in fp64
+        if not np.array_equal(f.astype(np.float64), d, equal_nan=True):
             raise ValueError(f"{name}: mxfp4 values outside the float32 range")
         w[name] = f
     xs = np.asarray(x)

@@ -54,6 +54,12 @@ _SIGS = {
     "moe_combine": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_forward": ([ctypes.POINTER(moe_config_t)] + [_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_forward_routed": ([ctypes.POINTER(moe_config_t)] + [_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_shard_capacity_left": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_int32, ctypes.c_int32, _P, _P],
+                                ctypes.c_int),
+    "moe_shard_capacity_left_host": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_int32, ctypes.c_int32, _P],
+                                     ctypes.c_int),
+    "moe_balance_losses": ([ctypes.c_int32, ctypes.c_int64, _P, _P, ctypes.POINTER(ctypes.c_double)],
+                           ctypes.c_int),
     "moe_get_device_status": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_size_t, _P,
                                ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
     "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -110,6 +116,13 @@ def capacity(cfg: moe_config_t) -> int:
     return load().moe_capacity(ctypes.byref(cfg))
 
 
+def _host(a):
+    """A host numpy view of a tensor or array (device tensors are copied)."""
+    if hasattr(a, "is_cuda"):
+        return a.detach().cpu().numpy()
+    return a
+
+
 def _ptr(t):
     if t is None:
         return None
@@ -155,31 +168,23 @@ def moe_route_importance(cfg, x, router_w, router_b, topk_idx, topk_w, importanc
                                        _ptr(topk_idx), _ptr(topk_w), _ptr(importance), *_ws(ws), _stream(stream)))
 
 
-def balance_losses(importance, load, T: int) -> dict:
-    """Load-balance penalties from the per-expert statistics (host arithmetic
-    on E numbers; importance from moe_route_importance, load = the top-k
-    counts from moe_permute or moe_forward):
-      kl     = (1/E) sum_e (1/E) (log(1/E) - log(importance_e / T + 1e-8)),
-               KL from uniform to the mean gate probability
-               ("模型的“分工的艺术”…", section 3.1);
-      std    = std(importance) + std(load), unbiased
-               ("2026年人工智能MoE混合专家模型入门指南", MoE layer; the page's
-               load, a count of positive softmax probabilities, is T for every
-               expert, so the top-k counts stand in for it);
-      switch = E sum_e (load_e / T)(importance_e / T), the Switch-Transformer
-               form."""
+def moe_balance_losses(importance, counts, T: int) -> dict:
+    """The library's load-balance penalties (kl, std, switch; fp64) from the
+    per-expert importance (moe_route_importance) and load (the top-k counts
+    from moe_permute or moe_forward) covering T tokens.  Tensors on a device
+    are copied to the host first (the C function reads host arrays)."""
     import numpy as np
-    imp = np.asarray(importance, dtype=np.float64).ravel()
-    ld = np.asarray(load, dtype=np.float64).ravel()
-    E = imp.size
-    if E < 2 or ld.size != E or T <= 0:
-        raise ValueError("need E >= 2 experts, matching lengths and T > 0")
-    mean_prob = imp / T
-    kl = float(np.sum((np.log(1.0 / E) - np.log(mean_prob + 1e-8)) / E) / E)
-    dev_i, dev_l = imp - imp.mean(), ld - ld.mean()
-    std = float(np.sqrt(np.dot(dev_i, dev_i) / (E - 1)) + np.sqrt(np.dot(dev_l, dev_l) / (E - 1)))
-    switch = float(E * np.dot(ld / T, mean_prob))
-    return dict(kl=kl, std=std, switch=switch)
+
+    imp = np.ascontiguousarray(_host(importance), dtype=np.float32).ravel()
+    ld = np.ascontiguousarray(_host(counts), dtype=np.int32).ravel()
+    if ld.size != imp.size:
+        raise MoeError(1, f"importance has {imp.size} experts, load {ld.size}")
+    out = (ctypes.c_double * 3)()
+    _check(load().moe_balance_losses(imp.size, int(T), imp.ctypes.data, ld.ctypes.data, out))
+    return dict(kl=out[0], std=out[1], switch=out[2])
+
+
+balance_losses = moe_balance_losses
 
 
 def moe_permute(cfg, topk_idx, counts, offsets, perm_rows, row_of, dropped, ws, stream=None):
@@ -229,18 +234,27 @@ def moe_forward_routed(cfg, x, topk_idx, topk_w, capacity_left, w_gate, w_up, w_
                                      _stream(stream)))
 
 
-def shard_capacity_left(counts_per_shard, capacity: int, shard: int):
-    """Capacity left for each expert in token shard `shard` of a batch whose
-    capacity is `capacity` (served in global token order): capacity minus the
-    rows the earlier shards kept, i.e. max(0, C - sum_{q < shard} counts_q[e]).
+def moe_shard_capacity_left(cfg, counts_per_shard, shard: int, capacity_left, stream=None):
+    """capacity_left [E] int32 for token shard `shard` of the batch cfg
+    describes (cfg.T = tokens of all shards), from every shard's counts
+    counts_per_shard [n_shards, E] int32, both on the device."""
+    n = counts_per_shard.shape[0]
+    _check(load().moe_shard_capacity_left(ctypes.byref(cfg), _ptr(counts_per_shard), n, shard, _ptr(capacity_left),
+                                          _stream(stream)))
 
-    counts_per_shard: [n_shards, E] integer array (every shard's counts before
-    the capacity cut, gathered from all shards); returns an int32 array [E]."""
+
+def moe_shard_capacity_left_host(cfg, counts_per_shard, shard: int):
+    """moe_shard_capacity_left on host arrays (counts gathered on the host);
+    returns an int32 numpy array [E]."""
     import numpy as np
 
-    c = np.asarray(counts_per_shard, dtype=np.int64)
-    before = c[:shard].sum(axis=0) if shard > 0 else np.zeros(c.shape[1], np.int64)
-    return np.maximum(0, int(capacity) - before).astype(np.int32)
+    c = np.ascontiguousarray(counts_per_shard, dtype=np.int32)
+    if c.ndim != 2 or c.shape[1] != cfg.E:
+        raise MoeError(1, f"counts_per_shard must be [n_shards, {cfg.E}]")
+    out = np.empty(cfg.E, np.int32)
+    _check(load().moe_shard_capacity_left_host(ctypes.byref(cfg), c.ctypes.data, c.shape[0], shard,
+                                               out.ctypes.data))
+    return out
 
 
 def moe_get_device_status(cfg, ws, stream=None) -> int:

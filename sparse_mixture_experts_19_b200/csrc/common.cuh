@@ -130,6 +130,13 @@ cudaError_t launch_combine_rows(const Plan& p, const void* rows, const int32_t* 
 cudaError_t launch_combine(const Plan& p, const float* expert_out, const int32_t* row_of,
                            const float* topk_w, void* y, cudaStream_t st);
 
+// capacity_left[e] = max(0, C - sum_{q < shard} counts[q][e]) for one token
+// shard of a batch with capacity C (device kernel / host loop).
+cudaError_t launch_shard_capacity_left(int64_t C, const int32_t* counts, int n_shards, int shard, int E,
+                                       int32_t* capacity_left, cudaStream_t st);
+void shard_capacity_left_host(int64_t C, const int32_t* counts, int n_shards, int shard, int E,
+                              int32_t* capacity_left);
+
 // Kernel-trace hooks (moe_abi.cu): bracket one launch with events.
 void trace_before(const char* name, cudaStream_t st);
 void trace_after(cudaStream_t st);

@@ -442,6 +442,70 @@ moe_status_t moe_forward_routed(const moe_config_t* cfg, const void* x, const in
                                  st);
 }
 
+static moe_status_t check_shard_args(const moe_config_t* cfg, const int32_t* counts, int32_t n_shards,
+                                     int32_t shard, const int32_t* out, int64_t* C) {
+    moe_status_t s = check_config(cfg);
+    if (s != MOE_OK) return s;
+    *C = capacity_of(cfg);
+    if (*C <= 0) return fail(MOE_ERR_INVALID_ARG, "the batch has no capacity limit (capacity_factor <= 0)");
+    if (n_shards < 1) return fail(MOE_ERR_INVALID_ARG, "n_shards = %d < 1", n_shards);
+    if (shard < 0 || shard >= n_shards)
+        return fail(MOE_ERR_INVALID_ARG, "shard = %d outside [0, %d)", shard, n_shards);
+    if (!counts) return fail(MOE_ERR_INVALID_ARG, "counts_per_shard is NULL");
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "capacity_left is NULL");
+    return MOE_OK;
+}
+
+moe_status_t moe_shard_capacity_left(const moe_config_t* cfg, const int32_t* counts_per_shard, int32_t n_shards,
+                                     int32_t shard, int32_t* capacity_left, moe_stream_t stream) {
+    int64_t C = 0;
+    moe_status_t s = check_shard_args(cfg, counts_per_shard, n_shards, shard, capacity_left, &C);
+    if (s != MOE_OK) return s;
+    CUDA_TRY(launch_shard_capacity_left(C, counts_per_shard, n_shards, shard, cfg->E, capacity_left,
+                                        (cudaStream_t)stream),
+             "shard_capacity_left");
+    return MOE_OK;
+}
+
+moe_status_t moe_shard_capacity_left_host(const moe_config_t* cfg, const int32_t* counts_per_shard,
+                                          int32_t n_shards, int32_t shard, int32_t* capacity_left) {
+    int64_t C = 0;
+    moe_status_t s = check_shard_args(cfg, counts_per_shard, n_shards, shard, capacity_left, &C);
+    if (s != MOE_OK) return s;
+    shard_capacity_left_host(C, counts_per_shard, n_shards, shard, cfg->E, capacity_left);
+    return MOE_OK;
+}
+
+// Load-balance penalties in fp64 from importance [E] and load [E] (host
+// arrays): KL from uniform to the mean gate probability, std(importance) +
+// std(load) (unbiased), and E * sum f_e P_e.  Sums run in expert order.
+moe_status_t moe_balance_losses(int32_t E, int64_t T, const float* importance, const int32_t* load,
+                                double* out) {
+    if (E < 2) return fail(MOE_ERR_INVALID_ARG, "E = %d: the penalties need at least 2 experts", E);
+    if (T <= 0) return fail(MOE_ERR_INVALID_ARG, "T = %lld must be positive", (long long)T);
+    if (!importance || !load || !out) return fail(MOE_ERR_INVALID_ARG, "importance, load and out are required");
+    const double inv_e = 1.0 / E, tt = (double)T;
+    double kl = 0.0, sum_i = 0.0, sum_l = 0.0, sw = 0.0;
+    for (int e = 0; e < E; ++e) {
+        const double q = (double)importance[e] / tt;
+        kl += inv_e * (log(inv_e) - log(q + 1e-8));
+        sum_i += importance[e];
+        sum_l += load[e];
+        sw += ((double)load[e] / tt) * q;
+    }
+    const double mi = sum_i / E, ml = sum_l / E;
+    double vi = 0.0, vl = 0.0;
+    for (int e = 0; e < E; ++e) {
+        const double di = importance[e] - mi, dl = load[e] - ml;
+        vi += di * di;
+        vl += dl * dl;
+    }
+    out[0] = kl / E;
+    out[1] = sqrt(vi / (E - 1)) + sqrt(vl / (E - 1));
+    out[2] = E * sw;
+    return MOE_OK;
+}
+
 moe_status_t moe_get_device_status(const moe_config_t* cfg, void* ws, size_t ws_bytes,
                                    moe_stream_t stream, int32_t* flags_out) {
     Plan p;

@@ -22,6 +22,11 @@ ORDER_MARGIN = 1e-3
 TOL = {"bf16": 2e-2, "f32": 1e-4}
 
 
+def cap_of(wl) -> int:
+    """The oracle's per-expert capacity of workload wl (0 = unlimited)."""
+    return oracle.capacity(wl.capacity_factor, wl.T, wl.k, wl.E)
+
+
 def dev(a, dtype):
     if a is None:
         return None
@@ -75,7 +80,7 @@ def oracle_given_selection(wl, inp, logits, sel, tokens):
     """The oracle's layer output for `tokens`, with the routing selection `sel`
     (all T tokens) taken as given: weights, grouping and FFN from the oracle."""
     w = oracle.weights_for(logits, sel)
-    perm = oracle.permute(sel, wl.E, wl.capacity())
+    perm = oracle.permute(sel, wl.E, cap_of(wl))
     y = oracle.moe_tokens(inp["x"], inp["w_gate"], inp["w_up"], inp["w_down"], sel, w, wl.dtype,
                           row_of=perm["row_of"], ws_gate=inp["ws_gate"], ws_up=inp["ws_up"],
                           ws_down=inp["ws_down"], tokens=tokens)

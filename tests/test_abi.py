@@ -146,18 +146,33 @@ def test_route_importance_validates(lib):
     assert lib.moe_route_importance(ctypes.byref(c0), None, None, None, None, None, FAKE, FAKE, need, None) == 0
 
 
-def test_balance_losses_host_helper_matches_oracle():
+def test_balance_losses_call_matches_oracle():
+    """moe_balance_losses (host C, fp64) against the oracle's penalties on the
+    same float32 importance."""
     import oracle
     rng = np.random.default_rng(11)
     for E, T in ((2, 10), (8, 1000), (256, 16384)):
-        imp = rng.dirichlet(np.ones(E)) * T
-        load = rng.integers(0, 8 * T // E + 1, E)
-        got = moe.balance_losses(imp, load, T)
-        ref = oracle.balance_losses(imp, load, T)
+        imp = (rng.dirichlet(np.ones(E)) * T).astype(np.float32)
+        load = rng.integers(0, 8 * T // E + 1, E).astype(np.int32)
+        got = moe.moe_balance_losses(imp, load, T)
+        ref = oracle.balance_losses(imp.astype(np.float64), load, T)
         for key in ("kl", "std", "switch"):
             assert abs(got[key] - ref[key]) <= 1e-12 * max(1.0, abs(ref[key])), (E, key)
-    with pytest.raises(ValueError):
-        moe.balance_losses(np.ones(1), np.ones(1), 4)
+    with pytest.raises(moe.MoeError):
+        moe.moe_balance_losses(np.ones(1), np.ones(1), 4)
+    with pytest.raises(moe.MoeError):
+        moe.moe_balance_losses(np.ones(4), np.ones(4), 0)
+    with pytest.raises(moe.MoeError):
+        moe.moe_balance_losses(np.ones(4), np.ones(3), 4)
+
+
+def test_shard_capacity_left_validates(lib):
+    c = cfg(capacity_factor=1.0)
+    assert lib.moe_shard_capacity_left(ctypes.byref(c), FAKE, 2, 2, FAKE, None) == 1
+    assert lib.moe_shard_capacity_left(ctypes.byref(c), FAKE, 0, 0, FAKE, None) == 1
+    assert lib.moe_shard_capacity_left(ctypes.byref(c), None, 2, 1, FAKE, None) == 1
+    assert lib.moe_shard_capacity_left(ctypes.byref(cfg()), FAKE, 2, 1, FAKE, None) == 1
+    assert "capacity" in moe.moe_last_error()
 
 
 def call_forward_routed(lib, c, ws, ws_bytes, **ptrs):

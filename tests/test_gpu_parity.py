@@ -12,7 +12,7 @@ import torch
 
 import moe_inputs as mi
 import oracle
-from parity_util import (TOL, check_selection, host_f64, oracle_given_selection, rowwise_rel_err,
+from parity_util import (TOL, cap_of, check_selection, host_f64, oracle_given_selection, rowwise_rel_err,
                          to_device)
 
 pytestmark = pytest.mark.gpu
@@ -205,7 +205,7 @@ def test_stages_route_permute_ffn_combine(gpu_lib, wl):
     perm_rows = torch.empty(T * k, dtype=torch.int32, device="cuda")
     row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
     moe.moe_permute(cfg, idx, counts, offsets, perm_rows, row_of, dropped, ws)
-    ref = oracle.permute(idx_g, E, wl.capacity())
+    ref = oracle.permute(idx_g, E, cap_of(wl))
     for name, t in (("counts", counts), ("dropped", dropped), ("offsets", offsets),
                     ("perm_rows", perm_rows)):
         assert np.array_equal(t.cpu().numpy(), ref[name]), name
@@ -278,7 +278,7 @@ def test_permute_is_bit_reproducible(gpu_lib):
     for r in res[1:]:
         for a, b in zip(res[0], r):
             assert np.array_equal(a, b)
-    ref = oracle.permute(idx.cpu().numpy(), wl.E, wl.capacity())
+    ref = oracle.permute(idx.cpu().numpy(), wl.E, cap_of(wl))
     assert np.array_equal(res[0][2], ref["perm_rows"])
 
 

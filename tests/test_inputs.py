@@ -51,11 +51,6 @@ def test_sample_tokens():
     assert np.array_equal(mi.sample_tokens(0, 10, 64), np.arange(10))
 
 
-def test_workload_capacity():
-    assert mi.QWEN3.capacity() == 2560
-    assert mi.MIXTRAL.capacity() == 0
-
-
 def test_mxfp4_weights_are_seeded_uniform_codes_with_clustered_scales():
     b1, s1 = mi.mxfp4_weights(0, mi.STREAM_MX_GATE, mi.STREAM_MXS_GATE, 4, 64, 2880, 2880)
     b2, s2 = mi.mxfp4_weights(0, mi.STREAM_MX_GATE, mi.STREAM_MXS_GATE, 4, 64, 2880, 2880)

@@ -80,7 +80,7 @@ def _ep_worker(rank, world, port, out):
     wl = mi.Workload("ep", T=40, H=48, I=32, E=8, k=2, I_shared=16, capacity_factor=0.75, dtype="bf16")
     inp = mi.make_inputs(wl)
     _, idx, w = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
-    row_of = oracle.permute(idx, wl.E, wl.capacity())["row_of"].copy()  # global capacity, token order
+    row_of = oracle.permute(idx, wl.E, oracle.capacity(wl.capacity_factor, wl.T, wl.k, wl.E))["row_of"].copy()  # global capacity, token order
     e0, e1 = rank * wl.E // world, (rank + 1) * wl.E // world
     row_of[(idx < e0) | (idx >= e1)] = -1  # other ranks' experts
     shared = rank == 0

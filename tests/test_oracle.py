@@ -137,6 +137,67 @@ def test_weights_sum_to_one_and_follow_scores(E, k):
     assert np.all(pk.min(1) >= np.sort(p, 1)[:, -k] - 1e-15)
 
 
+def test_topk_margin_golden():
+    g = json.load(open(os.path.join(GOLDEN, "topk_margin.json")))
+    for case in g["cases"]:
+        m = oracle.topk_margin(np.array([case["logits"]], np.float64), case["k"])
+        want = np.inf if case["margin"] is None else case["margin"]
+        assert m.tolist() == [want], case
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (32, 4), (256, 8), (7, 3)])
+def test_topk_margin_is_the_smallest_gap_across_the_selection(E, k):
+    """Brute force: the margin equals min over selected e and unselected e' of
+    l_e - l_e', with the selection taken from the C oracle's routing."""
+    wl = small(T=80, H=24, E=E, k=k, dtype="bf16", zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    logits, idx, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], k, "bf16")
+    m = oracle.topk_margin(logits, k)
+    for t in range(wl.T):
+        sel = set(idx[t].tolist())
+        gaps = [logits[t, a] - logits[t, b] for a in sel for b in range(E) if b not in sel]
+        assert m[t] == min(gaps), t
+    # a zero-input token with a repeated bias: an exact tie across the boundary
+    x0 = np.zeros((1, 8), np.float32)
+    b = np.array([2.0, 1.0, 1.0, 0.0], np.float32)
+    l0, _, _ = oracle.route(x0, mi.normal(0, 99, (4, 8), 1.0, "f32"), b, 2, "f32")
+    assert oracle.topk_margin(l0, 2).tolist() == [0.0]
+    assert oracle.topk_margin(l0, 4).tolist() == [np.inf]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_weights_for_equals_route_weights_and_transformers_router(dtype):
+    """weights_for on the oracle's own selection reproduces the C oracle's
+    weights and transformers' GptOssTopKRouter weights (fp64), in any order of
+    the selection; k = 1 gives exactly 1."""
+    from transformers import GptOssConfig
+    from transformers.models.gpt_oss.modeling_gpt_oss import GptOssTopKRouter
+
+    wl = small(T=60, H=40, E=16, k=4, dtype=dtype, zipf_s=1.1)
+    inp = mi.make_inputs(wl)
+    logits, idx, w = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, dtype)
+    got = oracle.weights_for(logits, idx)
+    np.testing.assert_allclose(got, w, rtol=0, atol=1e-14)
+    cfg = GptOssConfig(hidden_size=wl.H, num_local_experts=wl.E, num_experts_per_tok=wl.k)
+    r = GptOssTopKRouter(cfg).double()
+    with torch.no_grad():
+        r.weight.copy_(torch.from_numpy(f64(inp["router_w"], dtype)))
+        r.bias.copy_(torch.from_numpy(inp["router_b"].astype(np.float64)))
+        _, w_ref, idx_ref = r(torch.from_numpy(f64(inp["x"], dtype)))
+    np.testing.assert_allclose(oracle.weights_for(logits, idx_ref.numpy()), w_ref.numpy(), rtol=0, atol=1e-14)
+    rev = idx[:, ::-1]
+    np.testing.assert_allclose(oracle.weights_for(logits, rev), got[:, ::-1], rtol=0, atol=1e-15)
+    assert np.all(oracle.weights_for(logits, idx[:, :1]) == 1.0)
+
+
+def test_capacity_golden():
+    g = json.load(open(os.path.join(GOLDEN, "capacity_formula.json")))
+    for c in g["cases"]:
+        assert oracle.capacity(c["cf"], c["T"], c["k"], c["E"]) == c["C"], c
+    assert oracle.capacity(mi.QWEN3.capacity_factor, mi.QWEN3.T, mi.QWEN3.k, mi.QWEN3.E) == 2560
+    assert oracle.capacity(mi.MIXTRAL.capacity_factor, mi.MIXTRAL.T, mi.MIXTRAL.k, mi.MIXTRAL.E) == 0
+
+
 # ------------------------------------------------- load-balance statistics
 
 def test_importance_with_top_k_equal_E_is_the_sum_of_routing_weights():
@@ -249,7 +310,7 @@ def test_permute_invariants(cf):
     wl = small(T=3000, H=16, E=128, k=8, dtype="f32", zipf_s=1.1, capacity_factor=cf)
     inp = mi.make_inputs(wl)
     _, idx, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, "f32")
-    C = wl.capacity()
+    C = oracle.capacity(wl.capacity_factor, wl.T, wl.k, wl.E)
     r = oracle.permute(idx, wl.E, C)
     counts, dropped, off = r["counts"], r["dropped"], r["offsets"]
     assert counts.sum() == wl.T * wl.k
@@ -450,6 +511,26 @@ def test_mxfp4_scale_bytes_are_powers_of_two():
         assert np.all(got[s] == math.ldexp(1.0, s - 127)), s
     nan = oracle.mxfp4_dequantize(blocks[:1], np.array([[255]], np.uint8))
     assert np.all(np.isnan(nan))
+
+
+def test_mxfp4_nan_scale_propagates_to_the_tokens_that_read_it():
+    """A scale byte of 255 (the specification's NaN) in one block of one
+    expert's gate row: every token routed to that expert gets NaN outputs,
+    the other tokens are unchanged."""
+    wl = small(T=10, H=64, I=32, E=3, k=1, dtype="bf16")
+    inp = mi.make_inputs(wl, router_only=True)
+    mx = mi.make_mxfp4_experts(wl)
+    idx = (np.arange(wl.T) % wl.E).astype(np.int32)[:, None]
+    w = np.ones((wl.T, 1))
+    y0 = oracle.moe_tokens_mxfp4(inp["x"], mx, idx, w, "bf16")
+    blocks, scales = mx["w_gate"]
+    scales = scales.copy()
+    scales[1, 5, 1] = 255  # expert 1, gate row 5, second block
+    mx2 = dict(mx, w_gate=(blocks, scales))
+    y1 = oracle.moe_tokens_mxfp4(inp["x"], mx2, idx, w, "bf16")
+    hit = idx[:, 0] == 1
+    assert np.all(np.isnan(y1[hit]))
+    assert np.array_equal(y1[~hit], y0[~hit])
 
 
 def test_mxfp4_nibble_order_and_per_block_scales():

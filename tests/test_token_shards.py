@@ -24,6 +24,10 @@ import moe_inputs as mi
 import oracle
 import sparse_mixture_experts_19_b200 as moe_pkg
 
+
+def cap_of(wl) -> int:
+    return oracle.capacity(wl.capacity_factor, wl.T, wl.k, wl.E)
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 WL = mi.Workload("shards_cap", T=1200, H=256, I=192, E=8, k=2, capacity_factor=0.8)
@@ -58,7 +62,8 @@ def _shard_worker(rank, world, port, out):
     gathered = [torch.zeros_like(counts) for _ in range(world)]
     dist.all_gather(gathered, counts)  # the exchange step
     per_shard = torch.stack(gathered).numpy()
-    cap_left = moe_pkg.shard_capacity_left(per_shard, WL.capacity(), rank)
+    batch = moe_pkg.config(WL.T, WL.H, WL.I, WL.E, WL.k, 0, WL.capacity_factor, WL.dtype)
+    cap_left = moe_pkg.moe_shard_capacity_left_host(batch, per_shard, rank)  # the library's C call
     out[rank] = kept_in_shard(mine, cap_left)
     dist.barrier()
     dist.destroy_process_group()
@@ -73,16 +78,25 @@ def test_shard_capacity_exchange_matches_global_order_two_ranks():
         kept = np.concatenate([out[r] for r in range(world)])
     inp = mi.make_inputs(WL, router_only=True)
     _, idx, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], WL.k, WL.dtype)
-    ref = oracle.permute(idx, WL.E, WL.capacity())
-    assert WL.capacity() > 0 and int(ref["dropped"].sum()) > 0
+    ref = oracle.permute(idx, WL.E, cap_of(WL))
+    assert cap_of(WL) > 0 and int(ref["dropped"].sum()) > 0
     assert np.array_equal(kept, ref["row_of"].ravel() >= 0)
 
 
-def test_shard_capacity_left_helper():
+def test_shard_capacity_left_host_call():
+    """The C call on host counts, against values worked out by hand: a batch
+    of 18 tokens, 3 experts, top-1, cf 1.0 has C = 6."""
+    batch = moe_pkg.config(18, 64, 64, 3, 1, 0, 1.0, "bf16")
+    assert moe_pkg.capacity(batch) == 6
     counts = np.array([[5, 0, 3], [4, 2, 1], [1, 1, 9]])
-    assert moe_pkg.shard_capacity_left(counts, 6, 0).tolist() == [6, 6, 6]
-    assert moe_pkg.shard_capacity_left(counts, 6, 1).tolist() == [1, 6, 3]
-    assert moe_pkg.shard_capacity_left(counts, 6, 2).tolist() == [0, 4, 2]
+    assert moe_pkg.moe_shard_capacity_left_host(batch, counts, 0).tolist() == [6, 6, 6]
+    assert moe_pkg.moe_shard_capacity_left_host(batch, counts, 1).tolist() == [1, 6, 3]
+    assert moe_pkg.moe_shard_capacity_left_host(batch, counts, 2).tolist() == [0, 4, 2]
+    for bad in (-1, 3):
+        with pytest.raises(moe_pkg.MoeError):
+            moe_pkg.moe_shard_capacity_left_host(batch, counts, bad)
+    with pytest.raises(moe_pkg.MoeError):  # no capacity factor: nothing to split
+        moe_pkg.moe_shard_capacity_left_host(moe_pkg.config(18, 64, 64, 3, 1), counts, 0)
 
 
 # ------------------------------------------------------------------ GPU
@@ -113,12 +127,15 @@ def test_shards_reproduce_the_single_call(gpu_lib):
     bounds = [0, 400, 800, wl.T]
     idx_h = idx.cpu().numpy()
     per_shard = np.stack([np.bincount(idx_h[a:b].ravel(), minlength=wl.E) for a, b in zip(bounds, bounds[1:])])
+    per_shard_dev = torch.from_numpy(per_shard.astype(np.int32)).cuda()
     ys, dropped = [], np.zeros(wl.E, np.int64)
     for q, (a, b) in enumerate(zip(bounds, bounds[1:])):
         cfg_q = moe.config(b - a, wl.H, wl.I, wl.E, wl.k, 0, wl.capacity_factor, wl.dtype)
         ws_q = moe.workspace(cfg_q)
         ws_q.fill_(0)
-        cap_left = torch.from_numpy(moe_pkg.shard_capacity_left(per_shard, wl.capacity(), q)).cuda()
+        cap_left = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+        moe.moe_shard_capacity_left(cfg, per_shard_dev, q, cap_left)  # cfg: the whole batch
+        assert cap_left.cpu().numpy().tolist() == moe.moe_shard_capacity_left_host(cfg, per_shard, q).tolist()
         y_q = torch.empty((b - a, wl.H), dtype=d["x"].dtype, device="cuda")
         counts_q = torch.empty(wl.E, dtype=torch.int32, device="cuda")
         dropped_q = torch.empty(wl.E, dtype=torch.int32, device="cuda")
@@ -154,12 +171,14 @@ def test_decode_sized_shards_follow_the_global_capacity(gpu_lib):
     idx_h = idx.cpu().numpy()
     bounds = [0, 2, 4, 6]
     per_shard = np.stack([np.bincount(idx_h[a:b].ravel(), minlength=wl.E) for a, b in zip(bounds, bounds[1:])])
+    per_shard_dev = torch.from_numpy(per_shard.astype(np.int32)).cuda()
     ys, dropped = [], np.zeros(wl.E, np.int64)
     for q, (a, b) in enumerate(zip(bounds, bounds[1:])):
         cfg_q = moe.config(b - a, wl.H, wl.I, wl.E, wl.k, wl.I_shared, wl.capacity_factor, wl.dtype)
         ws_q = moe.workspace(cfg_q)
         ws_q.fill_(0)
-        cap_left = torch.from_numpy(moe_pkg.shard_capacity_left(per_shard, wl.capacity(), q)).cuda()
+        cap_left = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+        moe.moe_shard_capacity_left(cfg, per_shard_dev, q, cap_left)
         y_q = torch.empty((b - a, wl.H), dtype=d["x"].dtype, device="cuda")
         dropped_q = torch.empty(wl.E, dtype=torch.int32, device="cuda")
         moe.moe_forward_routed(cfg_q, d["x"][a:b].contiguous(), idx[a:b].contiguous(), w[a:b].contiguous(),
@@ -168,7 +187,7 @@ def test_decode_sized_shards_follow_the_global_capacity(gpu_lib):
         assert moe.moe_get_device_status(cfg_q, ws_q) == 0
         ys.append(y_q)
         dropped += dropped_q.cpu().numpy()
-    ref = oracle.permute(idx_h, wl.E, wl.capacity())
+    ref = oracle.permute(idx_h, wl.E, cap_of(wl))
     assert dropped.tolist() == ref["dropped"].tolist() and int(dropped.sum()) > 0
     logits, _, _ = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
     yhat, _, _ = oracle_given_selection(wl, inp, logits, idx_h, np.arange(wl.T, dtype=np.int32))
