@@ -169,14 +169,19 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32
  * counterpart of this entry point; it only changes where the scratch lives.
  *   Same arguments, outputs and bit-exact results as moe_permute, without
  *   `ws`: the grouping kernels' scratch (about 520 KB) is a fixed array in
- *   the library's device memory, which every GPU that loads the library
- *   holds until the process exits.  This call allocates nothing (no
- *   cudaMalloc, no allocating library routine).
+ *   the library's device memory.  A GPU holds that array from the moment
+ *   the library's grouping code is loaded on it (the first grouping call of
+ *   any entry point on that device, or context creation when CUDA loads
+ *   modules eagerly) until the process exits.
+ *   Set-up: the first call on each device (each CUDA context) loads that
+ *   code if it is not loaded yet, which itself takes device memory, and
+ *   looks up the array's device address.  Make that first call at
+ *   start-up, outside any allocator callback and before any stream capture;
+ *   every later call in the same context allocates nothing (no cudaMalloc,
+ *   no allocating library routine).  After cudaDeviceReset the next call is
+ *   a first call again.
  *   Limit: T * top_k <= 1048576 slots (E <= 256 as everywhere); larger
  *   inputs return MOE_ERR_UNSUPPORTED before anything is enqueued.
- *   The first call on a device looks up the array's device address (once
- *   per device, with that device current); make that first call before any
- *   stream capture.
  *   Every call on a device shares the one array, which keeps the last
  *   call's contents; calls that overlap on the GPU (concurrent streams)
  *   race and give wrong results, so order them.  An expert index outside

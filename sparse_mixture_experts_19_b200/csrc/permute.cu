@@ -17,6 +17,8 @@
 //      with per-warp counts; the rank of a pair is the number of earlier
 //      slots of the same expert.  Slot order is token-major, hence ranks
 //      follow ascending token order, and a pair is kept iff its rank < C.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -379,8 +381,10 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
 // application owns every device allocation, and tight serving loops that
 // forbid allocation after start-up.  For them the scratch of the grouping
 // kernels (per-chunk histograms, the offsets copy and a flag word) lives in
-// this fixed file-scope device array instead of a caller workspace.  Every
-// GPU that loads the library holds it until the process exits.
+// this fixed file-scope device array instead of a caller workspace.  A GPU
+// holds the array from the moment this file's device code is loaded on it
+// (its first grouping call of any entry point, or context creation when
+// modules load eagerly) until the process exits.
 namespace {
 
 constexpr int64_t kNoAllocChunks = kNoAllocMaxSlots / kPermuteChunk;
@@ -388,25 +392,70 @@ constexpr int64_t kNoAllocInts = kNoAllocChunks * kMaxExperts + 3 * (kMaxExperts
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocInts];
 
-// Device address of g_noalloc_scratch on each device, looked up once per
-// device (with that device current).  In host code the array's name is only
-// a host-side stand-in, never a device address.
-std::mutex g_noalloc_mu;
-int32_t* g_noalloc_ptr[64] = {};
+// Device address of g_noalloc_scratch, looked up once per CUDA context (the
+// context of the stream the call enqueues on, which is current on the
+// calling thread as for any launch) and cached under that context's unique
+// id: in host code the array's name is only a host-side stand-in, never a
+// device address, and an address found in one context means nothing in
+// another (after cudaDeviceReset the device gets a new primary context with
+// a new id, and the address is looked up again).
+typedef CUresult (*StreamGetCtxFn)(CUstream, CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-cudaError_t noalloc_scratch(int32_t** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+struct ScratchEntry {
+    unsigned long long ctx_id;
+    int32_t* ptr;
+};
+std::mutex g_noalloc_mu;
+ScratchEntry g_noalloc_cache[64];
+int g_noalloc_used = 0, g_noalloc_next = 0;
+
+cudaError_t stream_context_id(cudaStream_t st, unsigned long long* id) {
+    static StreamGetCtxFn get_ctx = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuStreamGetCtx", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_ctx = reinterpret_cast<StreamGetCtxFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (!get_ctx || !get_id) return cudaErrorNotSupported;
+    CUcontext ctx = nullptr;
+    if (get_ctx(reinterpret_cast<CUstream>(st), &ctx) != CUDA_SUCCESS || !ctx) {
+        // the default stream before the runtime bound a context to this
+        // thread: cudaFree(nullptr) binds the device's primary context
+        // (it frees and allocates nothing)
+        cudaError_t e = cudaFree(nullptr);
         if (e != cudaSuccess) return e;
-        g_noalloc_ptr[dev] = static_cast<int32_t*>(ptr);
+        if (get_ctx(reinterpret_cast<CUstream>(st), &ctx) != CUDA_SUCCESS || !ctx)
+            return cudaErrorDeviceUninitialized;
     }
-    *out = g_noalloc_ptr[dev];
+    if (get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    return cudaSuccess;
+}
+
+cudaError_t noalloc_scratch(cudaStream_t st, int32_t** out) {
+    unsigned long long id = 0;
+    cudaError_t e = stream_context_id(st, &id);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    for (int i = 0; i < g_noalloc_used; ++i)
+        if (g_noalloc_cache[i].ctx_id == id) {
+            *out = g_noalloc_cache[i].ptr;
+            return cudaSuccess;
+        }
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_cache[g_noalloc_next] = ScratchEntry{id, static_cast<int32_t*>(ptr)};
+    g_noalloc_next = (g_noalloc_next + 1) % 64;
+    if (g_noalloc_used < 64) ++g_noalloc_used;
+    *out = static_cast<int32_t*>(ptr);
     return cudaSuccess;
 }
 
@@ -417,7 +466,7 @@ cudaError_t launch_permute_noalloc(const Plan& sizes, const int32_t* topk_idx, i
                                    int32_t* dropped, cudaStream_t st) {
     if (sizes.S > kNoAllocMaxSlots) return cudaErrorInvalidValue;
     int32_t* scratch = nullptr;
-    cudaError_t e = noalloc_scratch(&scratch);
+    cudaError_t e = noalloc_scratch(st, &scratch);
     if (e != cudaSuccess) return e;
     Plan p = sizes;
     p.chunk_base = scratch;                                 // [kNoAllocChunks * E]
