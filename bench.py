@@ -39,7 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s at 1 B200 and % of roofline (tensor peak or HBM GB/s)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GATEUP_KERNELS = ("gateup_sm100", "gateup_simt", "decode_gateup")
+GATEUP_KERNELS = ("gateup_sm100", "gateup_simt", "decode_layer")
 
 
 def parse_args():
@@ -366,7 +366,10 @@ def run_ours(args, wl, world, rank, local):
 
     ms_local, _, clk = run_k_steps(False, True)              # the timed run: no trace events
     ms = max_over_ranks(ms_local)
-    _, trace_dom, _ = run_k_steps(True, False, "gateup")     # the dominant kernel alone
+    # the dominant kernel alone: the decode layer kernel at decode sizes (bf16,
+    # T*k <= 8), else the grouped gate/up GEMM
+    dom_filter = "decode_layer" if (wl.dtype == "bf16" and wl.T * wl.k <= 8) else "gateup"
+    _, trace_dom, _ = run_k_steps(True, False, dom_filter)
     _, trace, _ = run_k_steps(True, False)                   # every kernel
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host
@@ -447,13 +450,11 @@ def run_ours(args, wl, world, rank, local):
         dom_times.setdefault(name, []).append(t)
     dom = next((k for k in GATEUP_KERNELS if k in dom_times), None)
     roof = None
-    if dom == "decode_gateup":
-        # weight-streaming kernel: bound by HBM; algorithmic bytes = the active
-        # experts' gate and up rows + x read + h written
+    if dom == "decode_layer":
+        # the whole layer in one weight-streaming kernel: bound by HBM;
+        # algorithmic bytes = the active experts' weights + x + y + router
         t_avg = sum(dom_times[dom]) / len(dom_times[dom]) / 1e3
-        elt = 2
-        nbytes = (active * 2 * wl.I * wl.H + 2 * wl.I_shared * wl.H + wl.T * wl.H
-                  + wl.T * wl.k * wl.I + wl.T * wl.I_shared) * elt
+        nbytes = layer_bytes(wl, active)
         achieved = nbytes / t_avg / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(dom, wl),

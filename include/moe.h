@@ -319,6 +319,78 @@ moe_status_t moe_shard_capacity_left_host(const moe_config_t* cfg, const int32_t
 moe_status_t moe_balance_losses(int32_t E, int64_t T, const float* importance, const int32_t* load,
                                 double* out);
 
+/*
+ * moe_forward_expert_shard -- this device's share of the layer under expert
+ * parallelism ("Mixture of Experts (MoEs) in Transformers", section Expert
+ * Parallelism: each device holds a slice of the experts along their first
+ * dimension; the router's global expert indices are remapped to local ones,
+ * experts the device does not hold are left out, and the devices' partial
+ * outputs are summed with an all-reduce).
+ *   cfg describes the whole layer: E all experts, the batch's T tokens and
+ *   capacity factor (capacity is per expert and global: C = moe_capacity(cfg),
+ *   served in token order over all T tokens, which every shard sees).
+ *   x [T,H]; topk_idx [T,top_k] int32 and topk_w [T,top_k] float32 as
+ *   moe_route produces them for the whole layer (replicated routing).
+ *   This shard holds experts [expert_begin, expert_begin + expert_count):
+ *   w_gate, w_up [expert_count, I, H], w_down [expert_count, H, I].
+ *   ws_gate, ws_up, ws_down: the shared expert's weights on exactly one
+ *   shard (cfg->I_shared > 0), NULL on the others.
+ *   -> y_partial [T,H] float32: sum over this shard's kept (token, expert)
+ *      pairs of w * FFN_e(x[t]) in slot order (+ the shared expert's FFN
+ *      where its weights are given), each pair's output rounded to the layer
+ *      dtype as in moe_forward; counts_out / dropped_out [expert_count]
+ *      (nullable): the shard's experts' counts before the capacity cut and
+ *      dropped pairs.
+ * The sum of all shards' y_partial, rounded once (moe_reduce_partials after
+ * an all-reduce of y_partial, or on the stacked partials of one device), is
+ * the layer's output up to float32 summation order.  Workspace:
+ * moe_workspace_size(cfg) bytes suffice.  Errors as moe_forward_routed, and
+ * an expert range outside [0, E) is MOE_ERR_INVALID_ARG.
+ */
+moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                      const float* topk_w, int32_t expert_begin, int32_t expert_count,
+                                      const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                                      const void* ws_up, const void* ws_down, float* y_partial, int32_t* counts_out,
+                                      int32_t* dropped_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_forward_mxfp4 -- moe_forward with the routed experts' weights in the
+ * MXFP4 format of the OCP Microscaling (MX) v1.0 specification, for decode
+ * sizes ("Mixture of Experts (MoEs) in Transformers", section From Dense to
+ * Sparse: the gpt-oss generation speed is set by the bytes of the active
+ * parameters, and native mxfp4 kernels would raise it further).  An element
+ * is FP4 E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa bit); each
+ * block of 32 elements along the reduction dimension shares one E8M0 scale
+ * byte s standing for 2^(s - 127) (s = 255: NaN).  Storage order (the pages
+ * give none): two codes per byte, the element with the lower index in the
+ * low nibble; a row's blocks are contiguous.
+ *   w_gate_blocks, w_up_blocks [E, I, H/32, 16] uint8; w_gate_scales,
+ *   w_up_scales [E, I, H/32] uint8; w_down_blocks [E, H, I/32, 16],
+ *   w_down_scales [E, H, I/32].  Blocks 16-byte aligned; scales any alignment.
+ *   x, router_w, y bf16 (cfg->dtype MOE_BF16); the router is moe_forward's.
+ * The weights are used exactly (every dequantized value is exact in float32);
+ * each block's 32 products are summed in f16 with the token vector scaled by
+ * a power of two into f16's range, and the blocks' sums in float32; h is
+ * rounded to bf16 between the two projections as in moe_forward.
+ * Limits: T * top_k <= 8, no shared expert (I_shared = 0), H and I multiples
+ * of 32; otherwise MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG before anything
+ * is enqueued.  Outputs and errors otherwise as moe_forward.
+ */
+moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const void* router_w, const float* router_b,
+                               const uint8_t* w_gate_blocks, const uint8_t* w_gate_scales, const uint8_t* w_up_blocks,
+                               const uint8_t* w_up_scales, const uint8_t* w_down_blocks, const uint8_t* w_down_scales,
+                               void* y, int32_t* topk_idx_out, int32_t* counts_out, int32_t* dropped_out, void* ws,
+                               size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_reduce_partials -- y = sum over i < n of partials[i], float32 in order
+ * i = 0..n-1, rounded once to the layer dtype: the last step of an
+ * expert-parallel layer (n = 1 after an all-reduce of the partial outputs).
+ *   partials [n, T, H] float32, y [T, H] layer dtype (cfg->dtype), device.
+ */
+moe_status_t moe_reduce_partials(const moe_config_t* cfg, const float* partials, int32_t n, void* y,
+                                 moe_stream_t stream);
+
 /* Waits for `stream`, then returns the device check flags (MOE_DEVFLAG_*)
  * accumulated in `ws` since the last call and clears them.  Returns
  * MOE_ERR_DEVICE_CHECK if any flag was set, MOE_OK otherwise. */

@@ -60,6 +60,10 @@ _SIGS = {
                                      ctypes.c_int),
     "moe_balance_losses": ([ctypes.c_int32, ctypes.c_int64, _P, _P, ctypes.POINTER(ctypes.c_double)],
                            ctypes.c_int),
+    "moe_forward_expert_shard": ([ctypes.POINTER(moe_config_t), _P, _P, _P, ctypes.c_int32, ctypes.c_int32]
+                                 + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_forward_mxfp4": ([ctypes.POINTER(moe_config_t)] + [_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_reduce_partials": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_int32, _P, _P], ctypes.c_int),
     "moe_get_device_status": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_size_t, _P,
                                ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
     "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -255,6 +259,56 @@ def moe_shard_capacity_left_host(cfg, counts_per_shard, shard: int):
     _check(load().moe_shard_capacity_left_host(ctypes.byref(cfg), c.ctypes.data, c.shape[0], shard,
                                                out.ctypes.data))
     return out
+
+
+def moe_forward_expert_shard(cfg, x, topk_idx, topk_w, expert_begin: int, expert_count: int, w_gate, w_up, w_down,
+                             ws_gate, ws_up, ws_down, y_partial, counts_out=None, dropped_out=None, ws=None,
+                             stream=None):
+    """This shard's float32 partial output of the layer cfg describes (experts
+    [expert_begin, expert_begin + expert_count) held here)."""
+    p, n = _ws(ws)
+    _check(load().moe_forward_expert_shard(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(topk_w), expert_begin,
+                                           expert_count, _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate),
+                                           _ptr(ws_up), _ptr(ws_down), _ptr(y_partial), _ptr(counts_out),
+                                           _ptr(dropped_out), p, n, _stream(stream)))
+
+
+def moe_forward_mxfp4(cfg, x, router_w, router_b, w_gate_blocks, w_gate_scales, w_up_blocks, w_up_scales,
+                      w_down_blocks, w_down_scales, y, topk_idx_out=None, counts_out=None, dropped_out=None, ws=None,
+                      stream=None):
+    """moe_forward with MXFP4 routed experts (uint8 blocks [E, rows, K/32, 16]
+    and scales [E, rows, K/32]); decode sizes, T * top_k <= 8."""
+    p, n = _ws(ws)
+    _check(load().moe_forward_mxfp4(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(w_gate_blocks),
+                                    _ptr(w_gate_scales), _ptr(w_up_blocks), _ptr(w_up_scales), _ptr(w_down_blocks),
+                                    _ptr(w_down_scales), _ptr(y), _ptr(topk_idx_out), _ptr(counts_out),
+                                    _ptr(dropped_out), p, n, _stream(stream)))
+
+
+def moe_reduce_partials(cfg, partials, y, stream=None):
+    """y = the float32 sum of partials [n, T, H] in order, rounded once."""
+    n = 1 if partials.dim() == 2 else partials.shape[0]
+    _check(load().moe_reduce_partials(ctypes.byref(cfg), _ptr(partials), n, _ptr(y), _stream(stream)))
+
+
+def forward_expert_parallel(cfg, x, topk_idx, topk_w, expert_begin: int, expert_count: int, w_gate, w_up, w_down,
+                            ws_gate=None, ws_up=None, ws_down=None, group=None, ws=None, stream=None):
+    """y on every rank of `group` (torch.distributed, NCCL over NVLink): this
+    rank's shard of the experts, an all-reduce of the float32 partial outputs,
+    one rounding to the layer dtype."""
+    import torch
+    import torch.distributed as dist
+
+    T, H = x.shape
+    y32 = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(cfg, x.device)
+    moe_forward_expert_shard(cfg, x, topk_idx, topk_w, expert_begin, expert_count, w_gate, w_up, w_down, ws_gate,
+                             ws_up, ws_down, y32, ws=ws, stream=stream)
+    dist.all_reduce(y32, group=group)  # the exchange step
+    y = torch.empty_like(x)
+    moe_reduce_partials(cfg, y32, y, stream)
+    return y
 
 
 def moe_get_device_status(cfg, ws, stream=None) -> int:

@@ -26,6 +26,8 @@ struct Plan {
     const int32_t* cap_left_arr;   // [E] device or null: capacity left per expert (token shards)
     float* importance;             // [E] device or null: router importance, added to
     bool bf16;
+    bool drop_negative;            // expert index -1 = another shard's expert: dropped, not counted, no flag
+    bool y_f32;                    // y is a float32 partial sum (expert shards), not the layer dtype
     int64_t nchunks;               // ceil(S / kPermuteChunk)
     int64_t h_rows;                // S + (Is ? T : 0)
     int64_t I_max;                 // max(I, Is)
@@ -44,8 +46,8 @@ struct Plan {
     void* xperm;          // [S, H] layer dtype: x rows in grouped order
     void* h;              // [S, I] + [T, Is] layer dtype: SwiGLU activations
     void* rows;           // [S + T, H] layer dtype: routing-weighted expert output rows
-    float* dec_part;      // decode FFN (S <= kDecodeMaxSlots): [H, S + T] partial dot products
-    int32_t* dec_cnt;     // decode FFN: [H] arrivals per output column
+    double* dec_scores;   // decode layer (S <= kDecodeMaxSlots): [T, E] router scores
+    unsigned int* dec_bar;  // decode layer: [2] grid-barrier arrival counters
     size_t bytes;         // total workspace bytes
 };
 
@@ -85,13 +87,22 @@ cudaError_t launch_router_decode(const Plan& p, const void* x, const void* route
 // Scores of T*E*H at most this many multiply-adds go to the per-token router
 // (its weight traffic, T*E*H*2 bytes from L2, stays small).
 constexpr int64_t kDecodeRouterMaxMacs = int64_t(1) << 26;
-// Decode FFN (bf16, T*k <= kDecodeMaxSlots): expert FFNs and the weighted
-// combine as two weight-streaming kernels, y written directly; also writes
-// counts and dropped.
+// Decode layer (bf16, T*k <= kDecodeMaxSlots): routing (unless given), the
+// expert FFNs and the weighted combine in one cooperative weight-streaming
+// kernel, y written directly; also writes counts and dropped, and
+// topk_idx_out when non-null.
 bool decode_ffn_eligible(const Plan& p);
-cudaError_t launch_decode_ffn(const Plan& p, const void* x, const int32_t* topk_idx, const void* w_gate,
-                              const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
-                              const void* ws_down, void* y, int32_t* counts, int32_t* dropped, cudaStream_t st);
+cudaError_t launch_decode_layer(const Plan& p, const void* x, const void* router_w, const float* router_b,
+                                const int32_t* topk_idx_in, const float* topk_w_in, int32_t* topk_idx_out,
+                                const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                                const void* ws_up, const void* ws_down, void* y, int32_t* counts,
+                                int32_t* dropped, cudaStream_t st);
+// The same with the routed experts in MXFP4 (no shared expert; H, I multiples
+// of 32): mx = {gate blocks, gate scales, up blocks, up scales, down blocks,
+// down scales}.
+cudaError_t launch_decode_layer_mxfp4(const Plan& p, const void* x, const void* router_w, const float* router_b,
+                                      int32_t* topk_idx_out, const uint8_t* const (&mx)[6], void* y, int32_t* counts,
+                                      int32_t* dropped, cudaStream_t st);
 cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
                            int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
                            int32_t* dropped, cudaStream_t st);
@@ -129,6 +140,14 @@ cudaError_t launch_combine_rows(const Plan& p, const void* rows, const int32_t* 
 // Stage API: y[t] = sum_j topk_w[t,j] * expert_out[row_of[t,j]] (+ shared row).
 cudaError_t launch_combine(const Plan& p, const float* expert_out, const int32_t* row_of,
                            const float* topk_w, void* y, cudaStream_t st);
+
+// Expert shards: topk_idx -> shard-local expert ids (expert - begin for
+// experts in [begin, begin + count), else -1).
+cudaError_t launch_remap_experts(const int32_t* idx, int64_t S, int begin, int count, int32_t* local,
+                                 cudaStream_t st);
+// y[t, h] = dtype(sum over i < n of partials[i][t][h]), float32, i in order.
+cudaError_t launch_reduce_partials(const float* partials, int n, int64_t count, bool bf16_out, void* y,
+                                   cudaStream_t st);
 
 // capacity_left[e] = max(0, C - sum_{q < shard} counts[q][e]) for one token
 // shard of a batch with capacity C (device kernel / host loop).

@@ -180,9 +180,9 @@ __global__ void scatter_x_rows_kernel(const uint4* __restrict__ x, const int32_t
 
 // y[t] = sum_j rows[row_of[t,j]] (+ rows[S + t]); one thread per 16-byte chunk
 // of a token's row, float32 sum in slot order, one rounding at the end.
-template <typename TV>
+template <typename TV, typename TOut>
 __global__ void combine_rows_kernel(const TV* __restrict__ rows, const int32_t* __restrict__ row_of,
-                                    int64_t T, int H, int k, int64_t S, int shared, TV* __restrict__ y) {
+                                    int64_t T, int H, int k, int64_t S, int shared, TOut* __restrict__ y) {
     constexpr int V = 16 / sizeof(TV);
     const int chunks = H / V;
     const int64_t n = T * chunks;
@@ -204,11 +204,17 @@ __global__ void combine_rows_kernel(const TV* __restrict__ rows, const int32_t* 
             if (r >= 0) add_row(r);
         }
         if (shared) add_row(S + t);
-        uint4 o;
-        TV* ov = reinterpret_cast<TV*>(&o);
+        TOut* dst = y + t * H + (int64_t)c * V;
+        if (sizeof(TOut) == sizeof(TV)) {
+            uint4 o;
+            TOut* ov = reinterpret_cast<TOut*>(&o);
 #pragma unroll
-        for (int v = 0; v < V; ++v) ov[v] = from_f32<TV>(acc[v]);
-        *reinterpret_cast<uint4*>(y + t * H + (int64_t)c * V) = o;
+            for (int v = 0; v < V; ++v) ov[v] = from_f32<TOut>(acc[v]);
+            *reinterpret_cast<uint4*>(dst) = o;
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) dst[v] = from_f32<TOut>(acc[v]);
+        }
     }
 }
 
@@ -302,11 +308,14 @@ cudaError_t launch_combine_rows(const Plan& p, const void* rows, const int32_t* 
     const int64_t n = p.T * p.H / (p.bf16 ? 8 : 4);
     if (n == 0) return cudaSuccess;
     trace_before("combine_rows", st);
-    if (p.bf16)
-        combine_rows_kernel<bf16><<<grid_for(n, 256), 256, 0, st>>>(
+    if (p.bf16 && p.y_f32)
+        combine_rows_kernel<bf16, float><<<grid_for(n, 256), 256, 0, st>>>(
+            (const bf16*)rows, row_of, p.T, (int)p.H, (int)p.k, p.S, p.Is > 0, (float*)y);
+    else if (p.bf16)
+        combine_rows_kernel<bf16, bf16><<<grid_for(n, 256), 256, 0, st>>>(
             (const bf16*)rows, row_of, p.T, (int)p.H, (int)p.k, p.S, p.Is > 0, (bf16*)y);
     else
-        combine_rows_kernel<float><<<grid_for(n, 256), 256, 0, st>>>(
+        combine_rows_kernel<float, float><<<grid_for(n, 256), 256, 0, st>>>(
             (const float*)rows, row_of, p.T, (int)p.H, (int)p.k, p.S, p.Is > 0, (float*)y);
     trace_after(st);
     return cudaGetLastError();

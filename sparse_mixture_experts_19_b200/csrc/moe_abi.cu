@@ -107,6 +107,8 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->cap_left_arr = nullptr;
     p->importance = nullptr;
     p->bf16 = (c->dtype == MOE_BF16);
+    p->drop_negative = false;
+    p->y_f32 = false;
     p->nchunks = (p->S + kPermuteChunk - 1) / kPermuteChunk;
     p->h_rows = p->S + (p->Is ? p->T : 0);
     p->I_max = p->I > p->Is ? p->I : p->Is;
@@ -132,9 +134,9 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->xperm = take(elt * p->S * p->H);
     p->h = take(elt * (p->S * p->I + p->T * p->Is));
     p->rows = take(elt * (p->S + (p->Is ? p->T : 0)) * p->H);
-    const int64_t dec_cols = p->S <= kDecodeMaxSlots ? p->S + (p->Is ? p->T : 0) : 0;
-    p->dec_part = (float*)take(sizeof(float) * p->H * dec_cols);
-    p->dec_cnt = (int32_t*)take(dec_cols ? sizeof(int32_t) * p->H : 0);
+    const bool dec = p->S <= kDecodeMaxSlots;
+    p->dec_scores = (double*)take(dec ? sizeof(double) * p->T * p->E : 0);
+    p->dec_bar = (unsigned int*)take(dec ? 2 * sizeof(unsigned int) : 0);
     p->bytes = off;
 }
 
@@ -359,9 +361,10 @@ static moe_status_t forward_after_routing(Plan& p, const void* x, const int32_t*
                                           const void* ws_up, const void* ws_down, void* y, int32_t* counts,
                                           int32_t* dropped, cudaStream_t st) {
     if (decode_ffn_eligible(p)) {
-        // few slots: weight-streaming FFN kernels, no grouped rows
-        CUDA_TRY(launch_decode_ffn(p, x, idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, counts, dropped, st),
-                 "decode_ffn");
+        // few slots: the weight-streaming decode layer, no grouped rows
+        CUDA_TRY(launch_decode_layer(p, x, nullptr, nullptr, idx, p.topk_w, nullptr, w_gate, w_up, w_down, ws_gate,
+                                     ws_up, ws_down, y, counts, dropped, st),
+                 "decode_layer");
         return MOE_OK;
     }
     CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
@@ -402,6 +405,13 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* rou
     int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
+    if (decode_ffn_eligible(p)) {
+        // few slots: routing, expert FFNs and combine in one decode kernel
+        CUDA_TRY(launch_decode_layer(p, x, router_w, router_b, nullptr, nullptr, topk_idx_out, w_gate, w_up, w_down,
+                                     ws_gate, ws_up, ws_down, y, counts, dropped, st),
+                 "decode_layer");
+        return MOE_OK;
+    }
     CUDA_TRY(run_router(p, x, router_w, router_b, idx, p.topk_w, st), "router");
     return forward_after_routing(p, x, idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, counts, dropped, st);
 }
@@ -503,6 +513,110 @@ moe_status_t moe_balance_losses(int32_t E, int64_t T, const float* importance, c
     out[0] = kl / E;
     out[1] = sqrt(vi / (E - 1)) + sqrt(vl / (E - 1));
     out[2] = E * sw;
+    return MOE_OK;
+}
+
+moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                      const float* topk_w, int32_t expert_begin, int32_t expert_count,
+                                      const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                                      const void* ws_up, const void* ws_down, float* y_partial, int32_t* counts_out,
+                                      int32_t* dropped_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status_t s = check_config(cfg);
+    if (s != MOE_OK) return s;
+    if (expert_count < 1 || expert_begin < 0 || (int64_t)expert_begin + expert_count > cfg->E)
+        return fail(MOE_ERR_INVALID_ARG, "experts [%d, %d + %d) outside [0, %d)", expert_begin, expert_begin,
+                    expert_count, cfg->E);
+    if (ws_gate && cfg->I_shared == 0)
+        return fail(MOE_ERR_INVALID_ARG, "shared-expert weights given but I_shared = 0");
+    // the shard's plan: its experts only, the shared expert where its weights
+    // are given, the batch's capacity
+    moe_config_t local = *cfg;
+    local.E = expert_count;
+    local.I_shared = ws_gate ? cfg->I_shared : 0;
+    Plan p;
+    make_plan(&local, nullptr, &p);
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+    if ((uintptr_t)ws % kWsAlign) return fail(MOE_ERR_WORKSPACE, "workspace not %d-byte aligned", kWsAlign);
+    if (ws_bytes < p.bytes) return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, p.bytes);
+    make_plan(&local, ws, &p);
+    p.cap = capacity_of(cfg);
+    p.drop_negative = true;
+    p.y_f32 = true;
+    OPTIONAL_PTR(counts_out);
+    OPTIONAL_PTR(dropped_out);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (p.T == 0) {
+        if (counts_out) CUDA_TRY(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * p.E, st), "memset");
+        if (dropped_out) CUDA_TRY(cudaMemsetAsync(dropped_out, 0, sizeof(int32_t) * p.E, st), "memset");
+        return MOE_OK;
+    }
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    REQUIRE_PTR(w_gate);
+    REQUIRE_PTR(w_up);
+    REQUIRE_PTR(w_down);
+    REQUIRE_PTR(y_partial);
+    if ((s = check_shared(p, ws_gate, ws_up, ws_down)) != MOE_OK) return s;
+    CUDA_TRY(launch_remap_experts(topk_idx, p.S, expert_begin, expert_count, p.topk_idx, st), "remap_experts");
+    p.topk_w = const_cast<float*>(topk_w);  // read only on this path
+    int32_t* counts = counts_out ? counts_out : p.counts;
+    int32_t* dropped = dropped_out ? dropped_out : p.dropped;
+    return forward_after_routing(p, x, p.topk_idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y_partial, counts,
+                                 dropped, st);
+}
+
+moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const void* router_w, const float* router_b,
+                               const uint8_t* w_gate_blocks, const uint8_t* w_gate_scales, const uint8_t* w_up_blocks,
+                               const uint8_t* w_up_scales, const uint8_t* w_down_blocks, const uint8_t* w_down_scales,
+                               void* y, int32_t* topk_idx_out, int32_t* counts_out, int32_t* dropped_out, void* ws,
+                               size_t ws_bytes, moe_stream_t stream) {
+    Plan p;
+    moe_status_t s = plan_for(cfg, ws, ws_bytes, &p);
+    if (s != MOE_OK) return s;
+    if (!p.bf16) return fail(MOE_ERR_UNSUPPORTED, "moe_forward_mxfp4 takes bf16 activations (dtype MOE_BF16)");
+    if (p.Is > 0) return fail(MOE_ERR_UNSUPPORTED, "moe_forward_mxfp4 has no shared expert (I_shared must be 0)");
+    if (p.H % 32 || p.I % 32) return fail(MOE_ERR_INVALID_ARG, "H and I must be multiples of 32 (MXFP4 blocks)");
+    OPTIONAL_PTR(topk_idx_out);
+    OPTIONAL_PTR(counts_out);
+    OPTIONAL_PTR(dropped_out);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (p.T == 0) {
+        if (counts_out) CUDA_TRY(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * p.E, st), "memset");
+        if (dropped_out) CUDA_TRY(cudaMemsetAsync(dropped_out, 0, sizeof(int32_t) * p.E, st), "memset");
+        return MOE_OK;
+    }
+    if (!decode_ffn_eligible(p))
+        return fail(MOE_ERR_UNSUPPORTED, "moe_forward_mxfp4 serves T*top_k <= %d routed slots (got %lld)",
+                    kDecodeMaxSlots, (long long)p.S);
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(router_w);
+    OPTIONAL_PTR(router_b);
+    REQUIRE_PTR(w_gate_blocks);
+    REQUIRE_PTR(w_up_blocks);
+    REQUIRE_PTR(w_down_blocks);
+    if (!w_gate_scales || !w_up_scales || !w_down_scales)
+        return fail(MOE_ERR_INVALID_ARG, "the three scale arrays are required");
+    REQUIRE_PTR(y);
+    const uint8_t* mx[6] = {w_gate_blocks, w_gate_scales, w_up_blocks, w_up_scales, w_down_blocks, w_down_scales};
+    int32_t* counts = counts_out ? counts_out : p.counts;
+    int32_t* dropped = dropped_out ? dropped_out : p.dropped;
+    CUDA_TRY(launch_decode_layer_mxfp4(p, x, router_w, router_b, topk_idx_out, mx, y, counts, dropped, st),
+             "decode_layer_mxfp4");
+    return MOE_OK;
+}
+
+moe_status_t moe_reduce_partials(const moe_config_t* cfg, const float* partials, int32_t n, void* y,
+                                 moe_stream_t stream) {
+    moe_status_t s = check_config(cfg);
+    if (s != MOE_OK) return s;
+    if (n < 1) return fail(MOE_ERR_INVALID_ARG, "n = %d < 1", n);
+    if ((int64_t)cfg->T * cfg->H == 0) return MOE_OK;
+    REQUIRE_PTR(partials);
+    REQUIRE_PTR(y);
+    CUDA_TRY(launch_reduce_partials(partials, n, (int64_t)cfg->T * cfg->H, cfg->dtype == MOE_BF16, y,
+                                    (cudaStream_t)stream),
+             "reduce_partials");
     return MOE_OK;
 }
 

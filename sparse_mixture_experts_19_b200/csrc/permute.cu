@@ -34,7 +34,7 @@ constexpr int kChunkScanThreads = 1024;
 
 __global__ void __launch_bounds__(kHistThreads) permute_hist_kernel(
     const int32_t* __restrict__ idx, int64_t S, int E, int32_t* __restrict__ hist,
-    int32_t* __restrict__ flags) {
+    int32_t* __restrict__ flags, bool drop_negative) {
     __shared__ int32_t h[kMaxExperts];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kHistThreads) permute_hist_kernel(
         int e = idx[s];
         if (e >= 0 && e < E)
             atomicAdd(&h[e], 1);
-        else
+        else if (!(drop_negative && e == -1))
             bad = true;
     }
     if (bad) set_flag(flags, MOE_DEVFLAG_BAD_EXPERT_INDEX);
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
     int32_t* __restrict__ counts,
     int32_t* __restrict__ dropped, int32_t* offsets_out, int32_t* offsets_ws,
     int32_t* __restrict__ mtile_prefix, int32_t* __restrict__ mpair_prefix, int32_t shared_rows,
-    int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of, int32_t* __restrict__ flags) {
+    int32_t* __restrict__ perm_rows, int32_t* __restrict__ row_of, int32_t* __restrict__ flags, bool drop_negative) {
     __shared__ int32_t wcount[kSmallWarps][kScanThreads];  // per warp segment, per expert
     __shared__ int32_t sm[kScanThreads];
     __shared__ int32_t off[kScanThreads + 1];
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kScanThreads) permute_small_kernel(
         const int s = sb + lane;
         const int ex = (s < s1) ? idx[s] : -1;
         const bool valid = (ex >= 0 && ex < E);
-        if (s < s1 && !valid) bad = true;
+        if (s < s1 && !valid && !(drop_negative && ex == -1)) bad = true;
         const uint32_t peers = __match_any_sync(0xffffffffu, valid ? ex : -1);
         if (valid && (peers & lt) == 0) wcount[warp][ex] += __popc(peers);
         __syncwarp();
@@ -346,13 +346,14 @@ cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* coun
         trace_before("permute_small", st);
         permute_small_kernel<<<1, kScanThreads, 0, st>>>(topk_idx, (int)p.S, E, p.cap, p.cap_left_arr, counts, dropped, offsets,
                                                          p.offsets, p.mtile_prefix, p.mpair_prefix,
-                                                         (int32_t)(p.Is > 0 ? p.T : 0), perm_rows, row_of, p.flags);
+                                                         (int32_t)(p.Is > 0 ? p.T : 0), perm_rows, row_of, p.flags,
+                                                         p.drop_negative);
         trace_after(st);
         return cudaGetLastError();
     }
     trace_before("permute_hist", st);
     permute_hist_kernel<<<(unsigned)p.nchunks, kHistThreads, 0, st>>>(topk_idx, p.S, E,
-                                                                       p.chunk_base, p.flags);
+                                                                       p.chunk_base, p.flags, p.drop_negative);
     trace_after(st);
     trace_before("permute_scan_chunks", st);
     permute_scan_chunks_kernel<<<(unsigned)E, kChunkScanThreads, 0, st>>>(p.chunk_base, p.nchunks, E, counts);
@@ -415,12 +416,16 @@ cudaError_t stream_context_id(cudaStream_t st, unsigned long long* id) {
     static CtxGetIdFn get_id = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
+        // the entry points of the CUDA 12.0 ABI, whose signatures the
+        // typedefs above spell out (a plain lookup would return the newest
+        // version, e.g. the three-argument cuStreamGetCtx of CUDA 12.5)
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuStreamGetCtx", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        if (cudaGetDriverEntryPointByVersion("cuStreamGetCtx", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             get_ctx = reinterpret_cast<StreamGetCtxFn>(p);
-        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             get_id = reinterpret_cast<CtxGetIdFn>(p);
     });

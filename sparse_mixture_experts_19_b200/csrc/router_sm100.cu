@@ -15,13 +15,34 @@
 // the softmax of those k.  The epilogue of one tile overlaps the loads and
 // MMAs of the next.
 //
-// Exactness of the decision.  Tensor-core float32 sums differ from exact
-// sums by a small accumulation error.  A token whose approximate k-th and
-// (k+1)-th scores are within delta (8x a bound on that error) has the
-// experts of the band [s_k - delta, s_{k+1} + delta] rescored exactly in
-// fp64 (bf16 products are exact) by warp-cooperative dot products, and its
-// selection is completed from those exact scores.  Experts above the band
-// are certainly selected, experts below it certainly not.
+// Exactness of the decision and of the order.  Tensor-core float32 sums
+// differ from the exact scores; the epilogue bounds that difference for each
+// token by
+//   delta_t = c_H * ||x_t|| * max_e ||w_e|| + 2^-23 * (||x_t|| max_e ||w_e|| + max_e |b_e|),
+// where ||x_t|| * ||w_e|| >= sum_h |x_th w_eh| (Cauchy-Schwarz) and
+// c_H = 17 * 2^-23 * (number of MMA steps + 1).  The constant rests on a
+// model of the tensor core, assumed rather than documented: one kind::f16
+// step adds its 16 exact bf16 products to the float32 accumulator D with an
+// error of at most 17 * 2^-23 * (|D| + sum |products|), which is what 16
+// float32 additions with round-toward-zero can lose in any order, and what
+// a multi-term adder that aligns every term to the largest and truncates
+// below 24 bits of it can lose.  Summed over the steps, the error of a score
+// is at most c_H * sum_h |x_th w_eh|; the last term covers the rounding of
+// the bias addition.  The norms come from the MMA warp's idle lanes, which
+// read every x stage (and, on the CTA's first tile, every router-weight
+// stage) from shared memory after issuing its MMAs; they are summed in
+// float32 and inflated by 1 + H * 2^-22 to stay upper bounds.
+//   Selection: an expert whose approximate score exceeds the (k+1)-th
+// approximate score by more than 2 delta is certainly selected, one below the
+// k-th by more than 2 delta certainly not; the experts in between (the band)
+// are rescored exactly in fp64 (bf16 products are exact) by warp-cooperative
+// dot products and the selection is completed from those exact scores,
+// ties to the lower index.
+//   Order: two selected experts whose approximate scores are more than
+// 2 delta apart are in the right order; every selected expert with another
+// one within 2 delta gets its exact score too, and the k are sorted with
+// exact scores where both have one (ties to the lower index) and
+// approximate ones otherwise.  The result is the exact order.
 //
 // Importance (optional).  Before the accumulator is handed back, each thread
 // forms its token's softmax over all E float32 scores, each warp sums the 32
@@ -43,6 +64,31 @@ constexpr int kMaxStages = 8;
 constexpr int kThreads = 192;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kQueue = 512;  // exact-rescoring queue entries per CTA and tile
+
+constexpr int kBRowsMax = kMaxExperts;  // router rows per stage at most (E padded to 16)
+
+// Sum of squares of the 64 bf16 values of one 128-byte row of a swizzled
+// shared-memory tile at shared address `row`; lane l reads its 16-byte
+// chunks starting at chunk l % 8, so 32 lanes reading 32 rows at once touch
+// every bank equally.
+__device__ __forceinline__ float row_sumsq(uint32_t row, int lane) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(row + (uint32_t)(((i + lane) & 7) * 16)));
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            s = fmaf(f.x, f.x, s);
+            s = fmaf(f.y, f.y, s);
+        }
+    }
+    return s;
+}
 
 // (a, ea) ranks before (b, eb): larger score, then lower expert index.
 __device__ __forceinline__ bool ranks_before(float a, int ea, float b, int eb) {
@@ -144,16 +190,20 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     uint8_t* tail = smem + stages * stage_bytes;
     int2* qp = reinterpret_cast<int2*>(tail);                   // [kQueue] (row, expert)
     double* qs = reinterpret_cast<double*>(qp + kQueue);       // [kQueue] exact scores
-    uint8_t* misc = reinterpret_cast<uint8_t*>(qs + kQueue);   // 1024-aligned, 256 bytes
+    float* qa = reinterpret_cast<float*>(qs + kQueue);         // [kQueue] approximate scores
+    uint8_t* misc = reinterpret_cast<uint8_t*>(qa + kQueue);   // 1024-aligned, 256 bytes
     uint64_t* full = reinterpret_cast<uint64_t*>(misc);        // [stages]
     uint64_t* empty = full + kMaxStages;
     uint64_t* tfull = empty + kMaxStages;
     uint64_t* tempty = tfull + 2;
-    uint64_t* drain = tempty + 2;
+    uint64_t* nready = tempty + 2;  // squared x norms of an accumulator's tile written
+    uint64_t* drain = nready + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     int* qn = reinterpret_cast<int*>(tmem_holder + 2);
-    float* bs = reinterpret_cast<float*>(misc + 256);  // [E rounded up to 64], 16-byte aligned
+    float* wmax2 = reinterpret_cast<float*>(tmem_holder + 3);  // max_e ||w_e||^2 (after the first tile)
+    float* xnorm2 = reinterpret_cast<float*>(misc + 256);      // [2][128] ||x_t||^2 per accumulator
+    float* bs = xnorm2 + 2 * kBM;                              // [E rounded up to 64], 16-byte aligned
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const bool has_bias = bias != nullptr;
@@ -162,14 +212,16 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], 2);  // the MMAs' commit and the norm pass of the MMA warp
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], 128);
+            mbar_init(&nready[i], 1);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
+        *wmax2 = 0.f;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -204,35 +256,71 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                 drain_wait(&full[j % stages], (j / stages) & 1);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(kBM, Npad);
-            uint32_t it = 0, tc = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
-                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-                if (!wait_or_abort(&tempty[acc], aph ^ 1, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) break;
+        // ------------------------------------------------ MMA issuer (lane 0) + norms (all lanes)
+        const uint32_t idesc = idesc_bf16(kBM, Npad);
+        uint32_t it = 0, tc = 0;
+        float wsq[kBRowsMax / 32];  // ||w_e||^2 of router rows lane + 32 i (first tile)
+#pragma unroll
+        for (int i = 0; i < kBRowsMax / 32; ++i) wsq[i] = 0.f;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok && !*abort_flag; tile += gridDim.x, ++tc) {
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!wait_or_abort(&tempty[acc], aph ^ 1, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + acc * acc_cols;
+            float xsq[kBM / 32];  // ||x_t||^2 of tile rows lane + 32 q
+#pragma unroll
+            for (int q = 0; q < kBM / 32; ++q) xsq[q] = 0.f;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % stages;
+                const uint32_t ph = (it / stages) & 1;
+                if (!wait_or_abort(&full[s], ph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t d = tmem_base + acc * acc_cols;
-                bool ok = true;
-                for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % stages;
-                    const uint32_t ph = (it / stages) & 1;
-                    if (!wait_or_abort(&full[s], ph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(smem + s * stage_bytes);
-                    const uint32_t b0 = a0 + kABytes;
+                const uint32_t a0 = smem_u32(smem + s * stage_bytes);
+                const uint32_t b0 = a0 + kABytes;
+                if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
                         mma_bf16(d, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc,
                                  (kb | kk) != 0);
                     mma_commit(&empty[s]);
                 }
-                if (!ok) break;
-                mma_commit(&tfull[acc]);
+                // squared norms of the stage's rows (128-byte rows, 16-byte
+                // chunks permuted inside a row by the swizzle, which a sum of
+                // squares does not see); lane l reads chunk (i + l) % 8 in
+                // step i, so a warp's 32 loads spread over all banks
+#pragma unroll
+                for (int q = 0; q < kBM / 32; ++q) xsq[q] += row_sumsq(a0 + (uint32_t)(lane + 32 * q) * 128u, lane);
+                if (tc == 0) {
+#pragma unroll
+                    for (int i = 0; i < kBRowsMax / 32; ++i)
+                        if (lane + 32 * i < Npad) wsq[i] += row_sumsq(b0 + (uint32_t)(lane + 32 * i) * 128u, lane);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
             }
+            if (!ok) break;
+            if (lane == 0) mma_commit(&tfull[acc]);
+#pragma unroll
+            for (int q = 0; q < kBM / 32; ++q) xnorm2[acc * kBM + lane + 32 * q] = xsq[q];
+            if (tc == 0) {
+                float m = 0.f;
+#pragma unroll
+                for (int i = 0; i < kBRowsMax / 32; ++i) m = fmaxf(m, wsq[i]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) *wmax2 = m;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&nready[acc]);  // release: the norms above are visible to its waiters
+        }
+        if (lane == 0) {
             mma_commit(drain);
             drain_wait(drain, 0);
         }
@@ -241,16 +329,26 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
         const int q = warp & 3;
         const int r = q * 32 + lane;  // token row of this thread within the tile
         const int ew = warp - 2;      // epilogue warp 0..3
+        // the bound on |approximate - exact score| (see the file comment)
+        const float u23 = 1.1920929e-7f;  // 2^-23
+        const float cH = 17.f * u23 * (float)(4 * nkb + 1) * 1.01f;
+        const float slack = 1.f + (float)H * 2.3841858e-7f;  // 1 + H 2^-22: float32 sums of squares as upper bounds
+        float bmax = 0.f;
+        for (int e = 0; e < E; ++e) bmax = fmaxf(bmax, fabsf(bs[e]));
         uint32_t tc = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-            const bool ready = wait_or_abort(&tfull[acc], aph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT);
+            bool ready = wait_or_abort(&tfull[acc], aph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT);
+            ready = ready && wait_or_abort(&nready[acc], aph, abort_flag, flags, MOE_DEVFLAG_WAIT_TIMEOUT);
             // all 128 epilogue threads take the same branch, so every named
             // barrier below is reached by all of them
             if (!epilogue_all(ready)) break;
             tc_fence_after();
             const int t = tile * kBM + r;
             const uint32_t tq = tmem_base + acc * acc_cols + ((uint32_t)(q * 32) << 16);
+            // twice the bound: the width of the uncertain band on each side
+            const float anorm = sqrtf(xnorm2[acc * kBM + r] * slack) * sqrtf(*wmax2 * slack);
+            const float del2 = 2.f * 1.001f * (cH * anorm + u23 * (anorm + bmax));
 
             // pass 1: the k (+1) best approximate scores, picked in k (+1)
             // rounds; round j takes the best score ranking after the pick of
@@ -259,7 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
             float tv[KMAX + 1];
             int te[KMAX + 1];
             const int kk = k < E ? k + 1 : k;
-            float amax = 0.f;
             float pv = INFINITY;
             int pe = -1;
 #pragma unroll
@@ -273,23 +370,19 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                     for (int c0 = 0; c0 < E; c0 += 64) {
                         float v[64];
                         tmem_ld64(tq + c0, v);  // columns past E (up to the allocation) are ignored
-                        if (j == 0) {
-                            // round 0: magnitude of the raw sums, then the bias is added
-                            // once and the biased scores are written back to TMEM for
-                            // the later rounds and the band pass
+                        if (j == 0 && has_bias) {
+                            // round 0: the bias is added once and the biased
+                            // scores are written back to TMEM for the later
+                            // rounds and the band pass
 #pragma unroll
-                            for (int i = 0; i < 64; ++i) amax = fmaxf(amax, (c0 + i < E) ? fabsf(v[i]) : 0.f);
-                            if (has_bias) {
-#pragma unroll
-                                for (int i = 0; i < 64; i += 4) {
-                                    const float4 b4 = *reinterpret_cast<const float4*>(bs + c0 + i);
-                                    v[i] += b4.x;
-                                    v[i + 1] += b4.y;
-                                    v[i + 2] += b4.z;
-                                    v[i + 3] += b4.w;
-                                }
-                                tmem_st64(tq + c0, v);
+                            for (int i = 0; i < 64; i += 4) {
+                                const float4 b4 = *reinterpret_cast<const float4*>(bs + c0 + i);
+                                v[i] += b4.x;
+                                v[i + 1] += b4.y;
+                                v[i + 2] += b4.z;
+                                v[i + 3] += b4.w;
                             }
+                            tmem_st64(tq + c0, v);
                         }
 #pragma unroll
                         for (int i = 0; i < 64; ++i) {
@@ -326,11 +419,10 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                     if (j == k - 1) kth = tv[j];
                     if (j == k) next = tv[j];
                 }
-                const float delta = 0.5f * (float)H * 1.1920929e-7f * fmaxf(amax, 1.0f);
-                if (kth - next <= delta) {
+                if (kth - next <= del2) {
                     uncertain = true;
-                    band_lo = kth - delta;
-                    band_hi = next + delta;
+                    band_lo = kth - del2;
+                    band_hi = next + del2;
                     n_in = 0;
 #pragma unroll
                     for (int j = 0; j < KMAX; ++j)
@@ -339,14 +431,17 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
             }
 
             // final selection state: certain prefix + the best `need` band
-            // members by exact score (ties to the lower index)
+            // members by exact score (ties to the lower index), with their
+            // approximate scores
             const int need = k - n_in;
             double bv[KMAX];
             int be[KMAX];
+            float ba[KMAX];
 #pragma unroll
             for (int j = 0; j < KMAX; ++j) {
                 bv[j] = -INFINITY;
                 be[j] = 0x7fffffff;
+                ba[j] = -INFINITY;
             }
             // pass 2, in rounds of at most kQueue band members per tile: queue
             // them (scores re-read from TMEM), rescore them exactly with whole
@@ -369,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                                     const int slot = atomicAdd(qn, 1);
                                     if (slot < kQueue) {
                                         qp[slot] = make_int2(r, e);
+                                        qa[slot] = sv;
                                     } else {
                                         stop = true;  // queue full: resume here next round
                                         cursor = e;
@@ -394,15 +490,19 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                         // insert (qs[i], pr.y) into the `need` best, ties to the lower index
                         double cv = qs[i];
                         int ce = pr.y;
+                        float ca = qa[i];
 #pragma unroll
                         for (int j = 0; j < KMAX; ++j) {
                             if (j < need && (cv > bv[j] || (cv == bv[j] && ce < be[j]))) {
                                 const double ov = bv[j];
                                 const int oe = be[j];
+                                const float oa = ba[j];
                                 bv[j] = cv;
                                 be[j] = ce;
+                                ba[j] = ca;
                                 cv = ov;
                                 ce = oe;
+                                ca = oa;
                             }
                         }
                     }
@@ -435,12 +535,17 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
 
-            float fv[KMAX];
+            // the k selected: approximate score fa, expert fe, exact score fx
+            // where known (bit j of has_x)
+            float fa[KMAX];
             int fe[KMAX];
+            double fx[KMAX];
+            uint32_t has_x = 0;
 #pragma unroll
             for (int j = 0; j < KMAX; ++j) {
-                fv[j] = tv[j];
+                fa[j] = tv[j];
                 fe[j] = te[j];
+                fx[j] = 0.0;
             }
             if (!kDense && uncertain) {
                 // move the band picks to slots n_in..k-1: n_in predicated
@@ -452,30 +557,103 @@ __global__ void __launch_bounds__(kThreads, 1) router_sm100_kernel(
                         for (int j = KMAX - 1; j > 0; --j) {
                             bv[j] = bv[j - 1];
                             be[j] = be[j - 1];
+                            ba[j] = ba[j - 1];
                         }
                     }
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
                     if (j >= n_in && j < k) {
-                        fv[j] = (float)bv[j];
+                        fa[j] = ba[j];
                         fe[j] = be[j];
+                        fx[j] = bv[j];
+                        has_x |= 1u << j;
                     }
             }
+            // order: every selected expert with another selected one within
+            // 2 delta (approximate scores) needs its exact score
+            uint32_t pending = 0;
             if (t < T) {
-                float m = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < KMAX; ++i)
+#pragma unroll
+                    for (int j = i + 1; j < KMAX; ++j)
+                        if (j < k && fabsf(fa[i] - fa[j]) <= del2) pending |= (1u << i) | (1u << j);
+                pending &= ~has_x;
+            }
+            while (epilogue_any(pending != 0)) {
+                if (threadIdx.x == 64) *qn = 0;
+                epilogue_sync();
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
-                    if (j < k) m = fmaxf(m, fv[j]);
+                    if ((pending >> j) & 1u) {
+                        const int slot = atomicAdd(qn, 1);
+                        if (slot < kQueue) {
+                            qp[slot] = make_int2(r, fe[j]);
+                            pending &= ~(1u << j);
+                        }
+                    }
+                epilogue_sync();
+                const int nq = min(*qn, kQueue);
+                for (int i = ew; i < nq; i += 4) {
+                    const int2 pr = qp[i];
+                    const double sd = exact_score(x_rows, wr_rows, tile * kBM + pr.x, pr.y, H, lane);
+                    if (lane == 0) qs[i] = sd + (double)bs[pr.y];
+                }
+                epilogue_sync();
+                for (int i = 0; i < nq; ++i) {
+                    const int2 pr = qp[i];
+                    if (pr.x != r) continue;
+#pragma unroll
+                    for (int j = 0; j < KMAX; ++j)
+                        if (j < k && fe[j] == pr.y) {
+                            fx[j] = qs[i];
+                            has_x |= 1u << j;
+                        }
+                }
+            }
+            // sort the k by (score desc, index asc): exact scores where both
+            // have one, else approximate ones (more than 2 delta apart, so in
+            // the right order); every comparison gives the exact order
+#pragma unroll 1
+            for (int pass = 0; pass + 1 < KMAX; ++pass) {
+#pragma unroll
+                for (int j = 0; j + 1 < KMAX; ++j) {
+                    if (j + 1 < k) {
+                        const bool both = ((has_x >> j) & (has_x >> (j + 1)) & 1u) != 0;
+                        const bool swap = both ? (fx[j + 1] > fx[j] || (fx[j + 1] == fx[j] && fe[j + 1] < fe[j]))
+                                               : ranks_before(fa[j + 1], fe[j + 1], fa[j], fe[j]);
+                        if (swap) {
+                            const float ta = fa[j];
+                            fa[j] = fa[j + 1];
+                            fa[j + 1] = ta;
+                            const int tei = fe[j];
+                            fe[j] = fe[j + 1];
+                            fe[j + 1] = tei;
+                            const double tx = fx[j];
+                            fx[j] = fx[j + 1];
+                            fx[j + 1] = tx;
+                            const uint32_t bj = (has_x >> j) & 1u, bj1 = (has_x >> (j + 1)) & 1u;
+                            has_x = (has_x & ~(3u << j)) | (bj << (j + 1)) | (bj1 << j);
+                        }
+                    }
+                }
+            }
+            if (t < T) {
+                // softmax over the k selected; score differences taken in fp64
+                // where both scores are exact
+                double sj[KMAX];
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) sj[j] = ((has_x >> j) & 1u) ? fx[j] : (double)fa[j];
                 float z = 0.f;
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
-                    if (j < k) z += expf(fv[j] - m);
+                    if (j < k) z += expf((float)(sj[j] - sj[0]));
                 const float inv = 1.0f / z;
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
                     if (j < k) {
                         topk_idx[(int64_t)t * k + j] = fe[j] < E ? fe[j] : -1;
-                        topk_w[(int64_t)t * k + j] = expf(fv[j] - m) * inv;
+                        topk_w[(int64_t)t * k + j] = expf((float)(sj[j] - sj[0])) * inv;
                     }
             }
         }
@@ -502,8 +680,10 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     if (!make_map_bf16(&mx, x, p.H, p.T, 1, kBK, kBM) || !make_map_bf16(&mw, router_w, p.H, E, 1, kBK, Npad))
         return cudaErrorInvalidValue;
     const int stage_bytes = kABytes + Npad * kBK * 2;
-    // alignment slack + queue + barrier block (168 B used of 256) + bias
-    const size_t fixed = 1024 + (size_t)kQueue * 16 + 256 + sizeof(float) * ((E + 63) / 64 * 64);
+    // alignment slack + queue (pairs, exact and approximate scores) + barrier
+    // block (204 B used of 256) + squared x norms [2][128] + bias
+    const size_t fixed = 1024 + (size_t)kQueue * 20 + 256 + sizeof(float) * 2 * kBM +
+                         sizeof(float) * ((E + 63) / 64 * 64);
     int stages = (int)((227 * 1024 - fixed) / stage_bytes);
     stages = stages > kMaxStages ? kMaxStages : stages;
     const size_t smem = (size_t)stages * stage_bytes + fixed;
