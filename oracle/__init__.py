@@ -12,7 +12,8 @@ experts (+ the always-on shared expert).  Router statistics for the
 load-balance penalties: per-expert importance (sum over tokens of the softmax
 over all E scores) and the penalties built from it and the top-k counts.
 Expert weights in the MXFP4 microscaling format: dequantization from the
-format's definition and the layer on those weights.
+format's definition and the layer on those weights.  The backward pass:
+every gradient of the layer by the chain rule through those steps.
 
 Parity pins of every function here live in ``tests/test_oracle.py``.
 """
@@ -52,7 +53,8 @@ def _L():
         _lib.oracle_permute.argtypes = [i64, i32, i32, i64, P, P, P, P, P, P]
         _lib.oracle_moe_tokens.argtypes = [i64, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P,
                                            P, P, P, i64, P, P]
-        for f in (_lib.oracle_route, _lib.oracle_permute, _lib.oracle_moe_tokens):
+        _lib.oracle_moe_backward.argtypes = [i64, i32, i32, i32, i32, i32, i32] + [P] * 21
+        for f in (_lib.oracle_route, _lib.oracle_permute, _lib.oracle_moe_tokens, _lib.oracle_moe_backward):
             f.restype = ctypes.c_int
         _lib.oracle_threads.argtypes = []
         _lib.oracle_threads.restype = ctypes.c_int
@@ -189,6 +191,37 @@ def expert_rows(x, w_gate, w_up, w_down, tokens, experts, dtype: str) -> np.ndar
     xs = np.ascontiguousarray(np.asarray(x)[tokens])
     e = np.asarray(experts, np.int32).reshape(-1, 1)
     return moe_tokens(xs, w_gate, w_up, w_down, e, np.ones(e.shape), dtype)
+
+
+def moe_backward(x, router_w, w_gate, w_up, w_down, topk_idx, topk_w, dy, dtype: str, row_of=None,
+                 ws_gate=None, ws_up=None, ws_down=None) -> dict:
+    """Gradients of the layer for upstream gradient dy [T, H] (fp64): dx,
+    d_router_w, d_router_b, d_w_gate, d_w_up, d_w_down (and d_ws_* with a
+    shared expert), by the chain rule through the forward's steps (see
+    oracle_moe_backward in moe_oracle.c)."""
+    x, router_w, w_gate, w_up, w_down = _c(x), _c(router_w), _c(w_gate), _c(w_up), _c(w_down)
+    ws_gate, ws_up, ws_down = _c(ws_gate), _c(ws_up), _c(ws_down)
+    topk_idx = _c(topk_idx, np.int32)
+    topk_w = _c(topk_w, np.float64)
+    row_of = _c(row_of, np.int32)
+    dy = _c(dy, np.float64)
+    T, H = x.shape
+    E, I, _ = w_gate.shape
+    k = topk_idx.shape[1]
+    Is = 0 if ws_gate is None else ws_gate.shape[0]
+    out = dict(dx=np.empty((T, H)), d_router_w=np.empty((E, H)), d_router_b=np.empty(E),
+               d_w_gate=np.empty((E, I, H)), d_w_up=np.empty((E, I, H)), d_w_down=np.empty((E, H, I)))
+    if Is:
+        out.update(d_ws_gate=np.empty((Is, H)), d_ws_up=np.empty((Is, H)), d_ws_down=np.empty((H, Is)))
+    rc = _L().oracle_moe_backward(T, H, I, E, k, Is, DTYPE_CODE[dtype], _ptr(x), _ptr(router_w), _ptr(w_gate),
+                                  _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down),
+                                  _ptr(topk_idx), _ptr(topk_w), _ptr(row_of), _ptr(dy), _ptr(out["dx"]),
+                                  _ptr(out["d_router_w"]), _ptr(out["d_router_b"]), _ptr(out["d_w_gate"]),
+                                  _ptr(out["d_w_up"]), _ptr(out["d_w_down"]), _ptr(out.get("d_ws_gate")),
+                                  _ptr(out.get("d_ws_up")), _ptr(out.get("d_ws_down")))
+    if rc != 0:
+        raise ValueError(f"oracle_moe_backward failed ({rc})")
+    return out
 
 
 def importance(logits) -> np.ndarray:

@@ -271,3 +271,232 @@ int oracle_moe_tokens(int64_t T, int H, int I, int E, int k, int Is, int dtype, 
     }
     return rc;
 }
+
+/*
+ * Backward pass of the layer, given the upstream gradient dy [T,H] (fp64),
+ * for the forward that oracle_route / oracle_permute / oracle_moe_tokens
+ * define (the training use of the grouped-GEMM backend, "Mixture of Experts
+ * (MoEs) in Transformers", section Training MoEs with Transformers).  Every
+ * formula is the chain rule through the forward's steps, in fp64 on the
+ * exact input values:
+ *   kept pair (t, j) with expert e, weight w:
+ *     g = W_gate[e] x, u = W_up[e] x, a = silu(g) * u, o = W_down[e] a
+ *     dw_j = dy . o                         (dropped pairs: dw_j = 0)
+ *     da = w * W_down[e]^T dy
+ *     dg = da * u * silu'(g),  silu'(z) = s(z) (1 + z (1 - s(z))), s = sigmoid
+ *     du = da * silu(g)
+ *     dW_down[e] += w * dy a^T,  dW_gate[e] += dg x^T,  dW_up[e] += du x^T
+ *     dx += W_gate[e]^T dg + W_up[e]^T du
+ *   softmax over the selected scores (every selected pair, kept or not):
+ *     dl_j = w_j (dw_j - sum_i w_i dw_i)
+ *     dW_router[e_j] += dl_j x,  db[e_j] += dl_j,  dx += dl_j W_router[e_j]
+ *   shared expert: the same with w = 1, always kept.
+ * The selection itself (top-k) and the capacity cut are piecewise constant:
+ * no gradient flows through them.
+ * Outputs (all fp64, written, not accumulated into): dx [T,H], d_router_w
+ * [E,H], d_router_b [E], d_w_gate, d_w_up [E,I,H], d_w_down [E,H,I] and,
+ * when Is > 0, d_ws_gate, d_ws_up [Is,H], d_ws_down [H,Is].
+ */
+int oracle_moe_backward(int64_t T, int H, int I, int E, int k, int Is, int dtype, const void* x,
+                        const void* router_w, const void* w_gate, const void* w_up, const void* w_down,
+                        const void* ws_gate, const void* ws_up, const void* ws_down, const int32_t* topk_idx,
+                        const double* topk_w, const int32_t* row_of, const double* dy, double* dx,
+                        double* d_router_w, double* d_router_b, double* d_w_gate, double* d_w_up,
+                        double* d_w_down, double* d_ws_gate, double* d_ws_up, double* d_ws_down) {
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || Is < 0) return -1;
+    if (Is > 0 && (!ws_gate || !ws_up || !ws_down || !d_ws_gate || !d_ws_up || !d_ws_down)) return -1;
+    const int64_t S = T * (int64_t)k;
+    /* per slot: a (activation), dg, du, and the token's dl */
+    double* A = (double*)calloc((size_t)S * I, sizeof(double));
+    double* DG = (double*)calloc((size_t)S * I, sizeof(double));
+    double* DU = (double*)calloc((size_t)S * I, sizeof(double));
+    double* DL = (double*)calloc((size_t)S, sizeof(double));
+    double* AS = Is > 0 ? (double*)calloc((size_t)T * Is, sizeof(double)) : NULL;
+    double* DGS = Is > 0 ? (double*)calloc((size_t)T * Is, sizeof(double)) : NULL;
+    double* DUS = Is > 0 ? (double*)calloc((size_t)T * Is, sizeof(double)) : NULL;
+    int rc = 0;
+    if (!A || !DG || !DU || !DL || (Is > 0 && (!AS || !DGS || !DUS))) rc = -2;
+    int imax = I > Is ? I : Is;
+    /* phase 1, per token: slot quantities, dl, and dx */
+    if (rc == 0) {
+#pragma omp parallel
+        {
+            double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+            double* g = (double*)malloc(sizeof(double) * (size_t)imax);
+            double* u = (double*)malloc(sizeof(double) * (size_t)imax);
+            double* dw = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+            double* col = (double*)malloc(sizeof(double) * (size_t)(H > imax ? H : imax));
+            if (!xr || !g || !u || !dw || !col) {
+#pragma omp atomic write
+                rc = -2;
+            }
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < T; ++t) {
+                if (!xr || !g || !u || !dw || !col) continue;
+                load_row(x, dtype, t * (int64_t)H, H, xr);
+                const double* dyt = dy + t * (int64_t)H;
+                double* dxt = dx + t * (int64_t)H;
+                for (int h = 0; h < H; ++h) dxt[h] = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    const int64_t s = t * k + j;
+                    dw[j] = 0.0;
+                    if (row_of && row_of[s] < 0) continue; /* dropped: no output, no gradient */
+                    const int64_t e = topk_idx[s];
+                    const double w = topk_w[s];
+                    double* a = A + s * (int64_t)I;
+                    for (int i = 0; i < I; ++i) {
+                        g[i] = dot_row(xr, w_gate, dtype, (e * I + i) * (int64_t)H, H);
+                        u[i] = dot_row(xr, w_up, dtype, (e * I + i) * (int64_t)H, H);
+                        a[i] = silu(g[i]) * u[i];
+                    }
+                    /* da' = W_down[e]^T dy (unweighted); dw = da' . a = dy . o */
+                    for (int i = 0; i < I; ++i) col[i] = 0.0;
+                    for (int h = 0; h < H; ++h) {
+                        for (int i = 0; i < I; ++i) {
+                            double v;
+                            load_row(w_down, dtype, (e * H + h) * (int64_t)I + i, 1, &v);
+                            col[i] += v * dyt[h];
+                        }
+                    }
+                    double d = 0.0;
+                    for (int i = 0; i < I; ++i) d += col[i] * a[i];
+                    dw[j] = d;
+                    double* dg = DG + s * (int64_t)I;
+                    double* du = DU + s * (int64_t)I;
+                    for (int i = 0; i < I; ++i) {
+                        const double da = w * col[i];
+                        const double sg = 1.0 / (1.0 + exp(-g[i]));
+                        dg[i] = da * u[i] * sg * (1.0 + g[i] * (1.0 - sg));
+                        du[i] = da * g[i] * sg;
+                    }
+                    for (int h = 0; h < H; ++h) {
+                        double acc = 0.0;
+                        for (int i = 0; i < I; ++i) {
+                            double vg, vu;
+                            load_row(w_gate, dtype, (e * I + i) * (int64_t)H + h, 1, &vg);
+                            load_row(w_up, dtype, (e * I + i) * (int64_t)H + h, 1, &vu);
+                            acc += vg * dg[i] + vu * du[i];
+                        }
+                        dxt[h] += acc;
+                    }
+                }
+                /* softmax over the selected scores */
+                double sw = 0.0;
+                for (int j = 0; j < k; ++j) sw += topk_w[t * k + j] * dw[j];
+                for (int j = 0; j < k; ++j) {
+                    const int64_t s = t * k + j;
+                    DL[s] = topk_w[s] * (dw[j] - sw);
+                    double* wr = col;
+                    load_row(router_w, dtype, (int64_t)topk_idx[s] * H, H, wr);
+                    for (int h = 0; h < H; ++h) dxt[h] += DL[s] * wr[h];
+                }
+                if (Is > 0) {
+                    double* as = AS + t * (int64_t)Is;
+                    double* dgs = DGS + t * (int64_t)Is;
+                    double* dus = DUS + t * (int64_t)Is;
+                    for (int i = 0; i < Is; ++i) {
+                        g[i] = dot_row(xr, ws_gate, dtype, (int64_t)i * H, H);
+                        u[i] = dot_row(xr, ws_up, dtype, (int64_t)i * H, H);
+                        as[i] = silu(g[i]) * u[i];
+                        double c = 0.0;
+                        for (int h = 0; h < H; ++h) {
+                            double v;
+                            load_row(ws_down, dtype, (int64_t)h * Is + i, 1, &v);
+                            c += v * dyt[h];
+                        }
+                        const double sg = 1.0 / (1.0 + exp(-g[i]));
+                        dgs[i] = c * u[i] * sg * (1.0 + g[i] * (1.0 - sg));
+                        dus[i] = c * g[i] * sg;
+                    }
+                    for (int h = 0; h < H; ++h) {
+                        double acc = 0.0;
+                        for (int i = 0; i < Is; ++i) {
+                            double vg, vu;
+                            load_row(ws_gate, dtype, (int64_t)i * H + h, 1, &vg);
+                            load_row(ws_up, dtype, (int64_t)i * H + h, 1, &vu);
+                            acc += vg * dgs[i] + vu * dus[i];
+                        }
+                        dxt[h] += acc;
+                    }
+                }
+            }
+            free(xr);
+            free(g);
+            free(u);
+            free(dw);
+            free(col);
+        }
+    }
+    /* phase 2, per expert: weight gradients (and the router's) */
+    if (rc == 0) {
+#pragma omp parallel
+        {
+            double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+            if (!xr) {
+#pragma omp atomic write
+                rc = -2;
+            }
+#pragma omp for schedule(dynamic, 1)
+            for (int e = 0; e < E; ++e) {
+                if (!xr) continue;
+                double* dWg = d_w_gate + (int64_t)e * I * H;
+                double* dWu = d_w_up + (int64_t)e * I * H;
+                double* dWd = d_w_down + (int64_t)e * H * I;
+                double* dWr = d_router_w + (int64_t)e * H;
+                for (int64_t q = 0; q < (int64_t)I * H; ++q) dWg[q] = dWu[q] = dWd[q] = 0.0;
+                for (int h = 0; h < H; ++h) dWr[h] = 0.0;
+                d_router_b[e] = 0.0;
+                for (int64_t t = 0; t < T; ++t)
+                    for (int j = 0; j < k; ++j) {
+                        const int64_t s = t * k + j;
+                        if (topk_idx[s] != e) continue;
+                        load_row(x, dtype, t * (int64_t)H, H, xr);
+                        for (int h = 0; h < H; ++h) dWr[h] += DL[s] * xr[h];
+                        d_router_b[e] += DL[s];
+                        if (row_of && row_of[s] < 0) continue;
+                        const double w = topk_w[s];
+                        const double* a = A + s * (int64_t)I;
+                        const double* dg = DG + s * (int64_t)I;
+                        const double* du = DU + s * (int64_t)I;
+                        const double* dyt = dy + t * (int64_t)H;
+                        for (int i = 0; i < I; ++i)
+                            for (int h = 0; h < H; ++h) {
+                                dWg[(int64_t)i * H + h] += dg[i] * xr[h];
+                                dWu[(int64_t)i * H + h] += du[i] * xr[h];
+                            }
+                        for (int h = 0; h < H; ++h)
+                            for (int i = 0; i < I; ++i) dWd[(int64_t)h * I + i] += w * dyt[h] * a[i];
+                    }
+            }
+            free(xr);
+        }
+        if (Is > 0) {
+            for (int64_t q = 0; q < (int64_t)Is * H; ++q) d_ws_gate[q] = d_ws_up[q] = d_ws_down[q] = 0.0;
+            double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+            if (!xr) rc = -2;
+            for (int64_t t = 0; t < T && xr; ++t) {
+                load_row(x, dtype, t * (int64_t)H, H, xr);
+                const double* as = AS + t * (int64_t)Is;
+                const double* dgs = DGS + t * (int64_t)Is;
+                const double* dus = DUS + t * (int64_t)Is;
+                const double* dyt = dy + t * (int64_t)H;
+                for (int i = 0; i < Is; ++i)
+                    for (int h = 0; h < H; ++h) {
+                        d_ws_gate[(int64_t)i * H + h] += dgs[i] * xr[h];
+                        d_ws_up[(int64_t)i * H + h] += dus[i] * xr[h];
+                    }
+                for (int h = 0; h < H; ++h)
+                    for (int i = 0; i < Is; ++i) d_ws_down[(int64_t)h * Is + i] += dyt[h] * as[i];
+            }
+            free(xr);
+        }
+    }
+    free(A);
+    free(DG);
+    free(DU);
+    free(DL);
+    free(AS);
+    free(DGS);
+    free(DUS);
+    return rc;
+}

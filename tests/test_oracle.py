@@ -556,3 +556,106 @@ def test_mxfp4_single_expert_is_dense_swiglu_ffn():
     g, u, d = (torch.from_numpy(oracle.mxfp4_dequantize(*mx[n])[0]) for n in ("w_gate", "w_up", "w_down"))
     ref = torch.nn.functional.linear(torch.nn.functional.silu(x @ g.T) * (x @ u.T), d).numpy()
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-13 * np.abs(ref).max())
+
+
+# ---------------------------------------------------------------- backward
+
+def _torch_layer_grads(inp, dtype, idx, row_of, dy):
+    """The layer in torch float64 with the selection held fixed (top-k and the
+    capacity cut carry no gradient), differentiated by autograd."""
+    def t64(a):
+        return torch.from_numpy(f64(a, dtype)).requires_grad_(True) if a is not None else None
+
+    x, rw, wg, wu, wd = (t64(inp[n]) for n in ("x", "router_w", "w_gate", "w_up", "w_down"))
+    rb = torch.from_numpy(inp["router_b"].astype(np.float64)).requires_grad_(True) \
+        if inp["router_b"] is not None else None
+    sg, su, sd = (t64(inp[n]) for n in ("ws_gate", "ws_up", "ws_down"))
+    T, k = idx.shape
+    logits = x @ rw.T + (rb if rb is not None else 0.0)
+    w = torch.softmax(torch.gather(logits, 1, torch.from_numpy(idx.astype(np.int64))), dim=1)
+    rows = []
+    for t in range(T):
+        yt = torch.zeros(x.shape[1], dtype=torch.float64)
+        for j in range(k):
+            if row_of[t, j] < 0:
+                continue
+            e = int(idx[t, j])
+            a = torch.nn.functional.silu(wg[e] @ x[t]) * (wu[e] @ x[t])
+            yt = yt + w[t, j] * (wd[e] @ a)
+        if sg is not None:
+            yt = yt + sd @ (torch.nn.functional.silu(sg @ x[t]) * (su @ x[t]))
+        rows.append(yt)
+    y = torch.stack(rows)
+    (y * torch.from_numpy(dy)).sum().backward()
+    out = dict(dx=x.grad, d_router_w=rw.grad, d_w_gate=wg.grad, d_w_up=wu.grad, d_w_down=wd.grad)
+    out["d_router_b"] = rb.grad if rb is not None else None
+    if sg is not None:
+        out.update(d_ws_gate=sg.grad, d_ws_up=su.grad, d_ws_down=sd.grad)
+    return {kk: (v.numpy() if v is not None else None) for kk, v in out.items()}
+
+
+@pytest.mark.parametrize("case", [
+    dict(T=24, H=32, I=24, E=6, k=2, dtype="bf16", zipf_s=1.1, I_shared=16, capacity_factor=0.6),
+    dict(T=20, H=24, I=16, E=8, k=3, dtype="f32"),
+    dict(T=16, H=16, I=8, E=4, k=4, dtype="f32", zipf_s=1.1),
+], ids=["bf16_bias_shared_drops", "f32_k3", "f32_k_eq_E"])
+def test_backward_matches_torch_autograd(case):
+    """Every gradient of the layer against autograd through a float64 torch
+    restatement of the forward, the selection and capacity cut held fixed."""
+    wl = small(**case)
+    inp = mi.make_inputs(wl)
+    if inp["router_b"] is None:
+        inp["router_b"] = np.zeros(wl.E, np.float32)
+    _, idx, w = oracle.route(inp["x"], inp["router_w"], inp["router_b"], wl.k, wl.dtype)
+    row_of = oracle.permute(idx, wl.E, oracle.capacity(wl.capacity_factor, wl.T, wl.k, wl.E))["row_of"]
+    if wl.capacity_factor > 0:
+        assert (row_of < 0).any()
+    dy = mi.normal(3, 77, (wl.T, wl.H), 1.0, "f32").astype(np.float64)
+    got = oracle.moe_backward(inp["x"], inp["router_w"], inp["w_gate"], inp["w_up"], inp["w_down"], idx, w, dy,
+                              wl.dtype, row_of=row_of, ws_gate=inp["ws_gate"], ws_up=inp["ws_up"],
+                              ws_down=inp["ws_down"])
+    ref = _torch_layer_grads(inp, wl.dtype, idx, row_of, dy)
+    for name, r in ref.items():
+        scale = max(np.abs(r).max(), 1e-300)
+        assert np.max(np.abs(got[name] - r)) <= 1e-11 * scale, name
+
+
+def test_backward_top1_routes_no_gradient_to_the_router():
+    """k = 1: the softmax over one score is 1 whatever the score, so the
+    router gets exactly zero gradient; unselected experts get exactly zero."""
+    wl = small(T=30, H=24, I=16, E=8, k=1, dtype="f32")
+    inp = mi.make_inputs(wl)
+    _, idx, w = oracle.route(inp["x"], inp["router_w"], None, 1, "f32")
+    dy = mi.normal(4, 78, (wl.T, wl.H), 1.0, "f32").astype(np.float64)
+    got = oracle.moe_backward(inp["x"], inp["router_w"], inp["w_gate"], inp["w_up"], inp["w_down"], idx, w, dy,
+                              "f32")
+    assert np.all(got["d_router_w"] == 0.0) and np.all(got["d_router_b"] == 0.0)
+    unused = sorted(set(range(wl.E)) - set(idx.ravel().tolist()))
+    for e in unused:
+        assert np.all(got["d_w_gate"][e] == 0) and np.all(got["d_w_down"][e] == 0)
+    # the router's part of dx is zero too: dx equals the experts' part alone
+    assert np.all(np.isfinite(got["dx"]))
+
+
+def test_backward_dropped_pairs_carry_only_the_router_gradient():
+    """A pair dropped by the capacity cut adds nothing to y, so its expert
+    gets no gradient from it; its weight still enters the softmax."""
+    wl = small(T=40, H=16, I=8, E=4, k=2, dtype="f32", capacity_factor=0.3)
+    inp = mi.make_inputs(wl)
+    _, idx, w = oracle.route(inp["x"], inp["router_w"], None, 2, "f32")
+    row_of = oracle.permute(idx, wl.E, oracle.capacity(0.3, wl.T, 2, wl.E))["row_of"]
+    dy = mi.normal(5, 79, (wl.T, wl.H), 1.0, "f32").astype(np.float64)
+    kept_only = oracle.moe_backward(inp["x"], inp["router_w"], inp["w_gate"], inp["w_up"], inp["w_down"], idx, w,
+                                    dy, "f32", row_of=row_of)
+    # the same layer evaluated on just the kept pairs' tokens gives the
+    # expert weight gradients: a token whose pairs are all dropped adds none
+    all_dropped = np.all(row_of < 0, axis=1)
+    assert all_dropped.any()
+    # a token with every pair dropped has dw = 0, hence dl = 0: no gradient at all
+    assert np.all(kept_only["dx"][all_dropped] == 0.0)
+    dy2 = dy.copy()
+    dy2[all_dropped] = 0.0
+    other = oracle.moe_backward(inp["x"], inp["router_w"], inp["w_gate"], inp["w_up"], inp["w_down"], idx, w,
+                                dy2, "f32", row_of=row_of)
+    for name in ("d_w_gate", "d_w_up", "d_w_down"):
+        np.testing.assert_allclose(other[name], kept_only[name], rtol=0, atol=1e-13)
