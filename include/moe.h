@@ -391,6 +391,41 @@ moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const voi
 moe_status_t moe_reduce_partials(const moe_config_t* cfg, const float* partials, int32_t n, void* y,
                                  moe_stream_t stream);
 
+/*
+ * moe_backward -- every gradient of the layer for an upstream gradient dy
+ * (the training use of the grouped-GEMM backend, "Mixture of Experts (MoEs)
+ * in Transformers", section Training MoEs with Transformers), bf16 layer.
+ * For a kept (token t, expert e) pair with weight w, g = W_gate[e] x,
+ * u = W_up[e] x, h = silu(g) u (bf16 as in the forward):
+ *   dW_down[e] += w dy h^T;  da = w W_down[e]^T dy;  dw = (W_down[e]^T dy) . h
+ *   dW_gate[e] += (da u silu'(g)) x^T;  dW_up[e] += (da silu(g)) x^T
+ *   dx += W_gate[e]^T (da u silu'(g)) + W_up[e]^T (da silu(g))
+ * and through the softmax over the selected scores (every selected pair; a
+ * pair the capacity dropped has dw = 0): dl_j = w_j (dw_j - sum_i w_i dw_i),
+ * d_router_w[e_j] += dl_j x, d_router_b[e_j] += dl_j, dx += dl_j router_w[e_j].
+ * The shared expert (I_shared > 0) is one more expert with w = 1.  The top-k
+ * selection and the capacity cut carry no gradient.
+ *   x, dy [T,H] bf16; topk_idx [T,top_k] int32 and topk_w [T,top_k] float32
+ *   as moe_route gave them for this forward; router_w and the expert weights
+ *   as in moe_forward.
+ *   -> float32, written (not accumulated into): dx [T,H], d_router_w [E,H],
+ *      d_router_b [E], d_w_gate, d_w_up [E,I,H], d_w_down [E,H,I], and with a
+ *      shared expert d_ws_gate, d_ws_up [I_shared,H], d_ws_down [H,I_shared]
+ *      (NULL otherwise).  Experts with no kept rows get exact zeros.
+ * The products run as tcgen05 grouped GEMMs: the weight gradients reduce
+ * over each expert's rows (operands read MN-major from shared memory), the
+ * input gradients use the weights in their other orientation without a
+ * copy.  ws: moe_backward_workspace_size(cfg) bytes.  Errors as moe_forward;
+ * the float32 layer is MOE_ERR_UNSUPPORTED.
+ */
+size_t moe_backward_workspace_size(const moe_config_t* cfg);
+moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* dy, const int32_t* topk_idx,
+                          const float* topk_w, const void* router_w, const void* w_gate, const void* w_up,
+                          const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down, float* dx,
+                          float* d_router_w, float* d_router_b, float* d_w_gate, float* d_w_up, float* d_w_down,
+                          float* d_ws_gate, float* d_ws_up, float* d_ws_down, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
 /* Waits for `stream`, then returns the device check flags (MOE_DEVFLAG_*)
  * accumulated in `ws` since the last call and clears them.  Returns
  * MOE_ERR_DEVICE_CHECK if any flag was set, MOE_OK otherwise. */

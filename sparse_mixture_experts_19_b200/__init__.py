@@ -63,6 +63,8 @@ _SIGS = {
     "moe_forward_expert_shard": ([ctypes.POINTER(moe_config_t), _P, _P, _P, ctypes.c_int32, ctypes.c_int32]
                                  + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_forward_mxfp4": ([ctypes.POINTER(moe_config_t)] + [_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_backward_workspace_size": ([ctypes.POINTER(moe_config_t)], ctypes.c_size_t),
+    "moe_backward": ([ctypes.POINTER(moe_config_t)] + [_P] * 20 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_reduce_partials": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_int32, _P, _P], ctypes.c_int),
     "moe_get_device_status": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_size_t, _P,
                                ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
@@ -283,6 +285,25 @@ def moe_forward_mxfp4(cfg, x, router_w, router_b, w_gate_blocks, w_gate_scales, 
                                     _ptr(w_gate_scales), _ptr(w_up_blocks), _ptr(w_up_scales), _ptr(w_down_blocks),
                                     _ptr(w_down_scales), _ptr(y), _ptr(topk_idx_out), _ptr(counts_out),
                                     _ptr(dropped_out), p, n, _stream(stream)))
+
+
+def moe_backward_workspace_size(cfg) -> int:
+    n = load().moe_backward_workspace_size(ctypes.byref(cfg))
+    if n == 0:
+        raise MoeError(1, load().moe_last_error().decode())
+    return n
+
+
+def moe_backward(cfg, x, dy, topk_idx, topk_w, router_w, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, dx,
+                 d_router_w, d_router_b, d_w_gate, d_w_up, d_w_down, d_ws_gate=None, d_ws_up=None, d_ws_down=None,
+                 ws=None, stream=None):
+    """Every gradient of the layer (float32 outputs, written) for upstream dy."""
+    p, n = _ws(ws)
+    _check(load().moe_backward(ctypes.byref(cfg), _ptr(x), _ptr(dy), _ptr(topk_idx), _ptr(topk_w), _ptr(router_w),
+                               _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down),
+                               _ptr(dx), _ptr(d_router_w), _ptr(d_router_b), _ptr(d_w_gate), _ptr(d_w_up),
+                               _ptr(d_w_down), _ptr(d_ws_gate), _ptr(d_ws_up), _ptr(d_ws_down), p, n,
+                               _stream(stream)))
 
 
 def moe_reduce_partials(cfg, partials, y, stream=None):

@@ -156,6 +156,15 @@ cudaError_t launch_shard_capacity_left(int64_t C, const int32_t* counts, int n_s
 void shard_capacity_left_host(int64_t C, const int32_t* counts, int n_shards, int shard, int E,
                               int32_t* capacity_left);
 
+// Backward pass (bf16): extra workspace after the forward plan's bytes, and
+// the whole pass (grouping of the given routing, then every gradient).
+size_t backward_workspace_bytes(const Plan& p);
+cudaError_t launch_backward(const Plan& p, void* bwd_ws, const void* x, const void* dy, const int32_t* idx,
+                            const float* topk_w, const void* router_w, const void* w_gate, const void* w_up,
+                            const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down,
+                            float* dx, float* d_router_w, float* d_router_b, float* d_w_gate, float* d_w_up,
+                            float* d_w_down, float* d_ws_gate, float* d_ws_up, float* d_ws_down, cudaStream_t st);
+
 // Kernel-trace hooks (moe_abi.cu): bracket one launch with events.
 void trace_before(const char* name, cudaStream_t st);
 void trace_after(cudaStream_t st);

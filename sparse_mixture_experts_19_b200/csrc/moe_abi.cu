@@ -620,6 +620,55 @@ moe_status_t moe_reduce_partials(const moe_config_t* cfg, const float* partials,
     return MOE_OK;
 }
 
+size_t moe_backward_workspace_size(const moe_config_t* cfg) {
+    if (check_config(cfg) != MOE_OK) return 0;
+    Plan p;
+    make_plan(cfg, nullptr, &p);
+    return p.bytes + backward_workspace_bytes(p);
+}
+
+moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* dy, const int32_t* topk_idx,
+                          const float* topk_w, const void* router_w, const void* w_gate, const void* w_up,
+                          const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down, float* dx,
+                          float* d_router_w, float* d_router_b, float* d_w_gate, float* d_w_up, float* d_w_down,
+                          float* d_ws_gate, float* d_ws_up, float* d_ws_down, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+    moe_status_t s = check_config(cfg);
+    if (s != MOE_OK) return s;
+    if (cfg->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "moe_backward takes the bf16 layer (MOE_BF16)");
+    Plan p;
+    make_plan(cfg, nullptr, &p);
+    const size_t need = p.bytes + backward_workspace_bytes(p);
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+    if ((uintptr_t)ws % kWsAlign) return fail(MOE_ERR_WORKSPACE, "workspace not %d-byte aligned", kWsAlign);
+    if (ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu (moe_backward_workspace_size)", ws_bytes,
+                    need);
+    make_plan(cfg, ws, &p);
+    if (p.T == 0) return MOE_OK;
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(dy);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    REQUIRE_PTR(router_w);
+    REQUIRE_PTR(w_gate);
+    REQUIRE_PTR(w_up);
+    REQUIRE_PTR(w_down);
+    REQUIRE_PTR(dx);
+    REQUIRE_PTR(d_router_w);
+    REQUIRE_PTR(d_router_b);
+    REQUIRE_PTR(d_w_gate);
+    REQUIRE_PTR(d_w_up);
+    REQUIRE_PTR(d_w_down);
+    if ((s = check_shared(p, ws_gate, ws_up, ws_down)) != MOE_OK) return s;
+    if ((s = check_shared(p, d_ws_gate, d_ws_up, d_ws_down)) != MOE_OK) return s;
+    CUDA_TRY(launch_backward(p, (char*)ws + p.bytes, x, dy, topk_idx, topk_w, router_w, w_gate, w_up, w_down, ws_gate,
+                             ws_up, ws_down, dx, d_router_w, d_router_b, d_w_gate, d_w_up, d_w_down, d_ws_gate,
+                             d_ws_up, d_ws_down, (cudaStream_t)stream),
+             "backward");
+    return MOE_OK;
+}
+
 moe_status_t moe_get_device_status(const moe_config_t* cfg, void* ws, size_t ws_bytes,
                                    moe_stream_t stream, int32_t* flags_out) {
     Plan p;

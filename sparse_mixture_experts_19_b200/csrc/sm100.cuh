@@ -289,6 +289,21 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t smem_addr) {
     return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major bf16 tile with the 128-byte
+// swizzle: each 128-byte row holds 64 consecutive M (or N) elements of one k;
+// 8 such rows form a 1024-byte atom; the next 8 k lie sbo bytes on (stride
+// byte offset) and the next 64 M (or N) elements lbo bytes on (leading byte
+// offset).  Advancing K by 16 elements adds 16 rows (2048 bytes) to the start.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;  // version
+    d |= (uint64_t)2u << 61;  // SWIZZLE_128B
+    return d;
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B (both K-major), f32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
     return (1u << 4)                          // D format f32
@@ -296,6 +311,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
            | (1u << 10)                       // B format bf16
            | ((uint32_t)(N >> 3) << 17)       // N / 8
            | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// The same with A and / or B MN-major (transpose bits 15 and 16).
+__host__ __device__ constexpr uint32_t idesc_bf16_major(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16(M, N) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 }
 
 // ------------------------------------------------------- CTA pairs
