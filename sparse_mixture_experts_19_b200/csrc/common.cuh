@@ -18,6 +18,7 @@ constexpr int kWsAlign = 256;
 constexpr int kGemmTileRows = 128;  // rows per tile of the tcgen05 grouped GEMMs
 constexpr int64_t kNoAllocMaxSlots = 1 << 20;  // T*k limit of moe_permute_noalloc
 constexpr int kDecodeMaxSlots = 8;             // T*k limit of the decode FFN kernels
+constexpr int kRouterMaxSplits = 8;            // reduction chunks of the tensor-core router
 
 // Everything the kernels of one call need, carved out of the caller's workspace.
 struct Plan {
@@ -46,6 +47,9 @@ struct Plan {
     void* xperm;          // [S, H] layer dtype: x rows in grouped order
     void* h;              // [S, I] + [T, Is] layer dtype: SwiGLU activations
     void* rows;           // [S + T, H] layer dtype: routing-weighted expert output rows
+    float* rt_part;       // tensor-core router: [splits, T, E] float32 partial scores
+    float* rt_xn2;        // [splits, T] squared norms of the x rows over each chunk
+    float* rt_wn2;        // [splits, E] squared norms of the router rows over each chunk
     double* dec_scores;   // decode layer (S <= kDecodeMaxSlots): [T, E] router scores
     unsigned int* dec_bar;  // decode layer: [2] grid-barrier arrival counters
     size_t bytes;         // total workspace bytes
@@ -80,6 +84,8 @@ cudaError_t launch_router_simt(const Plan& p, const void* x, const void* router_
 cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router_w,
                                 const float* router_b, int32_t* topk_idx, float* topk_w,
                                 cudaStream_t st);
+// Reduction chunks of the tensor-core router for hidden size H.
+void router_splits(int64_t H, int* ns, int* kchunk);
 // Router for few tokens: one CTA per token, exact fp64 scores.
 cudaError_t launch_router_decode(const Plan& p, const void* x, const void* router_w,
                                  const float* router_b, int32_t* topk_idx, float* topk_w,

@@ -134,6 +134,10 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->xperm = take(elt * p->S * p->H);
     p->h = take(elt * (p->S * p->I + p->T * p->Is));
     p->rows = take(elt * (p->S + (p->Is ? p->T : 0)) * p->H);
+    const bool tc_router = p->bf16 && p->T * p->E * p->H > kDecodeRouterMaxMacs;
+    p->rt_part = (float*)take(tc_router ? sizeof(float) * kRouterMaxSplits * p->T * p->E : 0);
+    p->rt_xn2 = (float*)take(tc_router ? sizeof(float) * kRouterMaxSplits * p->T : 0);
+    p->rt_wn2 = (float*)take(tc_router ? sizeof(float) * kRouterMaxSplits * p->E : 0);
     const bool dec = p->S <= kDecodeMaxSlots;
     p->dec_scores = (double*)take(dec ? sizeof(double) * p->T * p->E : 0);
     p->dec_bar = (unsigned int*)take(dec ? 2 * sizeof(unsigned int) : 0);
