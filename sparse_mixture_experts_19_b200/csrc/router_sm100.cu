@@ -63,7 +63,6 @@ constexpr int kMaxStages = 6;
 constexpr int kThreads = 192;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kMinChunk = 512;
-constexpr int kSelWarps = 8;  // tokens per block of the selection kernel
 
 // Sum of squares of the 64 bf16 values of one 128-byte row of a swizzled
 // shared-memory tile at shared address `row`; lane l reads its 16-byte
@@ -233,10 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1) router_partial_kernel(
     if (warp == 1) tmem_dealloc(tmem_base, acc_cols);
 }
 
-// Exact score x_t . W_r[e] (+ bias) in fp64 by one warp: bf16 products are
-// exact in float32, summed in fp64; every lane gets the result.
-__device__ __forceinline__ double exact_score(const bf16* x, const bf16* w, int64_t t, int e, int H, double b,
-                                              int lane) {
+// Exact score x_t . W_r[e] in fp64 by one warp (bf16 products are exact in
+// float32, summed in fp64); every lane gets the result.
+__device__ __forceinline__ double exact_score(const bf16* x, const bf16* w, int64_t t, int e, int H, int lane) {
     const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
     const uint4* wr = reinterpret_cast<const uint4*>(w + (int64_t)e * H);
     const int nch = H / 8;
@@ -264,265 +262,356 @@ __device__ __forceinline__ double exact_score(const bf16* x, const bf16* w, int6
     double sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    return sum + b;
+    return sum;
 }
 
 // (a, ea) ranks before (b, eb): larger score, then lower expert index.
-__device__ __forceinline__ bool before(double a, int ea, double b, int eb) { return a > b || (a == b && ea < eb); }
-
-// Warp-wide best (score desc, index asc) among the lanes' candidates.
-__device__ __forceinline__ void warp_best(double& v, int& e) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, v, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, e, o);
-        if (before(ov, oe, v, e)) {
-            v = ov;
-            e = oe;
-        }
-    }
+__device__ __forceinline__ bool ranks_before(float a, int ea, float b, int eb) {
+    return a > b || (a == b && ea < eb);
+}
+__device__ __forceinline__ bool ranks_before(double a, int ea, double b, int eb) {
+    return a > b || (a == b && ea < eb);
 }
 
-// One warp per token; lane l owns experts l, l + 32, ... (JE of them).
-template <int JE, int KMAX>
-__global__ void __launch_bounds__(32 * kSelWarps) router_select_kernel(
+constexpr int kSelThreads = 128;  // tokens per block of the selection kernel (a thread each)
+constexpr int kQueue = 512;       // exact-rescoring queue entries per block and round
+
+// Shared memory of the selection kernel: summed scores [128][E + 1] (the +1
+// spreads a column over the banks), then the rescoring queue.
+size_t select_smem_bytes(int E) {
+    return sizeof(float) * kSelThreads * (E + 1) + (size_t)kQueue * (8 + 8 + 4) + 64;
+}
+
+// One thread per token: its scores summed from the chunks' partials into
+// shared memory (float32, chunk order), then the selection of the one-pass
+// design: k (+1) rounds of "next best" over the row, the bound, the band
+// rescored exactly through a queue served by every warp of the block, the
+// exact order, the softmax over the k.
+template <int KMAX>
+__global__ void __launch_bounds__(kSelThreads) router_select_kernel(
     const float* __restrict__ part, const float* __restrict__ xn2, const float* __restrict__ wn2, int T, int H, int E,
     int k, int ns, float cH, const float* __restrict__ bias, const bf16* __restrict__ x,
     const bf16* __restrict__ wr, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     float* __restrict__ importance) {
+    constexpr bool kDense = (KMAX == kMaxTopK);
+    extern __shared__ __align__(16) uint8_t sm_raw[];
+    const int ld = E + 1;
+    float* sc = reinterpret_cast<float*>(sm_raw);                           // [128][E + 1]
+    int2* qp = reinterpret_cast<int2*>(sc + (size_t)kSelThreads * ld + 1);  // 8-byte aligned below
+    qp = reinterpret_cast<int2*>((reinterpret_cast<uintptr_t>(qp) + 15) & ~uintptr_t(15));
+    double* qs = reinterpret_cast<double*>(qp + kQueue);
+    float* qa = reinterpret_cast<float*>(qs + kQueue);
     __shared__ float wmax[kRouterMaxSplits];
-    __shared__ float imp[kMaxExperts];
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    __shared__ float bmax_s;
+    __shared__ int qn;
+    const int r = threadIdx.x, lane = r & 31, warp = r / 32;
+    const int t0 = blockIdx.x * kSelThreads;
+    const int rows = min(kSelThreads, T - t0);
     const float slack = 1.f + (float)H * 2.3841858e-7f;  // 1 + H 2^-22
-    if (threadIdx.x < ns) {
+    if (r < ns) {
         float m = 0.f;
-        for (int e = 0; e < E; ++e) m = fmaxf(m, wn2[threadIdx.x * E + e]);
-        wmax[threadIdx.x] = sqrtf(m * slack);
+        for (int e = 0; e < E; ++e) m = fmaxf(m, wn2[r * E + e]);
+        wmax[r] = sqrtf(m * slack);
     }
-    for (int e = threadIdx.x; e < kMaxExperts; e += blockDim.x) imp[e] = 0.f;
-    __syncthreads();
-    const int t = blockIdx.x * kSelWarps + warp;
-    if (t < T) {
-        // fp64 scores of this lane's experts
-        double s[JE];
-        double amag = 0.0;  // sum of |partials| (for the fp64 rounding term)
-#pragma unroll
-        for (int j = 0; j < JE; ++j) {
-            const int e = lane + 32 * j;
-            double acc = -INFINITY;
-            if (e < E) {
-                acc = bias ? (double)bias[e] : 0.0;
-                for (int c = 0; c < ns; ++c) {
-                    const double v = (double)part[((int64_t)c * T + t) * E + e];
-                    acc += v;
-                    amag += fabs(v);
-                }
-            }
-            s[j] = acc;
+    if (r == 32) {
+        float m = 0.f;
+        if (bias)
+            for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(bias[e]));
+        bmax_s = m;
+    }
+    // summed scores: the block's rows of each chunk are one contiguous run
+    for (int c = 0; c < ns; ++c) {
+        const float* src = part + ((int64_t)c * T + t0) * E;
+        for (int i = r; i < rows * E; i += kSelThreads) {
+            const int rr = i / E, e = i % E;
+            const float v = __ldg(src + i);
+            sc[rr * ld + e] = c == 0 ? v : sc[rr * ld + e] + v;
         }
-        float delta = 0.f;
-        for (int c = 0; c < ns; ++c) delta += cH * sqrtf(xn2[(int64_t)c * T + t] * slack) * wmax[c];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amag = fmax(amag, __shfl_xor_sync(0xffffffffu, amag, o));
-        const double del2 = 2.0 * (1.001 * (double)delta + 1e-14 * (amag + 1.0));
+    }
+    __syncthreads();
+    if (bias)
+        for (int i = r; i < rows * E; i += kSelThreads) sc[(i / E) * ld + i % E] += bias[i % E];
+    __syncthreads();
+    const int t = t0 + r;
+    const float* row = sc + r * ld;
+    // the bound on |approximate - exact score| for this token (file comment),
+    // with the float32 sums of the chunks and the bias counted in
+    float delta = 0.f, nsum = 0.f;
+    if (t < T)
+        for (int c = 0; c < ns; ++c) {
+            const float a = sqrtf(xn2[(int64_t)c * T + t] * slack) * wmax[c];
+            delta += cH * a;
+            nsum += a;
+        }
+    const float u24 = 5.9604645e-8f;
+    const float del2 = 2.f * 1.001f * (delta + (float)(ns + 1) * u24 * (nsum + bmax_s));
 
-        // the k (+1) best approximate scores, in rounds of warp arg-max
-        const int kk = k < E ? k + 1 : k;
-        double tv[KMAX + 1];
-        int te[KMAX + 1];
-        uint32_t taken = 0;  // bit j: expert lane + 32 j already picked
+    // pass 1: the k (+1) best approximate scores, picked in k (+1) rounds;
+    // round j takes the best score ranking after the pick of round j-1
+    float tv[KMAX + 1];
+    int te[KMAX + 1];
+    const int kk = k < E ? k + 1 : k;
+    float pv = INFINITY;
+    int pe = -1;
 #pragma unroll
-        for (int r = 0; r <= KMAX; ++r) {
-            double bv = -INFINITY;
-            int be = 0x7fffffff;
-            if (r < kk) {
+    for (int j = 0; j <= KMAX; ++j) {
+        // four running maxima (elements i % 4), merged at the end; each keeps
+        // the lower index on ties because it visits indices in ascending order
+        float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        int be[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+        if (j < kk && t < T) {
+            for (int e0 = 0; e0 < E; e0 += 4) {
 #pragma unroll
-                for (int j = 0; j < JE; ++j) {
-                    const int e = lane + 32 * j;
-                    if (e < E && !((taken >> j) & 1u) && before(s[j], e, bv, be)) {
-                        bv = s[j];
-                        be = e;
+                for (int i = 0; i < 4; ++i) {
+                    const int e = e0 + i;
+                    if (e < E) {
+                        const float cv = row[e];
+                        const bool after = (cv < pv) || (cv == pv && e > pe);
+                        if (after && cv > bv[i]) {
+                            bv[i] = cv;
+                            be[i] = e;
+                        }
                     }
                 }
-                warp_best(bv, be);
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
             }
-            tv[r] = bv;
-            te[r] = be;
-        }
-
-        // the k selected: approximate score fa, expert fe, exact score fx (bit j of has_x)
-        double fa[KMAX], fx[KMAX];
-        int fe[KMAX];
-        uint32_t has_x = 0;
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            fa[j] = tv[j];
-            fe[j] = te[j];
-            fx[j] = 0.0;
+            for (int c = 1; c < 4; ++c)
+                if (ranks_before(bv[c], be[c], bv[0], be[0])) {
+                    bv[0] = bv[c];
+                    be[0] = be[c];
+                }
+            pv = bv[0];
+            pe = be[0];
         }
-        double kth = 0.0, next = 0.0;
+        tv[j] = bv[0];
+        te[j] = be[0];
+    }
+
+    // certainty of the decision
+    float band_lo = 0.f, band_hi = 0.f;
+    bool uncertain = false;
+    int n_in = k;
+    if (!kDense && t < T && k < E) {
+        float kth = 0.f, next = 0.f;
 #pragma unroll
         for (int j = 0; j <= KMAX; ++j) {
             if (j == k - 1) kth = tv[j];
             if (j == k) next = tv[j];
         }
-        if (k < E && kth - next <= del2) {
-            // uncertain: rescore the band exactly and complete the selection
-            const double lo = kth - del2, hi = next + del2;
-            int n_in = 0;
+        if (kth - next <= del2) {
+            uncertain = true;
+            band_lo = kth - del2;
+            band_hi = next + del2;
+            n_in = 0;
 #pragma unroll
             for (int j = 0; j < KMAX; ++j)
-                if (j < k && tv[j] > hi) n_in = j + 1;
-            // exact scores of this lane's band experts (computed by the whole warp)
-            double ex[JE];
-            uint32_t band = 0;
+                if (j < k && tv[j] > band_hi) n_in = j + 1;
+        }
+    }
+    // band: the best `need` members by exact score (ties to the lower index)
+    const int need = k - n_in;
+    double bv[KMAX];
+    int be[KMAX];
+    float ba[KMAX];
 #pragma unroll
-            for (int j = 0; j < JE; ++j) {
-                const int e = lane + 32 * j;
-                ex[j] = -INFINITY;
-                const bool in = e < E && s[j] >= lo && s[j] <= hi;
-                uint32_t m = __ballot_sync(0xffffffffu, in);
-                if (in) band |= 1u << j;
-                while (m) {
-                    const int src = __ffs(m) - 1;
-                    m &= m - 1;
-                    const int eb = src + 32 * j;
-                    const double v = exact_score(x, wr, t, eb, H, bias ? (double)bias[eb] : 0.0, lane);
-                    if (lane == src) ex[j] = v;
+    for (int j = 0; j < KMAX; ++j) {
+        bv[j] = -INFINITY;
+        be[j] = 0x7fffffff;
+        ba[j] = -INFINITY;
+    }
+    int cursor = uncertain ? 0 : E;  // next expert this thread still has to scan
+    while (__syncthreads_or(cursor < E)) {
+        if (r == 0) qn = 0;
+        __syncthreads();
+        if (cursor < E) {
+            bool stop = false;
+            for (int e = cursor; e < E && !stop; ++e) {
+                const float sv = row[e];
+                if (sv >= band_lo && sv <= band_hi) {
+                    const int slot = atomicAdd(&qn, 1);
+                    if (slot < kQueue) {
+                        qp[slot] = make_int2(r, e);
+                        qa[slot] = sv;
+                    } else {
+                        stop = true;  // queue full: resume here next round
+                        cursor = e;
+                    }
                 }
             }
-            // the best (k - n_in) band members by exact score, ties to the lower index
-            uint32_t used = 0;
+            if (!stop) cursor = E;
+        }
+        __syncthreads();
+        const int nq = min(qn, kQueue);
+        for (int i = warp; i < nq; i += kSelThreads / 32) {
+            const int2 pr = qp[i];
+            const double sd = exact_score(x, wr, t0 + pr.x, pr.y, H, lane);
+            if (lane == 0) qs[i] = sd + (bias ? (double)bias[pr.y] : 0.0);
+        }
+        __syncthreads();
+        if (uncertain)
+            for (int i = 0; i < nq; ++i) {
+                const int2 pr = qp[i];
+                if (pr.x != r) continue;
+                double cv = qs[i];
+                int ce = pr.y;
+                float ca = qa[i];
 #pragma unroll
-            for (int r = 0; r < KMAX; ++r) {
-                if (r < k - n_in) {
-                    double bv = -INFINITY;
-                    int be = 0x7fffffff;
-                    double ba = 0.0;
-#pragma unroll
-                    for (int j = 0; j < JE; ++j) {
-                        const int e = lane + 32 * j;
-                        if (((band >> j) & 1u) && !((used >> j) & 1u) && before(ex[j], e, bv, be)) {
-                            bv = ex[j];
-                            be = e;
-                            ba = s[j];
-                        }
+                for (int j = 0; j < KMAX; ++j) {
+                    if (j < need && (cv > bv[j] || (cv == bv[j] && ce < be[j]))) {
+                        const double ov = bv[j];
+                        const int oe = be[j];
+                        const float oa = ba[j];
+                        bv[j] = cv;
+                        be[j] = ce;
+                        ba[j] = ca;
+                        cv = ov;
+                        ce = oe;
+                        ca = oa;
                     }
-                    double wv = bv;
-                    int we = be;
-                    warp_best(wv, we);
-                    // the winner's approximate score, from its lane
-                    const double wa = __shfl_sync(0xffffffffu, ba, we & 31);
-                    if (we == be) used |= 1u << (we >> 5);
-#pragma unroll
-                    for (int j = 0; j < KMAX; ++j)
-                        if (j == n_in + r) {
-                            fa[j] = wa;
-                            fe[j] = we;
-                            fx[j] = wv;
-                            has_x |= 1u << j;
-                        }
                 }
+            }
+    }
+    if (importance) {
+        // softmax over all E scores of the token, shifted by the largest
+        // (tv[0]); summed per expert over the block (shared memory is free
+        // again: every row's scores have been read), then added to global
+        __syncthreads();
+        float* imp = reinterpret_cast<float*>(qp);  // kQueue * 20 bytes >= E floats
+        for (int e = r; e < E; e += kSelThreads) imp[e] = 0.f;
+        __syncthreads();
+        if (t < T) {
+            const float m = tv[0];
+            float z = 0.f;
+            for (int e = 0; e < E; ++e) z += __expf(row[e] - m);
+            const float inv = 1.0f / z;
+            for (int i = 0; i < E; ++i) {
+                const int e = (i + lane) % E;  // lanes spread over experts
+                atomicAdd(&imp[e], __expf(row[e] - m) * inv);
             }
         }
-        // order: every selected expert with another selected one within 2
-        // delta (approximate scores) gets its exact score
-        uint32_t pending = 0;
+        __syncthreads();
+        for (int e = r; e < E; e += kSelThreads) atomicAdd(&importance[e], imp[e]);
+        __syncthreads();
+    }
+
+    // the k selected: approximate fa, expert fe, exact fx where known (has_x)
+    float fa[KMAX];
+    int fe[KMAX];
+    double fx[KMAX];
+    uint32_t has_x = 0;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        fa[j] = tv[j];
+        fe[j] = te[j];
+        fx[j] = 0.0;
+    }
+    if (!kDense && uncertain) {
+        // move the band picks to slots n_in..k-1 (predicated shifts keep
+        // every index static: registers, no stack)
+#pragma unroll
+        for (int sft = 0; sft < KMAX; ++sft)
+            if (sft < n_in) {
+#pragma unroll
+                for (int j = KMAX - 1; j > 0; --j) {
+                    bv[j] = bv[j - 1];
+                    be[j] = be[j - 1];
+                    ba[j] = ba[j - 1];
+                }
+            }
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (j >= n_in && j < k) {
+                fa[j] = ba[j];
+                fe[j] = be[j];
+                fx[j] = bv[j];
+                has_x |= 1u << j;
+            }
+    }
+    // order: every selected expert with another selected one within 2 delta
+    // needs its exact score
+    uint32_t pending = 0;
+    if (t < T) {
 #pragma unroll
         for (int i = 0; i < KMAX; ++i)
 #pragma unroll
             for (int j = i + 1; j < KMAX; ++j)
-                if (j < k && fabs(fa[i] - fa[j]) <= del2) pending |= (1u << i) | (1u << j);
+                if (j < k && fabsf(fa[i] - fa[j]) <= del2) pending |= (1u << i) | (1u << j);
         pending &= ~has_x;
+    }
+    while (__syncthreads_or(pending != 0)) {
+        if (r == 0) qn = 0;
+        __syncthreads();
 #pragma unroll
         for (int j = 0; j < KMAX; ++j)
             if ((pending >> j) & 1u) {
-                fx[j] = exact_score(x, wr, t, fe[j], H, bias ? (double)bias[fe[j]] : 0.0, lane);
-                has_x |= 1u << j;
-            }
-        // sort by (score desc, index asc): exact scores where both have one,
-        // else approximate ones (more than 2 delta apart, so in the right order)
-#pragma unroll 1
-        for (int pass = 0; pass + 1 < KMAX; ++pass) {
-#pragma unroll
-            for (int j = 0; j + 1 < KMAX; ++j) {
-                if (j + 1 < k) {
-                    const bool both = ((has_x >> j) & (has_x >> (j + 1)) & 1u) != 0;
-                    const bool swap = both ? before(fx[j + 1], fe[j + 1], fx[j], fe[j])
-                                           : before(fa[j + 1], fe[j + 1], fa[j], fe[j]);
-                    if (swap) {
-                        const double ta = fa[j];
-                        fa[j] = fa[j + 1];
-                        fa[j + 1] = ta;
-                        const double tx = fx[j];
-                        fx[j] = fx[j + 1];
-                        fx[j + 1] = tx;
-                        const int ti = fe[j];
-                        fe[j] = fe[j + 1];
-                        fe[j + 1] = ti;
-                        const uint32_t bj = (has_x >> j) & 1u, bj1 = (has_x >> (j + 1)) & 1u;
-                        has_x = (has_x & ~(3u << j)) | (bj << (j + 1)) | (bj1 << j);
-                    }
+                const int slot = atomicAdd(&qn, 1);
+                if (slot < kQueue) {
+                    qp[slot] = make_int2(r, fe[j]);
+                    pending &= ~(1u << j);
                 }
             }
-        }
-        if (lane == 0) {
-            double sj[KMAX];
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j) sj[j] = ((has_x >> j) & 1u) ? fx[j] : fa[j];
-            float z = 0.f;
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j)
-                if (j < k) z += expf((float)(sj[j] - sj[0]));
-            const float inv = 1.0f / z;
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j)
-                if (j < k) {
-                    topk_idx[(int64_t)t * k + j] = fe[j];
-                    topk_w[(int64_t)t * k + j] = expf((float)(sj[j] - sj[0])) * inv;
-                }
-        }
-        if (importance) {
-            // softmax over all E scores of the token, shifted by the largest
-            const double m = tv[0];
-            float z = 0.f;
-#pragma unroll
-            for (int j = 0; j < JE; ++j)
-                if (lane + 32 * j < E) z += expf((float)(s[j] - m));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-            const float inv = 1.0f / z;
-#pragma unroll
-            for (int j = 0; j < JE; ++j)
-                if (lane + 32 * j < E) atomicAdd(&imp[lane + 32 * j], expf((float)(s[j] - m)) * inv);
-        }
-    }
-    if (importance) {
         __syncthreads();
-        for (int e = threadIdx.x; e < E; e += blockDim.x) atomicAdd(&importance[e], imp[e]);
-    }
-}
-
-template <int KMAX>
-cudaError_t launch_select(int JE, const Plan& p, int ns, float cH, const void* x, const void* router_w,
-                          const float* router_b, int32_t* topk_idx, float* topk_w, cudaStream_t st) {
-    const dim3 grid((unsigned)((p.T + kSelWarps - 1) / kSelWarps));
-    const int T = (int)p.T, H = (int)p.H, E = (int)p.E, k = (int)p.k;
-#define SELECT_ARGS                                                                                              \
-    p.rt_part, p.rt_xn2, p.rt_wn2, T, H, E, k, ns, cH, router_b, (const bf16*)x, (const bf16*)router_w, topk_idx, \
-        topk_w, p.importance
-    if (KMAX > 8 || JE == 1) {
-        router_select_kernel<1, KMAX><<<grid, 32 * kSelWarps, 0, st>>>(SELECT_ARGS);
-    } else {
-        switch (JE) {
-            case 2: router_select_kernel<(KMAX > 8 ? 1 : 2), KMAX><<<grid, 32 * kSelWarps, 0, st>>>(SELECT_ARGS); break;
-            case 4: router_select_kernel<(KMAX > 8 ? 1 : 4), KMAX><<<grid, 32 * kSelWarps, 0, st>>>(SELECT_ARGS); break;
-            default: router_select_kernel<(KMAX > 8 ? 1 : 8), KMAX><<<grid, 32 * kSelWarps, 0, st>>>(SELECT_ARGS); break;
+        const int nq = min(qn, kQueue);
+        for (int i = warp; i < nq; i += kSelThreads / 32) {
+            const int2 pr = qp[i];
+            const double sd = exact_score(x, wr, t0 + pr.x, pr.y, H, lane);
+            if (lane == 0) qs[i] = sd + (bias ? (double)bias[pr.y] : 0.0);
+        }
+        __syncthreads();
+        for (int i = 0; i < nq; ++i) {
+            const int2 pr = qp[i];
+            if (pr.x != r) continue;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (j < k && fe[j] == pr.y) {
+                    fx[j] = qs[i];
+                    has_x |= 1u << j;
+                }
         }
     }
-#undef SELECT_ARGS
-    return cudaGetLastError();
+    // sort the k by (score desc, index asc): exact scores where both have
+    // one, else approximate ones (more than 2 delta apart, in the right order)
+#pragma unroll 1
+    for (int pass = 0; pass + 1 < KMAX; ++pass) {
+#pragma unroll
+        for (int j = 0; j + 1 < KMAX; ++j) {
+            if (j + 1 < k) {
+                const bool both = ((has_x >> j) & (has_x >> (j + 1)) & 1u) != 0;
+                const bool swap = both ? ranks_before(fx[j + 1], fe[j + 1], fx[j], fe[j])
+                                       : ranks_before(fa[j + 1], fe[j + 1], fa[j], fe[j]);
+                if (swap) {
+                    const float ta = fa[j];
+                    fa[j] = fa[j + 1];
+                    fa[j + 1] = ta;
+                    const int ti = fe[j];
+                    fe[j] = fe[j + 1];
+                    fe[j + 1] = ti;
+                    const double tx = fx[j];
+                    fx[j] = fx[j + 1];
+                    fx[j + 1] = tx;
+                    const uint32_t bj = (has_x >> j) & 1u, bj1 = (has_x >> (j + 1)) & 1u;
+                    has_x = (has_x & ~(3u << j)) | (bj << (j + 1)) | (bj1 << j);
+                }
+            }
+        }
+    }
+    if (t < T) {
+        // softmax over the k selected; differences in fp64 where both scores are exact
+        double sj[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) sj[j] = ((has_x >> j) & 1u) ? fx[j] : (double)fa[j];
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (j < k) z += expf((float)(sj[j] - sj[0]));
+        const float inv = 1.0f / z;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (j < k) {
+                topk_idx[(int64_t)t * k + j] = fe[j] < E ? fe[j] : -1;
+                topk_w[(int64_t)t * k + j] = expf((float)(sj[j] - sj[0])) * inv;
+            }
+    }
 }
 
 }  // namespace
@@ -566,12 +655,25 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // the bound's constant for the longest chunk: 4 MMA steps per 64 of reduction
     const float cH = 17.f * 1.1920929e-7f * (float)(4 * ((kchunk + kBK - 1) / kBK) + 1) * 1.01f;
-    const int JE = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
+    const size_t ssm = select_smem_bytes(E);
+    const dim3 sgrid((unsigned)((p.T + kSelThreads - 1) / kSelThreads));
     trace_before("router_select", st);
-    // top_k > 8 only as top_k == E <= 32: one expert per lane
-    e = p.k <= 8 ? launch_select<8>(JE, p, ns, cH, x, router_w, router_b, topk_idx, topk_w, st)
-                 : launch_select<kMaxTopK>(1, p, ns, cH, x, router_w, router_b, topk_idx, topk_w, st);
+    // top_k > 8 only as top_k == E <= 32
+    if (p.k <= 8) {
+        e = ensure_smem_attr(router_select_kernel<8>, ssm);
+        if (e == cudaSuccess)
+            router_select_kernel<8><<<sgrid, kSelThreads, ssm, st>>>(
+                p.rt_part, p.rt_xn2, p.rt_wn2, (int)p.T, (int)p.H, E, (int)p.k, ns, cH, router_b, (const bf16*)x,
+                (const bf16*)router_w, topk_idx, topk_w, p.importance);
+    } else {
+        e = ensure_smem_attr(router_select_kernel<kMaxTopK>, ssm);
+        if (e == cudaSuccess)
+            router_select_kernel<kMaxTopK><<<sgrid, kSelThreads, ssm, st>>>(
+                p.rt_part, p.rt_xn2, p.rt_wn2, (int)p.T, (int)p.H, E, (int)p.k, ns, cH, router_b, (const bf16*)x,
+                (const bf16*)router_w, topk_idx, topk_w, p.importance);
+    }
     trace_after(st);
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e;
 }
 
