@@ -18,6 +18,7 @@ constexpr int kWsAlign = 256;
 constexpr int kGemmTileRows = 128;  // rows per tile of the tcgen05 grouped GEMMs
 constexpr int64_t kNoAllocMaxSlots = 1 << 20;  // T*k limit of moe_permute_noalloc
 constexpr int kDecodeMaxSlots = 8;             // T*k limit of the decode FFN kernels
+constexpr int kDecodeCounters = 2 + kDecodeMaxSlots;  // decode layer: grid barrier + one per expert group
 constexpr int kRouterMaxSplits = 8;            // reduction chunks of the tensor-core router
 
 // Everything the kernels of one call need, carved out of the caller's workspace.
@@ -51,7 +52,7 @@ struct Plan {
     float* rt_xn2;        // [splits, T] squared norms of the x rows over each chunk
     float* rt_wn2;        // [splits, E] squared norms of the router rows over each chunk
     double* dec_scores;   // decode layer (S <= kDecodeMaxSlots): [T, E] router scores
-    unsigned int* dec_bar;  // decode layer: [2] grid-barrier arrival counters
+    unsigned int* dec_bar;  // decode layer: [kDecodeCounters] arrival counters
     size_t bytes;         // total workspace bytes
 };
 

@@ -11,30 +11,35 @@
 // all padding, so the layer is written as one read of the selected experts'
 // weight rows, spread evenly over every SM.  One CTA per SM (512 threads),
 // launched cooperatively so that all CTAs are resident and may wait for one
-// another; each grid-wide wait is bounded (about 2 s, then
-// MOE_DEVFLAG_WAIT_TIMEOUT is set and the CTA skips the rest).
+// another; each wait is bounded (about 2 s, then MOE_DEVFLAG_WAIT_TIMEOUT is
+// set and the CTA skips the rest).
 //
 //   0. scores (when the routing is not given): the T*E router scores are
-//      split over the CTAs, one warp per (token, expert), exact up to fp64
-//      rounding (a product of two bf16 values is exact in float32, and the
-//      products are summed in fp64); grid barrier.
+//      split over the CTAs (a CTA with few pairs splits each pair's H over
+//      its warps), exact up to fp64 rounding (a product of two bf16 values
+//      is exact in float32, and the products are summed in fp64); grid
+//      barrier.
 //   1. selection: every CTA reads the T*E scores and picks each token's k
 //      best (score descending, ties to the lower index) with warp arg-max
 //      rounds, then the softmax of those k; the same arithmetic in every
 //      CTA gives every CTA the same plan: the slots grouped by expert, the
 //      capacity cut in token order, the shared expert as one more group.
-//   2. gate/up: CTA c owns the intermediate rows i in [R c / G, R (c+1) / G)
-//      of every group (R = I, or I_s for the shared expert); a warp takes
-//      one (group, i) at a time and streams its gate and up rows with
-//      16-byte loads (L2 evict-first), dotting them with the group's token
-//      vectors from shared memory: h[slot][i] = bf16(silu(x.g) * (x.u)).
-//      Meanwhile the CTA's rows of phase 3 are prefetched into L2.
-//      Grid barrier.
-//   3. down: CTA c owns the output columns j in [H c / G, H (c+1) / G) of
-//      every group; a warp takes one (group, j) at a time and dots the down
-//      row (from L2) with the group's h rows; the CTA then writes
-//      y[t][j] = bf16(sum over the token's slots in order of w * d, + the
-//      shared expert's d), so y is bit-reproducible without atomics.
+//   2. gate/up and down, overlapped.  Eleven warps stream gate/up rows:
+//      CTA c owns the intermediate rows i in [R c / G, R (c+1) / G) of
+//      every group (R = I, or I_s for the shared expert), group by group,
+//      each row's gate and up rows read with 16-byte loads (L2
+//      evict-first) and dotted with the group's token vectors from shared
+//      memory: h[slot][i] = bf16(silu(x.g) * (x.u)).  When the CTA's rows
+//      of a group are written, the CTA publishes the group (a per-group
+//      counter in global memory).  The other five warps take the down rows
+//      group by group: once every CTA has published group g, they copy its
+//      h rows into shared memory and dot them with the down rows of this
+//      CTA's output columns j in [H c / G, H (c+1) / G), while the gate/up
+//      warps stream the next groups.  So the down rows are read during the
+//      gate/up stream instead of after it, and no grid barrier separates
+//      the two.
+//   3. y[t][j] = bf16(sum over the token's slots in order of w * d, + the
+//      shared expert's d): y is bit-reproducible without atomics.
 #include <algorithm>
 
 #include "common.cuh"
@@ -53,6 +58,16 @@ constexpr int kDlBatch = 4;                        // token vectors per pass ove
 constexpr int kDlUnroll = 6;                       // 16-byte chunks per lane in flight, per row
 constexpr int kDlMaxCols = 64;                     // output columns per CTA in phase 3 (H <= 64 * grid)
 constexpr int kDlSmemMax = 200 * 1024;
+constexpr int kDlDownWarps = 5;                      // warps on the down rows (about a third of the bytes)
+constexpr int kDlUpWarps = kDlWarps - kDlDownWarps;  // warps on the gate/up rows
+
+// Bytes of one group's h vectors in shared memory: a routed expert meets a
+// token at most once, so a group has at most T vectors (the shared expert
+// exactly T).
+__host__ __device__ __forceinline__ int dl_hbytes(int T, int I, int Is) {
+    const int r = I > Is ? I : Is;
+    return (T * r * 2 + 15) / 16 * 16;
+}
 
 struct DlArgs {
     const bf16* x;
@@ -71,7 +86,7 @@ struct DlArgs {
     bool y_f32;
     bool drop_negative;    // expert -1 = another shard's: dropped, not counted
     double* scores;        // [T, E] router scores
-    unsigned int* bar;     // [2] grid-barrier counters, zero at launch
+    unsigned int* bar;     // [1 + groups]: the grid barrier, then each group's publishing CTAs; zero at launch
     int32_t* counts;
     int32_t* dropped;
     int32_t* flags;
@@ -126,12 +141,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
-__device__ __forceinline__ uint64_t policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 // 16-byte load of data read once: no L1 allocation, L2 policy `pol`.
 __device__ __forceinline__ uint4 ld_stream(const void* ptr, uint64_t pol) {
     uint4 v;
@@ -139,11 +148,6 @@ __device__ __forceinline__ uint4 ld_stream(const void* ptr, uint64_t pol) {
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
         : "l"(ptr), "l"(pol));
     return v;
-}
-
-__device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes, uint64_t pol) {
-    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(ptr), "r"(bytes), "l"(pol)
-                 : "memory");
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -334,11 +338,21 @@ __device__ __forceinline__ float f16_stage_scale(float m) {
     return ldexpf(1.f, 8 - ex);
 }
 
-// n bf16 values at src -> f16 values * sc at dst (shared memory), all threads.
-__device__ __forceinline__ void stage_f16(uint8_t* dst, const bf16* src, int n, float sc, bool l2_only) {
+// Barrier of `n` threads of the CTA (named barrier `id`; id 0 = all threads).
+__device__ __forceinline__ void named_sync(int id, int n) {
+    if (id == 0)
+        __syncthreads();
+    else
+        asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// n bf16 values at src -> f16 values * sc at dst (shared memory), by the
+// nthr threads numbered tid = 0 .. nthr-1.
+__device__ __forceinline__ void stage_f16(uint8_t* dst, const bf16* src, int n, float sc, bool l2_only, int tid,
+                                          int nthr) {
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
-    for (int i = threadIdx.x; i < n / 8; i += kDlThreads) {
+    for (int i = tid; i < n / 8; i += nthr) {
         const uint4 v = l2_only ? __ldcg(s4 + i) : __ldg(s4 + i);
         const uint32_t in[4] = {v.x, v.y, v.z, v.w};
         uint32_t out[4];
@@ -352,11 +366,13 @@ __device__ __forceinline__ void stage_f16(uint8_t* dst, const bf16* src, int n, 
     }
 }
 
-// Largest magnitude of n bf16 values (block-wide; every thread gets it).
-__device__ float block_absmax(const bf16* src, int n, bool l2_only, float* red) {
+// Largest magnitude of n bf16 values, by the nthr threads (whole warps)
+// numbered tid = 0 .. nthr-1 that meet at named barrier `bar`; every one of
+// them gets it.
+__device__ float group_absmax(const bf16* src, int n, bool l2_only, float* red, int tid, int nthr, int bar) {
     float m = 0.f;
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
-    for (int i = threadIdx.x; i < n / 8; i += kDlThreads) {
+    for (int i = tid; i < n / 8; i += nthr) {
         const uint4 v = l2_only ? __ldcg(s4 + i) : __ldg(s4 + i);
         const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -367,28 +383,28 @@ __device__ float block_absmax(const bf16* src, int n, bool l2_only, float* red) 
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = m;
-    __syncthreads();
+    named_sync(bar, nthr);
+    if ((tid & 31) == 0) red[tid / 32] = m;
+    named_sync(bar, nthr);
     float r = 0.f;
-    for (int w = 0; w < kDlWarps; ++w) r = fmaxf(r, red[w]);
+    for (int w = 0; w < nthr / 32; ++w) r = fmaxf(r, red[w]);
     return r;
 }
 
-// Exact score x[t] . W_r[e] in fp64 by one warp (every lane gets it).
-__device__ __forceinline__ double exact_dot(const bf16* x, const bf16* w, int H) {
+// Part of an exact score x[t] . W_r[e] in fp64: the 16-byte chunks
+// [cb, ce) of the two rows, summed by one warp (every lane gets the sum).
+__device__ __forceinline__ double exact_dot_part(const bf16* x, const bf16* w, int cb, int ce) {
     const int lane = threadIdx.x & 31;
     const uint4* xr = reinterpret_cast<const uint4*>(x);
     const uint4* wr = reinterpret_cast<const uint4*>(w);
-    const int nch = H / 8;
     double acc[2] = {0.0, 0.0};
-    for (int c0 = lane; c0 < nch; c0 += 32 * kDlUnroll) {
+    for (int c0 = cb + lane; c0 < ce; c0 += 32 * kDlUnroll) {
         uint4 a[kDlUnroll], b[kDlUnroll];
 #pragma unroll
         for (int u = 0; u < kDlUnroll; ++u) {
             const int c = c0 + 32 * u;
-            a[u] = c < nch ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
-            b[u] = c < nch ? __ldg(wr + c) : make_uint4(0, 0, 0, 0);
+            a[u] = c < ce ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+            b[u] = c < ce ? __ldg(wr + c) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < kDlUnroll; ++u) {
@@ -451,25 +467,61 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
     extern __shared__ __align__(128) uint8_t dsm[];
     __shared__ DlPlan pl;
     __shared__ int ok_s;
-    __shared__ float red[kDlWarps];
-    __shared__ float inv_sc[kDecodeMaxSlots];  // MXFP4: 1 / staging scale of each token or h vector
+    __shared__ float red[2 * kDlWarps];        // block reductions (the down warps use the second half)
+    __shared__ float inv_sx[kDecodeMaxSlots];  // MXFP4: 1 / staging scale of each token vector
+    __shared__ float inv_sh[kDecodeMaxSlots];  // MXFP4: 1 / staging scale of each h vector
+    __shared__ double dpart[kDlWarps];         // parts of the router scores
+    __shared__ int up_done[kDlMaxGroups];      // gate/up warps done with each group
+    __shared__ int down_ok;
+    __shared__ int last_state;  // the last group's h rows: 0 not yet staged, 1 staged, 2 abandoned
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int G = gridDim.x, c = blockIdx.x;
     const uint64_t pol_first = policy_evict_first();
 
     // ---------------------------------------------------------- routing
     if (!a.idx_in) {
-        const int P = a.T * a.E;
+        const int P = a.T * a.E, nch = a.H / 8;
+        // CTA c scores the pairs p0 .. p1-1 (p = t E + e).  With at most one
+        // pair per warp, each pair's H is split over kDlWarps / n warps and
+        // their parts are added in slice order, so a score costs one pass
+        // of its rows' loads instead of H / (32 * unroll) passes.
         const int p0 = (int)((int64_t)P * c / G), p1 = (int)((int64_t)P * (c + 1) / G);
-        for (int p = p0 + warp; p < p1; p += kDlWarps) {
-            const int t = p / a.E, e = p % a.E;
-            const double s = exact_dot(a.x + (int64_t)t * a.H, a.router_w + (int64_t)e * a.H, a.H);
-            if (lane == 0) a.scores[p] = s + (a.router_b ? (double)a.router_b[e] : 0.0);
+        const int nd = p1 - p0;
+        if (nd > 0 && nd <= kDlWarps) {
+            const int spd = kDlWarps / nd;  // warps (slices) per pair
+            const int di = warp / spd, si = warp % spd;
+            if (di < nd) {
+                const int p = p0 + di, t = p / a.E, e = p % a.E;
+                const double s = exact_dot_part(a.x + (int64_t)t * a.H, a.router_w + (int64_t)e * a.H,
+                                                (int)((int64_t)nch * si / spd), (int)((int64_t)nch * (si + 1) / spd));
+                if (lane == 0) dpart[di * spd + si] = s;
+            }
+            __syncthreads();
+            if (threadIdx.x < nd) {
+                const int p = p0 + threadIdx.x;
+                double s = 0.0;
+                for (int q = 0; q < spd; ++q) s += dpart[threadIdx.x * spd + q];
+                a.scores[p] = s + (a.router_b ? (double)a.router_b[p % a.E] : 0.0);
+            }
+        } else {
+            for (int p = p0 + warp; p < p1; p += kDlWarps) {
+                const int t = p / a.E, e = p % a.E;
+                const double s = exact_dot_part(a.x + (int64_t)t * a.H, a.router_w + (int64_t)e * a.H, 0, nch);
+                if (lane == 0) a.scores[p] = s + (a.router_b ? (double)a.router_b[e] : 0.0);
+            }
         }
         if (!grid_barrier(&a.bar[0], a.flags, &ok_s)) return;
-        // warp t selects token t: k rounds of warp arg-max, ties to the lower index
+        // warp t selects token t: its E scores read once (lane l holds
+        // experts l, l + 32, ...), then k rounds of warp arg-max, ties to the
+        // lower index
         for (int t = warp; t < a.T; t += kDlWarps) {
             const double* sc = a.scores + (int64_t)t * a.E;
+            double sv[kMaxExperts / 32];
+#pragma unroll
+            for (int i = 0; i < kMaxExperts / 32; ++i) {
+                const int e = lane + 32 * i;
+                sv[i] = e < a.E ? __ldcg(sc + e) : 0.0;
+            }
             double pv = INFINITY;
             int pe = -1;
             double v0 = 0.0;
@@ -477,10 +529,12 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
             for (int j = 0; j < a.k; ++j) {
                 double bv = -INFINITY;
                 int be = 0x7fffffff;
-                for (int e = lane; e < a.E; e += 32) {
-                    const double v = __ldcg(sc + e);
+#pragma unroll
+                for (int i = 0; i < kMaxExperts / 32; ++i) {
+                    const int e = lane + 32 * i;
+                    const double v = sv[i];
                     const bool after = (v < pv) || (v == pv && e > pe);
-                    if (after && (v > bv || (v == bv && e < be))) {
+                    if (e < a.E && after && (v > bv || (v == bv && e < be))) {
                         bv = v;
                         be = e;
                     }
@@ -540,166 +594,224 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
         return;
     }
 
-    // ---------------------------------------------------------- gate/up
-    // this CTA's output columns of phase 3, and their down rows into L2
+    // ------------------------------------------- gate/up and down, overlapped
+    // Shared memory: the token vectors x [T][H] (bf16, or f16 scaled for
+    // MXFP4), one group's h vectors [n][R], the partial dots [cols][S + T].
     const int j0 = (int)((int64_t)a.H * c / G), j1 = (int)((int64_t)a.H * (c + 1) / G);
-    if (threadIdx.x == 0 && j1 > j0) {
-        const uint64_t pol_last = policy_evict_last();
-        for (int g = 0; g < ng; ++g) {
-            const bool sh = pl.gexp[g] == a.E;
-            const int R = sh ? a.Is : a.I;
-            const void* base = kMx ? (const void*)(a.mdb + ((int64_t)pl.gexp[g] * a.H + j0) * (R / 2))
-                                   : (const void*)(sh ? a.wsd + (int64_t)j0 * R
-                                                      : a.wd + ((int64_t)pl.gexp[g] * a.H + j0) * R);
-            const int64_t bytes = (int64_t)(j1 - j0) * R * 2 / (kMx ? 4 : 1);
-            for (int64_t off = 0; off < bytes; off += 32768)
-                prefetch_l2(reinterpret_cast<const uint8_t*>(base) + off, (uint32_t)std::min<int64_t>(32768, bytes - off),
-                            pol_last);
-        }
-    }
-    // the token vectors in shared memory: x rows [T][H]
+    const int cols = j1 - j0;  // this CTA's output columns
+    const int P = a.S + a.T;   // partial columns: routed slots, then shared rows
     const uint32_t xs = smem_u32(dsm);
+    const int xbytes = (a.T * a.H * 2 + 15) / 16 * 16;
+    const uint32_t hsm = xs + (uint32_t)xbytes;
+    float* part = reinterpret_cast<float*>(dsm + xbytes + dl_hbytes(a.T, a.I, a.Is));  // [cols][P]
     if (kMx) {
         // f16 copies of the token rows, each scaled by a power of two
         for (int t = 0; t < a.T; ++t) {
-            const float sc = f16_stage_scale(block_absmax(a.x + (int64_t)t * a.H, a.H, false, red));
-            if (threadIdx.x == 0) inv_sc[t] = 1.f / sc;
-            stage_f16(dsm + (int64_t)t * a.H * 2, a.x + (int64_t)t * a.H, a.H, sc, false);
+            const float sc = f16_stage_scale(group_absmax(a.x + (int64_t)t * a.H, a.H, false, red, threadIdx.x,
+                                                          kDlThreads, 0));
+            if (threadIdx.x == 0) inv_sx[t] = 1.f / sc;
+            stage_f16(dsm + (int64_t)t * a.H * 2, a.x + (int64_t)t * a.H, a.H, sc, false, threadIdx.x, kDlThreads);
         }
     } else {
         const uint4* src = reinterpret_cast<const uint4*>(a.x);
         uint4* dst = reinterpret_cast<uint4*>(dsm);
         for (int i = threadIdx.x; i < a.T * a.H / 8; i += kDlThreads) dst[i] = __ldg(src + i);
     }
+    if (threadIdx.x < kDlMaxGroups) up_done[threadIdx.x] = 0;
+    if (threadIdx.x == 0) {
+        down_ok = 1;
+        last_state = 0;
+    }
     __syncthreads();
-    {
-        // items (g, i): this CTA's rows i of every group, group-major
-        int pre[kDlMaxGroups + 1];
-        pre[0] = 0;
-        for (int g = 0; g < ng; ++g) {
-            const int R = pl.gexp[g] == a.E ? a.Is : a.I;
-            pre[g + 1] = pre[g] + (int)((int64_t)R * (c + 1) / G - (int64_t)R * c / G);
-        }
-        const int K8 = a.H / 8;
-        int g = 0;
-        for (int q = warp; q < pre[ng]; q += kDlWarps) {
-            while (q >= pre[g + 1]) ++g;
-            const bool sh = pl.gexp[g] == a.E;
-            const int R = sh ? a.Is : a.I;
-            const int i = (int)((int64_t)R * c / G) + (q - pre[g]);
-            const int64_t row = sh ? (int64_t)i : (int64_t)pl.gexp[g] * a.I + i;
-            const uint4* rows[2];
-            const uint8_t* scl[2] = {nullptr, nullptr};
-            if (kMx) {
-                rows[0] = reinterpret_cast<const uint4*>(a.mgb + row * (a.H / 2));
-                rows[1] = reinterpret_cast<const uint4*>(a.mub + row * (a.H / 2));
-                scl[0] = a.mgs + row * (a.H / 32);
-                scl[1] = a.mus + row * (a.H / 32);
-            } else {
-                rows[0] = reinterpret_cast<const uint4*>((sh ? a.wsg : a.wg) + row * a.H);
-                rows[1] = reinterpret_cast<const uint4*>((sh ? a.wsu : a.wu) + row * a.H);
+    unsigned int* gdone = a.bar + 1;  // [group]: CTAs whose h rows of the group are written
+    const uint64_t pol_dn = policy_evict_first();
+    // Down items of group g (its h rows staged at hsm): column pairs q =
+    // first, first + step, ... of this CTA's columns.  A warp takes two
+    // adjacent columns at a time (bf16 rows): their down rows share the
+    // group's h vectors, and twice the loads are in flight per pass.
+    constexpr int kCols = kMx ? 1 : 2;
+    const int cp = (cols + kCols - 1) / kCols;
+    auto down_items = [&](int g, int first, int step) {
+        const bool sh = pl.gexp[g] == a.E;
+        const int R = sh ? a.Is : a.I;
+        for (int q = first; q < cp; q += step) {
+            const int jl = kCols * q;
+            const bool two = kCols == 2 && jl + 1 < cols;
+            const uint4* rows[kCols];
+            const uint8_t* scl[kCols];
+#pragma unroll
+            for (int r = 0; r < kCols; ++r) {
+                const int j = j0 + jl + (two ? r : 0);
+                const int64_t drow = (int64_t)pl.gexp[g] * a.H + j;
+                rows[r] = kMx ? reinterpret_cast<const uint4*>(a.mdb + drow * (R / 2))
+                              : reinterpret_cast<const uint4*>(sh ? a.wsd + (int64_t)j * R : a.wd + drow * R);
+                scl[r] = kMx ? a.mds + drow * (R / 32) : nullptr;
             }
             for (int b = 0; b < pl.gcnt[g]; b += kDlBatch) {
                 const int nv = min(kDlBatch, pl.gcnt[g] - b);
                 uint32_t vec[kDlBatch];
 #pragma unroll
-                for (int n = 0; n < kDlBatch; ++n) {
-                    const int id = pl.gvec[g][b + min(n, nv - 1)];
-                    const int tok = sh ? id : id / a.k;
-                    vec[n] = xs + (uint32_t)(tok * a.H * 2);
-                }
-                float d[2][kDlBatch];
+                for (int n = 0; n < kDlBatch; ++n) vec[n] = hsm + (uint32_t)((b + min(n, nv - 1)) * R * 2);
+                float d[kCols][kDlBatch];
                 if (kMx)
-                    row_dots_mx_n<2>(rows, scl, a.H / 32, vec, nv, pol_first, d);
+                    row_dots_mx_n<kCols>(rows, scl, R / 32, vec, nv, pol_dn, d);
                 else
-                    row_dots_n<2>(rows, K8, vec, nv, pol_first, d);
+                    row_dots_n<kCols>(rows, R / 8, vec, nv, pol_dn, d);
 #pragma unroll
                 for (int n = 0; n < kDlBatch; ++n)
                     if (lane == n && n < nv) {
                         const int id = pl.gvec[g][b + n];
-                        if (kMx) {
-                            const float f = inv_sc[sh ? id : id / a.k];
-                            d[0][n] *= f;
-                            d[1][n] *= f;
-                        }
-                        const bf16 hv = __float2bfloat16_rn(silu_f32(d[0][n]) * d[1][n]);
-                        if (sh)
-                            a.hs[(int64_t)id * a.Is + i] = hv;
-                        else
-                            a.h[(int64_t)id * a.I + i] = hv;
+                        const int col = sh ? a.S + id : id;
+                        const float f = kMx ? inv_sh[id] : 1.f;
+                        part[jl * P + col] = d[0][n] * f;
+                        if (two) part[(jl + 1) * P + col] = d[kCols - 1][n] * f;
                     }
             }
         }
-    }
-    if (!grid_barrier(&a.bar[1], a.flags, &ok_s)) return;
+    };
 
-    // ---------------------------------------------------------- down
-    if (j1 <= j0) return;
-    // h rows of every group into shared memory (reusing the x area): group g,
-    // vector n at hoff[g] + n * R_g * 2
-    int hoff[kDlMaxGroups];
-    {
-        int off = 0;
-        for (int g = 0; g < ng; ++g) {
-            hoff[g] = off;
-            off += pl.gcnt[g] * (pl.gexp[g] == a.E ? a.Is : a.I) * 2;
-        }
+    if (warp < kDlUpWarps) {
+        // gate/up warps: this CTA's rows i in [R c / G, R (c+1) / G) of every
+        // group, group-major, dealt round-robin over the warps across group
+        // boundaries; a warp reports each group as done (the CTA's last warp
+        // to report publishes the group to the grid), so no warp waits.
+        const int K8 = a.H / 8;
+        int base = 0;  // index of the group's first item in the CTA's list
         for (int g = 0; g < ng; ++g) {
             const bool sh = pl.gexp[g] == a.E;
             const int R = sh ? a.Is : a.I;
+            const int i0 = (int)((int64_t)R * c / G), n_items = (int)((int64_t)R * (c + 1) / G) - i0;
+            int q = warp - base % kDlUpWarps;
+            if (q < 0) q += kDlUpWarps;
+            for (; q < n_items; q += kDlUpWarps) {
+                const int i = i0 + q;
+                const int64_t row = sh ? (int64_t)i : (int64_t)pl.gexp[g] * a.I + i;
+                const uint4* rows[2];
+                const uint8_t* scl[2] = {nullptr, nullptr};
+                if (kMx) {
+                    rows[0] = reinterpret_cast<const uint4*>(a.mgb + row * (a.H / 2));
+                    rows[1] = reinterpret_cast<const uint4*>(a.mub + row * (a.H / 2));
+                    scl[0] = a.mgs + row * (a.H / 32);
+                    scl[1] = a.mus + row * (a.H / 32);
+                } else {
+                    rows[0] = reinterpret_cast<const uint4*>((sh ? a.wsg : a.wg) + row * a.H);
+                    rows[1] = reinterpret_cast<const uint4*>((sh ? a.wsu : a.wu) + row * a.H);
+                }
+                for (int b = 0; b < pl.gcnt[g]; b += kDlBatch) {
+                    const int nv = min(kDlBatch, pl.gcnt[g] - b);
+                    uint32_t vec[kDlBatch];
+#pragma unroll
+                    for (int n = 0; n < kDlBatch; ++n) {
+                        const int id = pl.gvec[g][b + min(n, nv - 1)];
+                        const int tok = sh ? id : id / a.k;
+                        vec[n] = xs + (uint32_t)(tok * a.H * 2);
+                    }
+                    float d[2][kDlBatch];
+                    if (kMx)
+                        row_dots_mx_n<2>(rows, scl, a.H / 32, vec, nv, pol_first, d);
+                    else
+                        row_dots_n<2>(rows, K8, vec, nv, pol_first, d);
+#pragma unroll
+                    for (int n = 0; n < kDlBatch; ++n)
+                        if (lane == n && n < nv) {
+                            const int id = pl.gvec[g][b + n];
+                            if (kMx) {
+                                const float f = inv_sx[sh ? id : id / a.k];
+                                d[0][n] *= f;
+                                d[1][n] *= f;
+                            }
+                            const bf16 hv = __float2bfloat16_rn(silu_f32(d[0][n]) * d[1][n]);
+                            if (sh)
+                                a.hs[(int64_t)id * a.Is + i] = hv;
+                            else
+                                a.h[(int64_t)id * a.I + i] = hv;
+                        }
+                }
+            }
+            base += n_items;
+            // this warp's rows of group g are written: report; the last of
+            // the CTA's gate/up warps publishes the group
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();  // this warp's h rows, before its report
+                if (atomicAdd(&up_done[g], 1) == kDlUpWarps - 1) {
+                    __threadfence();  // every report seen, before the publication
+                    atomicAdd(&gdone[g], 1u);
+                }
+            }
+        }
+        // then the last group's down columns, with the down warps, once the
+        // down warps have staged its h rows (bounded wait)
+        if (cols > 0) {
+            int st = 0;
+            const uint64_t t0 = global_ns();
+            while ((st = *reinterpret_cast<volatile int*>(&last_state)) == 0) {
+                if (global_ns() - t0 > 2000000000ull) {
+                    if (lane == 0) atomicOr(a.flags, MOE_DEVFLAG_WAIT_TIMEOUT);
+                    break;
+                }
+                __nanosleep(128);
+            }
+            __syncwarp();
+            if (st == 1) down_items(ng - 1, warp, kDlWarps);
+        }
+    } else if (cols > 0) {
+        // down warps: group by group, once every CTA has published the
+        // group's h rows, those rows into shared memory and this CTA's
+        // columns j of the group's down rows dotted with them
+        const int dt = threadIdx.x - kDlUpWarps * 32, dw = warp - kDlUpWarps;
+        constexpr int kDn = kDlDownWarps * 32;
+        for (int g = 0; g < ng; ++g) {
+            const bool sh = pl.gexp[g] == a.E;
+            const int R = sh ? a.Is : a.I;
+            if (dt == 0) {
+                const uint64_t t0 = global_ns();
+                int ok = 1;
+                while (ld_acquire_u32(&gdone[g]) < (unsigned)G) {
+                    if (global_ns() - t0 > 2000000000ull) {
+                        atomicOr(a.flags, MOE_DEVFLAG_WAIT_TIMEOUT);
+                        ok = 0;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                __threadfence();
+                down_ok = ok;
+            }
+            named_sync(1, kDn);  // also: every down warp is done with group g-1's h
+            if (!down_ok) break;
             for (int n = 0; n < pl.gcnt[g]; ++n) {
                 const int id = pl.gvec[g][n];
                 const bf16* hrow = sh ? a.hs + (int64_t)id * R : a.h + (int64_t)id * R;
+                uint8_t* dst = dsm + xbytes + n * R * 2;
                 if (kMx) {
                     // routed groups only (no shared expert in this format): slot id
-                    const float sc = f16_stage_scale(block_absmax(hrow, R, true, red));
-                    if (threadIdx.x == 0) inv_sc[id] = 1.f / sc;
-                    stage_f16(dsm + hoff[g] + n * R * 2, hrow, R, sc, true);
+                    const float sc = f16_stage_scale(group_absmax(hrow, R, true, red + kDlWarps, dt, kDn, 1));
+                    if (dt == 0) inv_sh[id] = 1.f / sc;
+                    stage_f16(dst, hrow, R, sc, true, dt, kDn);
                 } else {
                     const uint4* src = reinterpret_cast<const uint4*>(hrow);
-                    uint4* dst = reinterpret_cast<uint4*>(dsm + hoff[g] + n * R * 2);
-                    for (int i = threadIdx.x; i < R / 8; i += kDlThreads) dst[i] = __ldcg(src + i);
+                    uint4* d4 = reinterpret_cast<uint4*>(dst);
+                    for (int i = dt; i < R / 8; i += kDn) d4[i] = __ldcg(src + i);
                 }
             }
-        }
-    }
-    const int cols = j1 - j0;
-    const int P = a.S + a.T;  // partial columns: routed slots, then shared rows
-    int hbytes = 0;
-    for (int g = 0; g < ng; ++g) hbytes += pl.gcnt[g] * (pl.gexp[g] == a.E ? a.Is : a.I) * 2;
-    float* part = reinterpret_cast<float*>(dsm + ((hbytes + 15) / 16) * 16);  // [cols][P]
-    __syncthreads();
-    {
-        const uint64_t pol_l2 = policy_evict_first();  // read once more, from L2
-        for (int q = warp; q < ng * cols; q += kDlWarps) {
-            const int g = q / cols, jl = q % cols, j = j0 + jl;
-            const bool sh = pl.gexp[g] == a.E;
-            const int R = sh ? a.Is : a.I;
-            const int64_t drow = (int64_t)pl.gexp[g] * a.H + j;
-            const uint4* rows[1] = {kMx ? reinterpret_cast<const uint4*>(a.mdb + drow * (R / 2))
-                                        : reinterpret_cast<const uint4*>(sh ? a.wsd + (int64_t)j * R
-                                                                            : a.wd + drow * R)};
-            const uint8_t* scl[1] = {kMx ? a.mds + drow * (R / 32) : nullptr};
-            for (int b = 0; b < pl.gcnt[g]; b += kDlBatch) {
-                const int nv = min(kDlBatch, pl.gcnt[g] - b);
-                uint32_t vec[kDlBatch];
-#pragma unroll
-                for (int n = 0; n < kDlBatch; ++n) vec[n] = xs + (uint32_t)(hoff[g] + (b + min(n, nv - 1)) * R * 2);
-                float d[1][kDlBatch];
-                if (kMx)
-                    row_dots_mx_n<1>(rows, scl, R / 32, vec, nv, pol_l2, d);
-                else
-                    row_dots_n<1>(rows, R / 8, vec, nv, pol_l2, d);
-#pragma unroll
-                for (int n = 0; n < kDlBatch; ++n)
-                    if (lane == n && n < nv) {
-                        const int id = pl.gvec[g][b + n];
-                        part[jl * P + (sh ? a.S + id : id)] = kMx ? d[0][n] * inv_sc[id] : d[0][n];
-                    }
+            named_sync(1, kDn);
+            if (g + 1 < ng) {
+                down_items(g, dw, kDlDownWarps);
+            } else {
+                // the last group: the gate/up warps are done with their rows
+                // and share its columns (all sixteen warps)
+                if (dt == 0) {
+                    __threadfence_block();
+                    *reinterpret_cast<volatile int*>(&last_state) = 1;
+                }
+                down_items(g, warp, kDlWarps);
             }
         }
+        if (dt == 0 && !down_ok) *reinterpret_cast<volatile int*>(&last_state) = 2;  // release the helpers
     }
     __syncthreads();
+    if (cols <= 0 || !down_ok) return;
     // y[t][j]: the token's kept slots in order, then the shared expert
     for (int q = threadIdx.x; q < a.T * cols; q += kDlThreads) {
         const int t = q / cols, jl = q % cols;
@@ -718,14 +830,12 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
     }
 }
 
-// Shared memory: the x rows in phase 2; the h rows of every group and the
-// partial dots [columns per CTA][S + T] in phase 3.
+// Shared memory: the x rows, one group's h rows, the partial dots
+// [columns per CTA][S + T].
 int64_t dl_smem_bytes(const Plan& p, int grid) {
-    const int64_t xb = p.T * p.H * 2;
-    const int64_t hb = (p.S * p.I + (p.Is ? p.T * p.Is : 0)) * 2;
+    const int64_t xb = (p.T * p.H * 2 + 15) / 16 * 16;
     const int64_t cols = (p.H + grid - 1) / grid;
-    const int64_t pb = (hb + 15) / 16 * 16 + cols * (p.S + p.T) * 4;
-    return std::max(xb, pb);
+    return xb + dl_hbytes((int)p.T, (int)p.I, (int)p.Is) + cols * (p.S + p.T) * 4;
 }
 
 }  // namespace
@@ -777,8 +887,8 @@ cudaError_t launch_typed(const Plan& p, const DlArgs& a, const char* name, cudaS
     const size_t smem = (size_t)dl_smem_bytes(p, grid);
     cudaError_t e = ensure_smem_attr(decode_layer_kernel<kMx>, kDlSmemMax);
     if (e != cudaSuccess) return e;
-    // the grid barriers count arrivals from zero
-    e = cudaMemsetAsync(p.dec_bar, 0, 2 * sizeof(unsigned int), st);
+    // the grid barrier and the group counters count arrivals from zero
+    e = cudaMemsetAsync(p.dec_bar, 0, kDecodeCounters * sizeof(unsigned int), st);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);

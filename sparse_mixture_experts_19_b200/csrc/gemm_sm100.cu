@@ -54,6 +54,8 @@ constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kIdesc = idesc_bf16(kBM, kBRows);
+constexpr int kSmallRows = 32;                   // A box rows of a group's short tile
+constexpr int kSmallABytes = kSmallRows * kBK * 2;
 
 struct GemmArgs {
     const int32_t* offsets;       // [E+2]
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
     const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
     const __grid_constant__ CUtensorMap tmBs0, const __grid_constant__ CUtensorMap tmBs1,
-    const GemmArgs a) {
+    const __grid_constant__ CUtensorMap tmAsm, const GemmArgs a) {
     constexpr int BN = kGateUp ? kBRows / 2 : kBRows;  // output columns per tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -350,7 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
             for (int64_t t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
                 TileInfo ti;
                 decode_tile(t, *tb, sc, a, BN, ti);
-                const CUtensorMap* mA = ti.shared ? &tmAs : &tmA;
+                // a group's last rows: a tile of at most kSmallRows rows loads
+                // only those (the MMA still covers 128 rows; the accumulator
+                // rows past ti.rows are never stored)
+                const bool small = !ti.shared && ti.rows <= kSmallRows;
+                const CUtensorMap* mA = ti.shared ? &tmAs : (small ? &tmAsm : &tmA);
+                const uint32_t stage_tx = small ? kStageBytes - kABytes + kSmallABytes : kStageBytes;
                 const CUtensorMap* mB0 = ti.shared ? &tmBs0 : &tmB0;
                 const CUtensorMap* mB1 = ti.shared ? &tmBs1 : &tmB1;
                 const int nkb = (ti.K + kBK - 1) / kBK;
@@ -360,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_sm100_kernel(
                     if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, a.flags)) break;
                     uint8_t* sa = smem + s * kStageBytes;
                     uint8_t* sb = sa + kABytes;
-                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    mbar_arrive_expect_tx(&full[s], stage_tx);
                     // every map is rank 3 (activations have depth 1): the load's
                     // dimensionality must match the map's rank
                     tma_load_3d(sa, mA, &full[s], kb * kBK, ti.arow, 0);
@@ -657,7 +664,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
 constexpr size_t kSmemBytes = kEpiStageOff + 4 * kEpiStageBytes + 1024;
 
 template <bool kGateUp>
-cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const GemmArgs& args,
+cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[7], const GemmArgs& args,
                            cudaStream_t st) {
     constexpr int BN = kGateUp ? kBRows / 2 : kBRows;
     cudaError_t e = ensure_smem_attr(grouped_gemm_sm100_kernel<kGateUp>, kSmemBytes);
@@ -667,14 +674,14 @@ cudaError_t launch_grouped(const Plan& p, const CUtensorMap (&maps)[6], const Ge
     const int64_t ub = ((p.S + kBM - 1) / kBM + p.E) * nb_r + ((p.T + kBM - 1) / kBM) * nb_s;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), ub));
     grouped_gemm_sm100_kernel<kGateUp><<<grid, kThreads, kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3],
-                                                                         maps[4], maps[5], args);
+                                                                         maps[4], maps[5], maps[6], args);
     return cudaGetLastError();
 }
 
 constexpr size_t kPSmemBytes = kPEpiStageOff + 4 * kEpiStageBytes + 1024;
 
 template <bool kGateUp>
-cudaError_t launch_grouped_pair(const Plan& p, const CUtensorMap (&maps)[6], const GemmArgs& args,
+cudaError_t launch_grouped_pair(const Plan& p, const CUtensorMap (&maps)[7], const GemmArgs& args,
                                 cudaStream_t st) {
     constexpr int BN = kGateUp ? kBRows / 2 : kBRows;
     cudaError_t e = ensure_smem_attr(grouped_gemm_pair_kernel<kGateUp>, kPSmemBytes);
@@ -716,8 +723,9 @@ cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate
     if (p.T == 0) return cudaSuccess;
     bf16* h = (bf16*)p.h;
     bf16* hs = h + p.S * p.I;
-    CUtensorMap m[6];
+    CUtensorMap m[7];
     bool ok = make_map_bf16(&m[0], p.xperm, p.H, p.S, 1, kBK, kBM) &&
+              make_map_bf16(&m[6], p.xperm, p.H, p.S, 1, kBK, kSmallRows) &&
               make_map_bf16(&m[2], w_gate, p.H, p.I, p.E, kBK, kBRows / 2) &&
               make_map_bf16(&m[3], w_up, p.H, p.I, p.E, kBK, kBRows / 2);
     if (ok && p.Is > 0)
@@ -748,11 +756,12 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     if (p.T == 0) return cudaSuccess;
     const bf16* h = (const bf16*)p.h;
     const bf16* hs = h + p.S * p.I;
-    CUtensorMap m[6];
+    CUtensorMap m[7];
     // a CTA pair stages half of the 256 output columns per CTA
     const bool pairs = use_pairs(p, false);
     const uint32_t brows = pairs ? kBRows / 2 : kBRows;
-    bool ok = make_map_bf16(&m[0], h, p.I, p.S, 1, kBK, kBM) && make_map_bf16(&m[2], w_down, p.I, p.H, p.E, kBK, brows);
+    bool ok = make_map_bf16(&m[0], h, p.I, p.S, 1, kBK, kBM) && make_map_bf16(&m[2], w_down, p.I, p.H, p.E, kBK, brows) &&
+              make_map_bf16(&m[6], h, p.I, p.S, 1, kBK, kSmallRows);
     if (ok && p.Is > 0)
         ok = make_map_bf16(&m[1], hs, p.Is, p.T, 1, kBK, kBM) && make_map_bf16(&m[4], ws_down, p.Is, p.H, 1, kBK, brows);
     else {

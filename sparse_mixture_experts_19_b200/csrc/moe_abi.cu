@@ -140,7 +140,7 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->rt_wn2 = (float*)take(tc_router ? sizeof(float) * kRouterMaxSplits * p->E : 0);
     const bool dec = p->S <= kDecodeMaxSlots;
     p->dec_scores = (double*)take(dec ? sizeof(double) * p->T * p->E : 0);
-    p->dec_bar = (unsigned int*)take(dec ? 2 * sizeof(unsigned int) : 0);
+    p->dec_bar = (unsigned int*)take(dec ? kDecodeCounters * sizeof(unsigned int) : 0);
     p->bytes = off;
 }
 

@@ -13,7 +13,7 @@
 //    read as zero) and writes the float32 partial scores P_c[t, e].  The MMA
 //    warp's idle lanes also read every staged x row and router row from
 //    shared memory for their squared norms over the chunk.
-// 2. router_select_kernel (CUDA cores, a warp per token): the partials are
+// 2. router_select_kernel (CUDA cores, a thread per token): the partials are
 //    summed in fp64 with the bias, the selection is made certain against a
 //    bound on the difference from the exact scores, the uncertain experts
 //    are rescored exactly, and the k selected experts are ordered exactly.
@@ -27,9 +27,11 @@
 // and truncates below 24 bits of it.  Summed over the steps, a partial score
 // differs from its exact value by at most c * sum_h |x_h w_h| over the chunk,
 // c = 17 * 2^-23 * (n + 1), and sum_h |x_h w_h| <= ||x_c|| ||w_c|| (Cauchy-
-// Schwarz on the chunk).  The fp64 sum of the partials and the bias adds a
-// relative 1e-14 at most.  So for token t every score is within
-//   delta_t = sum_c c * ||x_{t,c}|| * max_e ||w_{e,c}|| (+ the fp64 term)
+// Schwarz on the chunk).  The partials and the bias are then added in
+// float32, in chunk order; those ns additions add at most
+// (ns + 1) 2^-24 (sum_c ||x_{t,c}|| max_e ||w_{e,c}|| + max_e |b_e|).  So for
+// token t every score is within
+//   delta_t = sum_c c * ||x_{t,c}|| * max_e ||w_{e,c}|| (+ the sum's term)
 // of exact (norms from float32 sums of squares inflated by 1 + H 2^-22, and
 // the whole by 1.001).  Splitting the reduction makes the bound ns times
 // smaller than one float32 sum over all of H.
@@ -43,9 +45,10 @@
 // score, and the k are sorted with exact scores where both have one and
 // approximate ones otherwise, which is the exact order.
 //
-// Importance (optional): each warp forms its token's softmax over all E fp64
-// scores; a block sums its tokens' probabilities per expert in shared memory
-// and adds them to the importance with one atomic add per expert and block.
+// Importance (optional): each token's thread forms its softmax over all E
+// approximate scores; a block sums its tokens' probabilities per expert in
+// shared memory and adds them to the importance with one atomic add per
+// expert and block.
 #include <algorithm>
 
 #include "common.cuh"
@@ -273,20 +276,36 @@ __device__ __forceinline__ bool ranks_before(double a, int ea, double b, int eb)
     return a > b || (a == b && ea < eb);
 }
 
-constexpr int kSelThreads = 128;  // tokens per block of the selection kernel (a thread each)
-constexpr int kQueue = 512;       // exact-rescoring queue entries per block and round
+constexpr int kSelTokens = 32;                 // tokens per block of the selection kernel
+constexpr int kSelThreads = 256;               // eight warps
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelTokPerWarp = kSelTokens / kSelWarps;  // tokens a warp scans
+constexpr int kSeg = 32;                       // queue entries per warp and round (band members)
+constexpr int kPendQ = 128;                    // queue entries per round for certain picks
+constexpr int kQueue = kSelWarps * kSeg + kPendQ;
 
-// Shared memory of the selection kernel: summed scores [128][E + 1] (the +1
+// Shared memory of the selection kernel: summed scores [32][E + 1] (the +1
 // spreads a column over the banks), then the rescoring queue.
 size_t select_smem_bytes(int E) {
-    return sizeof(float) * kSelThreads * (E + 1) + (size_t)kQueue * (8 + 8 + 4) + 64;
+    return sizeof(float) * kSelTokens * (E + 1) + (size_t)kQueue * (8 + 8 + 4) + 64;
 }
 
-// One thread per token: its scores summed from the chunks' partials into
-// shared memory (float32, chunk order), then the selection of the one-pass
-// design: k (+1) rounds of "next best" over the row, the bound, the band
-// rescored exactly through a queue served by every warp of the block, the
-// exact order, the softmax over the k.
+// The token's scores summed from the chunks' partials into shared memory
+// (float32, chunk order); then
+//   scan (a warp per token, four tokens per warp at once): lane l holds the
+//     scores of experts l, l + 32, ...; the kk best are picked in kk rounds
+//     of warp arg-max (ties to the lower index); the importance adds its
+//     softmax over all E scores here;
+//   decision (a thread per token): the bound, the band, the certain picks
+//     that need exact scores for the order;
+//   rescoring (every warp): band members found by the token's warp (ballot
+//     over 32 experts at a time) and the certain picks go through a queue
+//     whose exact scores every warp computes;
+//   finish (a thread per token): the band decided from exact scores, the k
+//     ordered exactly, the softmax over the k.
+// Every long loop runs across a warp's lanes: a thread walking a whole row
+// of E scores alone spends most of its time waiting on its own dependent
+// instructions.
 template <int KMAX>
 __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
     const float* __restrict__ part, const float* __restrict__ xn2, const float* __restrict__ wn2, int T, int H, int E,
@@ -294,50 +313,215 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
     const bf16* __restrict__ wr, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     float* __restrict__ importance) {
     constexpr bool kDense = (KMAX == kMaxTopK);
+    constexpr int kNV = kMaxExperts / 32;  // scores per lane in the scan
     extern __shared__ __align__(16) uint8_t sm_raw[];
     const int ld = E + 1;
-    float* sc = reinterpret_cast<float*>(sm_raw);                           // [128][E + 1]
-    int2* qp = reinterpret_cast<int2*>(sc + (size_t)kSelThreads * ld + 1);  // 8-byte aligned below
+    float* sc = reinterpret_cast<float*>(sm_raw);                          // [32][E + 1]
+    int2* qp = reinterpret_cast<int2*>(sc + (size_t)kSelTokens * ld + 1);  // 16-byte aligned below
     qp = reinterpret_cast<int2*>((reinterpret_cast<uintptr_t>(qp) + 15) & ~uintptr_t(15));
     double* qs = reinterpret_cast<double*>(qp + kQueue);
     float* qa = reinterpret_cast<float*>(qs + kQueue);
     __shared__ float wmax[kRouterMaxSplits];
     __shared__ float bmax_s;
-    __shared__ int qn;
+    __shared__ float s_tv[kSelTokens][KMAX + 1];  // the scan's picks per token
+    __shared__ int s_te[kSelTokens][KMAX + 1];
+    __shared__ float s_lo[kSelTokens], s_hi[kSelTokens];  // band of each token
+    __shared__ int s_cur[kSelTokens];                     // next expert of the band scan (E: done)
+    __shared__ int s_segn[kSelWarps];                     // band entries per warp segment
+    __shared__ int s_pn;                                  // certain-pick entries
+    __shared__ float s_imp[kMaxExperts];
     const int r = threadIdx.x, lane = r & 31, warp = r / 32;
-    const int t0 = blockIdx.x * kSelThreads;
-    const int rows = min(kSelThreads, T - t0);
+    const int t0 = blockIdx.x * kSelTokens;
+    const int rows = min(kSelTokens, T - t0);
     const float slack = 1.f + (float)H * 2.3841858e-7f;  // 1 + H 2^-22
-    if (r < ns) {
+    if (importance)
+        for (int e = r; e < E; e += kSelThreads) s_imp[e] = 0.f;
+    // per chunk the largest router-row norm (warp c), and the largest |bias|
+    // (warp ns, or the last warp): lanes stride over the experts, so the
+    // loads are in flight together
+    for (int c = warp; c < ns; c += kSelWarps) {
         float m = 0.f;
-        for (int e = 0; e < E; ++e) m = fmaxf(m, wn2[r * E + e]);
-        wmax[r] = sqrtf(m * slack);
+        for (int e = lane; e < E; e += 32) m = fmaxf(m, wn2[c * E + e]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) wmax[c] = sqrtf(m * slack);
     }
-    if (r == 32) {
+    if (warp == min(ns, kSelWarps - 1)) {
         float m = 0.f;
         if (bias)
-            for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(bias[e]));
-        bmax_s = m;
+            for (int e = lane; e < E; e += 32) m = fmaxf(m, fabsf(bias[e]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) bmax_s = m;
     }
-    // summed scores: the block's rows of each chunk are one contiguous run
-    for (int c = 0; c < ns; ++c) {
-        const float* src = part + ((int64_t)c * T + t0) * E;
-        for (int i = r; i < rows * E; i += kSelThreads) {
-            const int rr = i / E, e = i % E;
-            const float v = __ldg(src + i);
-            sc[rr * ld + e] = c == 0 ? v : sc[rr * ld + e] + v;
+    // summed scores, chunks added in order 0..ns-1 and then the bias; the
+    // block's rows of each chunk are one contiguous run, and every chunk's
+    // load of an element is issued before the first add, so each thread
+    // keeps ns loads in flight (float4 ones when E is a multiple of 4)
+    {
+        const float* src = part + (int64_t)t0 * E;
+        const int64_t cstride = (int64_t)T * E;
+        if ((E & 3) == 0) {
+            const int n4 = rows * E / 4;
+            for (int i4 = r; i4 < n4; i4 += kSelThreads) {
+                float4 v[kRouterMaxSplits];
+#pragma unroll
+                for (int c = 0; c < kRouterMaxSplits; ++c)
+                    if (c < ns) v[c] = __ldg(reinterpret_cast<const float4*>(src + c * cstride) + i4);
+                float4 a = v[0];
+#pragma unroll
+                for (int c = 1; c < kRouterMaxSplits; ++c)
+                    if (c < ns) {
+                        a.x += v[c].x;
+                        a.y += v[c].y;
+                        a.z += v[c].z;
+                        a.w += v[c].w;
+                    }
+                const int rr = (4 * i4) / E, e = (4 * i4) % E;
+                if (bias) {
+                    a.x += bias[e];
+                    a.y += bias[e + 1];
+                    a.z += bias[e + 2];
+                    a.w += bias[e + 3];
+                }
+                float* d = sc + rr * ld + e;
+                d[0] = a.x;
+                d[1] = a.y;
+                d[2] = a.z;
+                d[3] = a.w;
+            }
+        } else {
+            for (int i = r; i < rows * E; i += kSelThreads) {
+                float v[kRouterMaxSplits];
+#pragma unroll
+                for (int c = 0; c < kRouterMaxSplits; ++c)
+                    if (c < ns) v[c] = __ldg(src + c * cstride + i);
+                float a = v[0];
+#pragma unroll
+                for (int c = 1; c < kRouterMaxSplits; ++c)
+                    if (c < ns) a += v[c];
+                if (bias) a += bias[i % E];
+                sc[(i / E) * ld + i % E] = a;
+            }
         }
     }
     __syncthreads();
-    if (bias)
-        for (int i = r; i < rows * E; i += kSelThreads) sc[(i / E) * ld + i % E] += bias[i % E];
+    const int kk = k < E ? k + 1 : k;  // picks of the scan: k, and the (k+1)-th unless k == E
+
+    // ---------------------------------------------------------- scan
+    // warp w takes tokens w, w + 8, w + 16, w + 24 together (independent
+    // chains hide each other's latency)
+    {
+        float v[kSelTokPerWarp][kNV];
+        float pv[kSelTokPerWarp], top[kSelTokPerWarp];
+        int pe[kSelTokPerWarp];
+#pragma unroll
+        for (int u = 0; u < kSelTokPerWarp; ++u) {
+            const int tt = warp + kSelWarps * u;
+            const float* row = sc + min(tt, kSelTokens - 1) * ld;
+#pragma unroll
+            for (int i = 0; i < kNV; ++i) {
+                const int e = lane + 32 * i;
+                v[u][i] = (tt < rows && e < E) ? row[e] : -INFINITY;
+            }
+            pv[u] = INFINITY;
+            pe[u] = -1;
+            top[u] = -INFINITY;
+        }
+#pragma unroll 1
+        for (int j = 0; j < kk; ++j) {
+            float bv[kSelTokPerWarp];
+            int be[kSelTokPerWarp];
+#pragma unroll
+            for (int u = 0; u < kSelTokPerWarp; ++u) {
+                // this lane's best score ranking after the previous pick
+                // (ascending experts: the first of equal scores is kept)
+                bv[u] = -INFINITY;
+                be[u] = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < kNV; ++i) {
+                    const int e = lane + 32 * i;
+                    const float c = v[u][i];
+                    const bool after = (c < pv[u]) || (c == pv[u] && e > pe[u]);
+                    if (e < E && after && c > -INFINITY && (c > bv[u] || (c == bv[u] && e < be[u]))) {
+                        bv[u] = c;
+                        be[u] = e;
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+                for (int u = 0; u < kSelTokPerWarp; ++u) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv[u], o);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be[u], o);
+                    if (ov > bv[u] || (ov == bv[u] && oe < be[u])) {
+                        bv[u] = ov;
+                        be[u] = oe;
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kSelTokPerWarp; ++u) {
+                const int tt = warp + kSelWarps * u;
+                pv[u] = bv[u];
+                pe[u] = be[u];
+                if (j == 0) top[u] = bv[u];
+                if (lane == 0 && tt < kSelTokens) {
+                    s_tv[tt][j] = bv[u];
+                    s_te[tt][j] = be[u];
+                }
+            }
+        }
+        if (lane == 0)
+#pragma unroll
+            for (int u = 0; u < kSelTokPerWarp; ++u) {
+                const int tt = warp + kSelWarps * u;
+                for (int j = kk; j <= KMAX; ++j) {
+                    s_tv[tt][j] = -INFINITY;
+                    s_te[tt][j] = 0x7fffffff;
+                }
+            }
+        if (importance) {
+            // softmax over all E scores of the token, shifted by its largest
+            // (the first pick), summed per expert over the block
+#pragma unroll
+            for (int u = 0; u < kSelTokPerWarp; ++u) {
+                const int tt = warp + kSelWarps * u;
+                if (tt >= rows) continue;
+                const float m = top[u];
+                float z = 0.f;
+#pragma unroll
+                for (int i = 0; i < kNV; ++i)
+                    if (lane + 32 * i < E) z += __expf(v[u][i] - m);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                const float inv = 1.0f / z;
+#pragma unroll
+                for (int i = 0; i < kNV; ++i)
+                    if (lane + 32 * i < E) atomicAdd(&s_imp[lane + 32 * i], __expf(v[u][i] - m) * inv);
+            }
+        }
+    }
     __syncthreads();
+    if (importance) {
+        for (int e = r; e < E; e += kSelThreads) atomicAdd(&importance[e], s_imp[e]);
+    }
+    // ---------------------------------------------------------- decision
+    // thread r carries token t = t0 + r (r < rows)
     const int t = t0 + r;
-    const float* row = sc + r * ld;
+    const bool own = r < rows;
+    float tv[KMAX + 1];
+    int te[KMAX + 1];
+#pragma unroll
+    for (int j = 0; j <= KMAX; ++j) {
+        tv[j] = own ? s_tv[r][j] : -INFINITY;
+        te[j] = own ? s_te[r][j] : 0x7fffffff;
+    }
     // the bound on |approximate - exact score| for this token (file comment),
     // with the float32 sums of the chunks and the bias counted in
     float delta = 0.f, nsum = 0.f;
-    if (t < T)
+    if (own)
         for (int c = 0; c < ns; ++c) {
             const float a = sqrtf(xn2[(int64_t)c * T + t] * slack) * wmax[c];
             delta += cH * a;
@@ -345,53 +529,10 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
         }
     const float u24 = 5.9604645e-8f;
     const float del2 = 2.f * 1.001f * (delta + (float)(ns + 1) * u24 * (nsum + bmax_s));
-
-    // pass 1: the k (+1) best approximate scores, picked in k (+1) rounds;
-    // round j takes the best score ranking after the pick of round j-1
-    float tv[KMAX + 1];
-    int te[KMAX + 1];
-    const int kk = k < E ? k + 1 : k;
-    float pv = INFINITY;
-    int pe = -1;
-#pragma unroll
-    for (int j = 0; j <= KMAX; ++j) {
-        // four running maxima (elements i % 4), merged at the end; each keeps
-        // the lower index on ties because it visits indices in ascending order
-        float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        int be[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
-        if (j < kk && t < T) {
-            for (int e0 = 0; e0 < E; e0 += 4) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int e = e0 + i;
-                    if (e < E) {
-                        const float cv = row[e];
-                        const bool after = (cv < pv) || (cv == pv && e > pe);
-                        if (after && cv > bv[i]) {
-                            bv[i] = cv;
-                            be[i] = e;
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int c = 1; c < 4; ++c)
-                if (ranks_before(bv[c], be[c], bv[0], be[0])) {
-                    bv[0] = bv[c];
-                    be[0] = be[c];
-                }
-            pv = bv[0];
-            pe = be[0];
-        }
-        tv[j] = bv[0];
-        te[j] = be[0];
-    }
-
-    // certainty of the decision
     float band_lo = 0.f, band_hi = 0.f;
     bool uncertain = false;
-    int n_in = k;
-    if (!kDense && t < T && k < E) {
+    int n_in = k;  // slots 0 .. n_in-1 hold certain picks
+    if (!kDense && own && k < E) {
         float kth = 0.f, next = 0.f;
 #pragma unroll
         for (int j = 0; j <= KMAX; ++j) {
@@ -408,6 +549,35 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
                 if (j < k && tv[j] > band_hi) n_in = j + 1;
         }
     }
+    if (r < kSelTokens) {
+        s_lo[r] = band_lo;
+        s_hi[r] = band_hi;
+        s_cur[r] = uncertain ? 0 : E;
+    }
+    // the k selected: approximate fa, expert fe, exact fx where known (has_x)
+    float fa[KMAX];
+    int fe[KMAX];
+    double fx[KMAX];
+    uint32_t has_x = 0;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        fa[j] = tv[j];
+        fe[j] = te[j];
+        fx[j] = 0.0;
+    }
+    // order: two selected experts within 2 delta need exact scores.  Among
+    // the certain picks (sorted) that is every pick with a neighbour within
+    // 2 delta; the last certain pick is also compared with the best band
+    // score, which bounds every band pick from above.  Band members are all
+    // rescored, so one rescoring pass covers selection and order.
+    uint32_t pend = 0;
+    if (own) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j + 1 < n_in && tv[j] - tv[j + 1] <= del2) pend |= 3u << j;
+            if (uncertain && j == n_in - 1 && tv[j] - tv[j + 1] <= del2) pend |= 1u << j;
+        }
+    }
     // band: the best `need` members by exact score (ties to the lower index)
     const int need = k - n_in;
     double bv[KMAX];
@@ -419,42 +589,89 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
         be[j] = 0x7fffffff;
         ba[j] = -INFINITY;
     }
-    int cursor = uncertain ? 0 : E;  // next expert this thread still has to scan
-    while (__syncthreads_or(cursor < E)) {
-        if (r == 0) qn = 0;
-        __syncthreads();
-        if (cursor < E) {
-            bool stop = false;
-            for (int e = cursor; e < E && !stop; ++e) {
-                const float sv = row[e];
-                if (sv >= band_lo && sv <= band_hi) {
-                    const int slot = atomicAdd(&qn, 1);
-                    if (slot < kQueue) {
-                        qp[slot] = make_int2(r, e);
+    if (r == 0) s_pn = 0;
+    __syncthreads();
+    // ---------------------------------------------------------- rescoring
+    constexpr int kCertain = 1 << 30;  // queue tag: a certain pick's rescoring
+    while (__syncthreads_or(pend != 0 || (own && s_cur[r] < E))) {
+        // band members of the warp's tokens, 32 experts per ballot, into the
+        // warp's segment of the queue; a token whose next hits do not fit
+        // resumes there next round (a segment holds one whole ballot)
+        {
+            int wn = 0;
+            bool full = false;
+#pragma unroll 1
+            for (int u = 0; u < kSelTokPerWarp && !full; ++u) {
+                const int tt = warp + kSelWarps * u;
+                if (tt >= rows) break;
+                int cur = s_cur[tt];
+                if (cur >= E) continue;
+                const float lo = s_lo[tt], hi = s_hi[tt];
+                const float* row = sc + tt * ld;
+                for (; cur < E; cur += 32) {
+                    const int e = cur + lane;
+                    const float sv = e < E ? row[e] : 0.f;
+                    const bool hit = e < E && sv >= lo && sv <= hi;
+                    const unsigned m = __ballot_sync(0xffffffffu, hit);
+                    const int nh = __popc(m);
+                    if (wn + nh > kSeg) {
+                        full = true;
+                        break;
+                    }
+                    if (hit) {
+                        const int slot = warp * kSeg + wn + __popc(m & ((1u << lane) - 1u));
+                        qp[slot] = make_int2(tt, e);
                         qa[slot] = sv;
-                    } else {
-                        stop = true;  // queue full: resume here next round
-                        cursor = e;
+                    }
+                    wn += nh;
+                }
+                __syncwarp();
+                if (lane == 0) s_cur[tt] = cur;  // >= E: done
+            }
+            if (lane == 0) s_segn[warp] = wn;
+        }
+        // certain picks that need exact scores for the order
+        if (pend != 0) {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if ((pend >> j) & 1u) {
+                    const int slot = atomicAdd(&s_pn, 1);
+                    if (slot < kPendQ) {
+                        qp[kSelWarps * kSeg + slot] = make_int2(r, te[j] | kCertain);
+                        pend &= ~(1u << j);
                     }
                 }
+        }
+        __syncthreads();
+        // exact scores of every entry: the warps' segments in warp order, then
+        // the certain picks
+        const int npn = min(s_pn, kPendQ);
+        int total = npn;
+#pragma unroll
+        for (int w = 0; w < kSelWarps; ++w) total += s_segn[w];
+        for (int i = warp; i < total; i += kSelWarps) {
+            int q = i, w = 0;
+            while (w < kSelWarps && q >= s_segn[w]) {
+                q -= s_segn[w];
+                ++w;
             }
-            if (!stop) cursor = E;
+            const int slot = w * kSeg + q;  // w == kSelWarps: the certain picks
+            const int2 pr = qp[slot];
+            const int e = pr.y & ~kCertain;
+            const double sd = exact_score(x, wr, t0 + pr.x, e, H, lane);
+            if (lane == 0) qs[slot] = sd + (bias ? (double)bias[e] : 0.0);
         }
         __syncthreads();
-        const int nq = min(qn, kQueue);
-        for (int i = warp; i < nq; i += kSelThreads / 32) {
-            const int2 pr = qp[i];
-            const double sd = exact_score(x, wr, t0 + pr.x, pr.y, H, lane);
-            if (lane == 0) qs[i] = sd + (bias ? (double)bias[pr.y] : 0.0);
-        }
-        __syncthreads();
-        if (uncertain)
-            for (int i = 0; i < nq; ++i) {
-                const int2 pr = qp[i];
+        if (own) {
+            // band members: only the segment of the warp that scanned token r
+            const int w0 = r % kSelWarps;
+            for (int q = 0; q < s_segn[w0]; ++q) {
+                const int slot = w0 * kSeg + q;
+                const int2 pr = qp[slot];
                 if (pr.x != r) continue;
-                double cv = qs[i];
+                double cv = qs[slot];
                 int ce = pr.y;
-                float ca = qa[i];
+                float ca = qa[slot];
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j) {
                     if (j < need && (cv > bv[j] || (cv == bv[j] && ce < be[j]))) {
@@ -470,40 +687,20 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
                     }
                 }
             }
-    }
-    if (importance) {
-        // softmax over all E scores of the token, shifted by the largest
-        // (tv[0]); summed per expert over the block (shared memory is free
-        // again: every row's scores have been read), then added to global
-        __syncthreads();
-        float* imp = reinterpret_cast<float*>(qp);  // kQueue * 20 bytes >= E floats
-        for (int e = r; e < E; e += kSelThreads) imp[e] = 0.f;
-        __syncthreads();
-        if (t < T) {
-            const float m = tv[0];
-            float z = 0.f;
-            for (int e = 0; e < E; ++e) z += __expf(row[e] - m);
-            const float inv = 1.0f / z;
-            for (int i = 0; i < E; ++i) {
-                const int e = (i + lane) % E;  // lanes spread over experts
-                atomicAdd(&imp[e], __expf(row[e] - m) * inv);
+            for (int q = 0; q < npn; ++q) {
+                const int slot = kSelWarps * kSeg + q;
+                const int2 pr = qp[slot];
+                if (pr.x != r) continue;
+                const int e = pr.y & ~kCertain;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (j < n_in && fe[j] == e) {
+                        fx[j] = qs[slot];
+                        has_x |= 1u << j;
+                    }
             }
         }
-        __syncthreads();
-        for (int e = r; e < E; e += kSelThreads) atomicAdd(&importance[e], imp[e]);
-        __syncthreads();
-    }
-
-    // the k selected: approximate fa, expert fe, exact fx where known (has_x)
-    float fa[KMAX];
-    int fe[KMAX];
-    double fx[KMAX];
-    uint32_t has_x = 0;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        fa[j] = tv[j];
-        fe[j] = te[j];
-        fx[j] = 0.0;
+        if (r == 0) s_pn = 0;  // read above into npn; the next pushes follow the loop's barrier
     }
     if (!kDense && uncertain) {
         // move the band picks to slots n_in..k-1 (predicated shifts keep
@@ -526,48 +723,6 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
                 fx[j] = bv[j];
                 has_x |= 1u << j;
             }
-    }
-    // order: every selected expert with another selected one within 2 delta
-    // needs its exact score
-    uint32_t pending = 0;
-    if (t < T) {
-#pragma unroll
-        for (int i = 0; i < KMAX; ++i)
-#pragma unroll
-            for (int j = i + 1; j < KMAX; ++j)
-                if (j < k && fabsf(fa[i] - fa[j]) <= del2) pending |= (1u << i) | (1u << j);
-        pending &= ~has_x;
-    }
-    while (__syncthreads_or(pending != 0)) {
-        if (r == 0) qn = 0;
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-            if ((pending >> j) & 1u) {
-                const int slot = atomicAdd(&qn, 1);
-                if (slot < kQueue) {
-                    qp[slot] = make_int2(r, fe[j]);
-                    pending &= ~(1u << j);
-                }
-            }
-        __syncthreads();
-        const int nq = min(qn, kQueue);
-        for (int i = warp; i < nq; i += kSelThreads / 32) {
-            const int2 pr = qp[i];
-            const double sd = exact_score(x, wr, t0 + pr.x, pr.y, H, lane);
-            if (lane == 0) qs[i] = sd + (bias ? (double)bias[pr.y] : 0.0);
-        }
-        __syncthreads();
-        for (int i = 0; i < nq; ++i) {
-            const int2 pr = qp[i];
-            if (pr.x != r) continue;
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j)
-                if (j < k && fe[j] == pr.y) {
-                    fx[j] = qs[i];
-                    has_x |= 1u << j;
-                }
-        }
     }
     // sort the k by (score desc, index asc): exact scores where both have
     // one, else approximate ones (more than 2 delta apart, in the right order)
@@ -595,7 +750,7 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
             }
         }
     }
-    if (t < T) {
+    if (own) {
         // softmax over the k selected; differences in fp64 where both scores are exact
         double sj[KMAX];
 #pragma unroll
@@ -656,7 +811,7 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     // the bound's constant for the longest chunk: 4 MMA steps per 64 of reduction
     const float cH = 17.f * 1.1920929e-7f * (float)(4 * ((kchunk + kBK - 1) / kBK) + 1) * 1.01f;
     const size_t ssm = select_smem_bytes(E);
-    const dim3 sgrid((unsigned)((p.T + kSelThreads - 1) / kSelThreads));
+    const dim3 sgrid((unsigned)((p.T + kSelTokens - 1) / kSelTokens));
     trace_before("router_select", st);
     // top_k > 8 only as top_k == E <= 32
     if (p.k <= 8) {
