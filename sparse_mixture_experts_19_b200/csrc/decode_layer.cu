@@ -24,14 +24,14 @@
 //      rounds, then the softmax of those k; the same arithmetic in every
 //      CTA gives every CTA the same plan: the slots grouped by expert, the
 //      capacity cut in token order, the shared expert as one more group.
-//   2. gate/up and down, overlapped.  Eleven warps stream gate/up rows:
+//   2. gate/up and down, overlapped.  Ten warps stream gate/up rows:
 //      CTA c owns the intermediate rows i in [R c / G, R (c+1) / G) of
 //      every group (R = I, or I_s for the shared expert), group by group,
 //      each row's gate and up rows read with 16-byte loads (L2
 //      evict-first) and dotted with the group's token vectors from shared
 //      memory: h[slot][i] = bf16(silu(x.g) * (x.u)).  When the CTA's rows
 //      of a group are written, the CTA publishes the group (a per-group
-//      counter in global memory).  The other five warps take the down rows
+//      counter in global memory).  The other six warps take the down rows
 //      group by group: once every CTA has published group g, they copy its
 //      h rows into shared memory and dot them with the down rows of this
 //      CTA's output columns j in [H c / G, H (c+1) / G), while the gate/up
@@ -58,7 +58,7 @@ constexpr int kDlBatch = 4;                        // token vectors per pass ove
 constexpr int kDlUnroll = 6;                       // 16-byte chunks per lane in flight, per row
 constexpr int kDlMaxCols = 64;                     // output columns per CTA in phase 3 (H <= 64 * grid)
 constexpr int kDlSmemMax = 200 * 1024;
-constexpr int kDlDownWarps = 5;                      // warps on the down rows (about a third of the bytes)
+constexpr int kDlDownWarps = 6;                      // warps on the down rows (a third of the bytes, and the waits)
 constexpr int kDlUpWarps = kDlWarps - kDlDownWarps;  // warps on the gate/up rows
 
 // Bytes of one group's h vectors in shared memory: a routed expert meets a
@@ -148,6 +148,11 @@ __device__ __forceinline__ uint4 ld_stream(const void* ptr, uint64_t pol) {
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
         : "l"(ptr), "l"(pol));
     return v;
+}
+
+// Bytes [ptr, ptr + bytes) into L2 (16-byte aligned, a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -741,8 +746,24 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
             }
         }
         // then the last group's down columns, with the down warps, once the
-        // down warps have staged its h rows (bounded wait)
+        // down warps have staged its h rows (bounded wait).  Meanwhile its
+        // down rows of this CTA's columns (consecutive rows) go into L2, in
+        // 2 KB prefetches dealt over the gate/up warps' lanes: a prefetch
+        // holds its warp up, and these warps have nothing else to do; the
+        // last group's dots then wait on L2 instead of HBM.
         if (cols > 0) {
+            {
+                const int g = ng - 1;
+                const bool sh = pl.gexp[g] == a.E;
+                const int R = sh ? a.Is : a.I;
+                const uint8_t* base =
+                    kMx ? a.mdb + ((int64_t)pl.gexp[g] * a.H + j0) * (R / 2)
+                        : reinterpret_cast<const uint8_t*>(sh ? a.wsd + (int64_t)j0 * R
+                                                              : a.wd + ((int64_t)pl.gexp[g] * a.H + j0) * R);
+                const int64_t bytes = (int64_t)cols * R * 2 / (kMx ? 4 : 1);
+                for (int64_t off = (int64_t)(warp * 32 + lane) * 2048; off < bytes; off += kDlUpWarps * 32 * 2048)
+                    prefetch_l2(base + off, (uint32_t)std::min<int64_t>(2048, bytes - off));
+            }
             int st = 0;
             const uint64_t t0 = global_ns();
             while ((st = *reinterpret_cast<volatile int*>(&last_state)) == 0) {

@@ -701,7 +701,7 @@ cudaError_t launch_grouped_pair(const Plan& p, const CUtensorMap (&maps)[7], con
 // were as fast or faster: in a pair each SM's tensor core still reads all of
 // B (its half from its own shared memory, the other half from the peer's),
 // so shared-memory traffic drops only by about a sixth.
-bool use_pairs(const Plan& p, bool gate_up) { return !gate_up && p.I <= 1024 && p.S >= 512 * p.E; }
+bool use_pairs(const Plan& p) { return p.I <= 1024 && p.S >= 512 * p.E; }
 
 GemmArgs base_args(const Plan& p) {
     GemmArgs a{};
@@ -743,10 +743,8 @@ cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate
     a.K = a.Ks = (int)p.H;
     a.h = h;
     a.hs = hs;
-    const bool pairs = use_pairs(p, true);
-    if (pairs) a.mtile_prefix = p.mpair_prefix;
     trace_before("gateup_sm100", st);
-    cudaError_t e = pairs ? launch_grouped_pair<true>(p, m, a, st) : launch_grouped<true>(p, m, a, st);
+    cudaError_t e = launch_grouped<true>(p, m, a, st);  // single CTAs (pairs measured no faster here)
     trace_after(st);
     return e;
 }
@@ -758,7 +756,7 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     const bf16* hs = h + p.S * p.I;
     CUtensorMap m[7];
     // a CTA pair stages half of the 256 output columns per CTA
-    const bool pairs = use_pairs(p, false);
+    const bool pairs = use_pairs(p);
     const uint32_t brows = pairs ? kBRows / 2 : kBRows;
     bool ok = make_map_bf16(&m[0], h, p.I, p.S, 1, kBK, kBM) && make_map_bf16(&m[2], w_down, p.I, p.H, p.E, kBK, brows) &&
               make_map_bf16(&m[6], h, p.I, p.S, 1, kBK, kSmallRows);

@@ -306,14 +306,14 @@ size_t select_smem_bytes(int E) {
 // Every long loop runs across a warp's lanes: a thread walking a whole row
 // of E scores alone spends most of its time waiting on its own dependent
 // instructions.
-template <int KMAX>
+template <int KMAX, int kNV>
 __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
     const float* __restrict__ part, const float* __restrict__ xn2, const float* __restrict__ wn2, int T, int H, int E,
     int k, int ns, float cH, const float* __restrict__ bias, const bf16* __restrict__ x,
     const bf16* __restrict__ wr, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     float* __restrict__ importance) {
     constexpr bool kDense = (KMAX == kMaxTopK);
-    constexpr int kNV = kMaxExperts / 32;  // scores per lane in the scan
+    // kNV = ceil(E / 32): scores per lane in the scan
     extern __shared__ __align__(16) uint8_t sm_raw[];
     const int ld = E + 1;
     float* sc = reinterpret_cast<float*>(sm_raw);                          // [32][E + 1]
@@ -813,20 +813,26 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     const size_t ssm = select_smem_bytes(E);
     const dim3 sgrid((unsigned)((p.T + kSelTokens - 1) / kSelTokens));
     trace_before("router_select", st);
-    // top_k > 8 only as top_k == E <= 32
-    if (p.k <= 8) {
-        e = ensure_smem_attr(router_select_kernel<8>, ssm);
-        if (e == cudaSuccess)
-            router_select_kernel<8><<<sgrid, kSelThreads, ssm, st>>>(
-                p.rt_part, p.rt_xn2, p.rt_wn2, (int)p.T, (int)p.H, E, (int)p.k, ns, cH, router_b, (const bf16*)x,
-                (const bf16*)router_w, topk_idx, topk_w, p.importance);
-    } else {
-        e = ensure_smem_attr(router_select_kernel<kMaxTopK>, ssm);
-        if (e == cudaSuccess)
-            router_select_kernel<kMaxTopK><<<sgrid, kSelThreads, ssm, st>>>(
-                p.rt_part, p.rt_xn2, p.rt_wn2, (int)p.T, (int)p.H, E, (int)p.k, ns, cH, router_b, (const bf16*)x,
-                (const bf16*)router_w, topk_idx, topk_w, p.importance);
-    }
+    // top_k > 8 only as top_k == E <= 32; kNV covers E in 32-expert steps
+    auto go = [&](auto kern) {
+        cudaError_t r = ensure_smem_attr(kern, ssm);
+        if (r == cudaSuccess)
+            kern<<<sgrid, kSelThreads, ssm, st>>>(p.rt_part, p.rt_xn2, p.rt_wn2, (int)p.T, (int)p.H, E, (int)p.k, ns,
+                                                  cH, router_b, (const bf16*)x, (const bf16*)router_w, topk_idx,
+                                                  topk_w, p.importance);
+        return r;
+    };
+    const int nv = (E + 31) / 32;
+    if (p.k > 8)
+        e = go(router_select_kernel<kMaxTopK, 1>);
+    else if (nv <= 1)
+        e = go(router_select_kernel<8, 1>);
+    else if (nv <= 2)
+        e = go(router_select_kernel<8, 2>);
+    else if (nv <= 4)
+        e = go(router_select_kernel<8, 4>);
+    else
+        e = go(router_select_kernel<8, 8>);
     trace_after(st);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e;
