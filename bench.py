@@ -465,13 +465,28 @@ def run_ours(args, wl, world, rank, local):
         if wl.capacity_factor > 0:
             kept = int(np.minimum(counts.cpu().numpy(), moe.capacity(cfg)).sum())
         flops = 2.0 * kept * 2 * wl.H * wl.I + 2.0 * wl.T * 2 * wl.H * wl.I_shared
-        achieved = flops / t_avg / 1e12
-        # one launch of the kernel lasts milliseconds at most: burst peak
-        peak = pk["bf16_tflops"]
-        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic_for(dom, wl),
-                "peak_kind": f"{pk_kind} bf16 dense, burst", "launch_ms": t_avg * 1e3,
-                "flops_per_launch": flops, "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
+        # the kernel's algorithmic bytes: the gate and up weights of the
+        # active experts (+ shared), its A rows read and its h rows written
+        elt = 2 if wl.dtype == "bf16" else 4
+        gu_bytes = float(elt * (2 * wl.H * (active * wl.I + wl.I_shared)
+                                + (kept + (wl.T if wl.I_shared else 0)) * wl.H
+                                + kept * wl.I + wl.T * wl.I_shared))
+        if gu_bytes / (pk["hbm_gbs"] * 1e9) > flops / (pk["bf16_tflops"] * 1e12):
+            # few rows per expert: the launch is bound by reading the weights
+            achieved = gu_bytes / t_avg / 1e9
+            roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(dom, wl),
+                    "peak_kind": f"{pk_kind} HBM copy", "launch_ms": t_avg * 1e3, "bytes_per_launch": gu_bytes,
+                    "flops_per_launch": flops}
+        else:
+            achieved = flops / t_avg / 1e12
+            # one launch of the kernel lasts milliseconds at most: burst peak
+            peak = pk["bf16_tflops"]
+            roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": traffic_for(dom, wl),
+                    "peak_kind": f"{pk_kind} bf16 dense, burst", "launch_ms": t_avg * 1e3,
+                    "flops_per_launch": flops, "bytes_per_launch": gu_bytes,
+                    "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
     F = layer_flops(wl)
     B = layer_bytes(wl, active)
     t_roof = max(F / (pk["bf16_tflops"] * 1e12), B / (pk["hbm_gbs"] * 1e9))
