@@ -92,7 +92,7 @@ __device__ __forceinline__ float row_sumsq(uint32_t row, int lane) {
 }
 
 // One CTA: tile `tile` of 128 tokens, chunk c of the reduction.
-__global__ void __launch_bounds__(kThreads, 1) router_partial_kernel(
+__global__ void __launch_bounds__(kThreads, 2) router_partial_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int H, int E, int Npad,
     int ns, int kchunk, int stages, uint32_t acc_cols, float* __restrict__ part, float* __restrict__ xn2,
     float* __restrict__ wn2, int32_t* flags) {
@@ -266,6 +266,16 @@ __device__ __forceinline__ double exact_score(const bf16* x, const bf16* w, int6
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     return sum;
+}
+
+// float -> unsigned with the same order (-0 taken as +0, so that equal floats
+// get equal keys), and back.
+__device__ __forceinline__ unsigned ordered_key(float v) {
+    const unsigned u = __float_as_uint(v == 0.f ? 0.f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_ordered_key(unsigned k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 // (a, ea) ranks before (b, eb): larger score, then lower expert index.
@@ -449,17 +459,19 @@ __global__ void __launch_bounds__(kSelThreads) router_select_kernel(
                     }
                 }
             }
+            // warp arg-max: the largest score (one max reduction over
+            // order-preserving keys), then the lowest expert index among the
+            // lanes holding it (one min reduction)
+            unsigned key[kSelTokPerWarp], m[kSelTokPerWarp];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
+            for (int u = 0; u < kSelTokPerWarp; ++u) {
+                key[u] = ordered_key(bv[u]);
+                m[u] = __reduce_max_sync(0xffffffffu, key[u]);
+            }
 #pragma unroll
-                for (int u = 0; u < kSelTokPerWarp; ++u) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv[u], o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be[u], o);
-                    if (ov > bv[u] || (ov == bv[u] && oe < be[u])) {
-                        bv[u] = ov;
-                        be[u] = oe;
-                    }
-                }
+            for (int u = 0; u < kSelTokPerWarp; ++u) {
+                be[u] = (int)__reduce_min_sync(0xffffffffu, key[u] == m[u] ? (unsigned)be[u] : 0xffffffffu);
+                bv[u] = from_ordered_key(m[u]);
             }
 #pragma unroll
             for (int u = 0; u < kSelTokPerWarp; ++u) {
@@ -795,8 +807,11 @@ cudaError_t launch_router_sm100(const Plan& p, const void* x, const void* router
     router_splits(p.H, &ns, &kchunk);
     const int stage_bytes = kABytes + Npad * kBK * 2;
     const size_t fixed = 1024 + 256;  // alignment slack + barrier block
-    int stages = (int)((227 * 1024 - fixed) / stage_bytes);
-    stages = std::min(stages, kMaxStages);
+    // a ring small enough for two CTAs per SM (and two accumulators in TMEM,
+    // 2 x 256 columns at most): one CTA's drain of its partials overlaps the
+    // other's loads and MMAs
+    int stages = (int)((113 * 1024 - fixed) / stage_bytes);
+    stages = std::max(2, std::min(stages, kMaxStages));
     stages = std::min(stages, (kchunk + kBK - 1) / kBK);
     const size_t smem = (size_t)stages * stage_bytes + fixed;
     const int ntiles = (int)((p.T + kBM - 1) / kBM);
