@@ -62,9 +62,9 @@ _SIGS = {
                            ctypes.c_int),
     "moe_forward_expert_shard": ([ctypes.POINTER(moe_config_t), _P, _P, _P, ctypes.c_int32, ctypes.c_int32]
                                  + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int),
-    "moe_forward_mxfp4": ([ctypes.POINTER(moe_config_t)] + [_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_forward_mxfp4": ([ctypes.POINTER(moe_config_t)] + [_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_backward_workspace_size": ([ctypes.POINTER(moe_config_t)], ctypes.c_size_t),
-    "moe_backward": ([ctypes.POINTER(moe_config_t)] + [_P] * 20 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_backward": ([ctypes.POINTER(moe_config_t)] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int),
     "moe_reduce_partials": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_int32, _P, _P], ctypes.c_int),
     "moe_get_device_status": ([ctypes.POINTER(moe_config_t), _P, ctypes.c_size_t, _P,
                                ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),

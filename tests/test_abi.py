@@ -40,6 +40,20 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
 
 
+def test_binding_signatures_match_the_header():
+    """Every declared function's ctypes argtypes has as many entries as the
+    header's parameter list: an argument past the argtypes would be converted
+    by ctypes' defaults (a Python int becomes a 32-bit C int), so a 64-bit
+    parameter there (the stream) would arrive with garbage upper bits."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"\b(moe_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S)
+    assert decls
+    for name, params in decls:
+        params = params.strip()
+        n = 0 if params in ("", "void") else len([q for q in params.split(",") if q.strip()])
+        assert len(moe._SIGS[name][0]) == n, f"{name}: header has {n} parameters, binding {len(moe._SIGS[name][0])}"
+
+
 def cfg(**kw):
     base = dict(T=64, H=128, I=256, E=8, top_k=2, I_shared=0, capacity_factor=0.0, dtype="bf16")
     base.update(kw)
