@@ -51,8 +51,9 @@ def parse_args():
     ap.add_argument("--workload", default="fine_grained_e256_layer")
     ap.add_argument("--T", type=int, default=0, help="override the token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=["forward", "route"], default="forward",
-                    help="route: time moe_route alone (only x and the router weights are allocated)")
+    ap.add_argument("--stage", choices=["forward", "route", "mxfp4", "backward"], default="forward",
+                    help="route: time moe_route alone (only x and the router weights are allocated); "
+                         "mxfp4: moe_forward_mxfp4 at decode sizes; backward: moe_backward")
     ap.add_argument("--importance", action="store_true",
                     help="with --stage route: also time moe_route_importance (router importance as a side output)")
     ap.add_argument("--no-graph", action="store_true",
@@ -582,11 +583,130 @@ def run_route_stage(args, wl):
     return out
 
 
+def _stage_setup(wl, router_only=False):
+    import numpy as np
+    import torch
+
+    import moe_inputs as mi
+    import sparse_mixture_experts_19_b200 as moe
+    from sparse_mixture_experts_19_b200 import build as moe_build
+
+    moe_build.build()
+    moe.load()
+    inp = mi.make_inputs(wl, router_only=router_only)
+
+    def to_dev(a):
+        if a is None:
+            return None
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.cuda()
+
+    return moe, inp, {k: to_dev(v) for k, v in inp.items()}
+
+
+def _time_calls(args, call):
+    """Device time of one call, averaged over K calls after W warm-up calls
+    (CUDA events on the current stream, nothing inside the K calls)."""
+    import torch
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / args.steps
+
+
+def run_mxfp4_stage(args, wl):
+    """moe_forward_mxfp4 (decode sizes, MXFP4 routed experts): one line, the
+    layer's time against the HBM copy peak for the bytes it must read."""
+    import numpy as np
+    import torch
+
+    import moe_inputs as mi
+
+    wl = wl.with_(I_shared=0)
+    moe, inp, d = _stage_setup(wl, router_only=True)
+    mx = mi.make_mxfp4_experts(wl)
+    dm = {n: tuple(torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in mx[n]) for n in mx}
+    cfg = moe.config(wl.T, wl.H, wl.I, wl.E, wl.k, 0, wl.capacity_factor, "bf16")
+    ws = moe.workspace(cfg)
+    y = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    call = lambda: moe.moe_forward_mxfp4(cfg, d["x"], d["router_w"], d["router_b"], *dm["w_gate"], *dm["w_up"],
+                                         *dm["w_down"], y, None, counts, None, ws)
+    ms = _time_calls(args, call)
+    if moe.moe_get_device_status(cfg, ws) != 0:
+        raise SystemExit("device check flags set")
+    active = int((counts > 0).sum().item())
+    # per active expert: three weight matrices of H*I E2M1 codes (half a
+    # byte each) and one scale byte per 32 elements; plus x, y, router rows
+    nbytes = active * 3 * wl.H * wl.I * (0.5 + 1.0 / 32) + 2 * wl.T * wl.H * 2 + wl.E * wl.H * 2
+    pk, pk_kind = peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"stage": "mxfp4", "config": config_of(wl), "ms_per_call": ms, "tokens_per_s": wl.T / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "bytes_per_launch": nbytes, "active_experts": active,
+                         "peak_kind": f"{pk_kind} HBM copy"}}
+
+
+def run_backward_stage(args, wl):
+    """moe_backward (every gradient of the bf16 layer): one line, its time
+    against the bf16 tensor peak for its GEMM flops."""
+    import torch
+
+    moe, inp, d = _stage_setup(wl)
+    dy = torch.randn((wl.T, wl.H), device="cuda").to(torch.bfloat16)
+    cfg = moe.config(wl.T, wl.H, wl.I, wl.E, wl.k, wl.I_shared, wl.capacity_factor, "bf16")
+    ws = torch.zeros(moe.moe_backward_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    moe.moe_route(cfg, d["x"], d["router_w"], d["router_b"], idx, w, ws)
+    E, H, I, Is, T = wl.E, wl.H, wl.I, wl.I_shared, wl.T
+    f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device="cuda")
+    g = [f32(T, H), f32(E, H), f32(E), f32(E, I, H), f32(E, I, H), f32(E, H, I)]
+    g += [f32(Is, H), f32(Is, H), f32(H, Is)] if Is else [None, None, None]
+    call = lambda: moe.moe_backward(cfg, d["x"], dy, idx, w, d["router_w"], d["w_gate"], d["w_up"], d["w_down"],
+                                    d["ws_gate"], d["ws_up"], d["ws_down"], *g, ws=ws)
+    ms = _time_calls(args, call)
+    if moe.moe_get_device_status(cfg, ws) != 0:
+        raise SystemExit("device check flags set")
+    # per-kernel times from one more, traced call (each launch bracketed by
+    # events: shares, not a breakdown of ms_per_call)
+    moe.moe_trace_begin(256)
+    call()
+    torch.cuda.synchronize()
+    kern = {}
+    for name, t in moe.moe_trace_end(256):
+        kern[name] = kern.get(name, 0.0) + t
+    counts = torch.bincount(idx.flatten().long(), minlength=E)
+    kept = int(counts.sum().item())
+    if wl.capacity_factor > 0:
+        kept = int(torch.clamp(counts, max=moe.capacity(cfg)).sum().item())
+    # GEMM flops: recomputed gate/up (4HI), dY.W_d (2HI), dGU.W_gu (4HI),
+    # dW_gate|up (4HI), dW_down (2HI) per kept row; the same for the shared
+    # expert per token; the router's weight gradient 2HE per token
+    flops = 16.0 * H * I * kept + 16.0 * H * Is * T + 2.0 * H * E * T
+    pk, pk_kind = peaks()
+    achieved = flops / (ms / 1e3) / 1e12
+    return {"stage": "backward", "config": config_of(wl), "ms_per_call": ms, "tokens_per_s": T / (ms / 1e3),
+            "kernels_ms_traced": kern,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "flops_per_launch": flops,
+                         "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
+                         "peak_kind": f"{pk_kind} bf16 dense, burst"}}
+
+
 def main():
     args = parse_args()
     wl = workload(args)
-    if args.stage == "route":
-        print(json.dumps(run_route_stage(args, wl)), flush=True)
+    if args.stage != "forward":
+        run = {"route": run_route_stage, "mxfp4": run_mxfp4_stage, "backward": run_backward_stage}[args.stage]
+        print(json.dumps(run(args, wl)), flush=True)
         return
     world, rank, local = dist_setup(args)
     if args.impl == "reference":

@@ -100,28 +100,51 @@ __device__ __forceinline__ float sigmoid_f32(float z) { return 1.f / (1.f + __ex
 
 // SwiGLU backward of one row: GU [2I] float32 (g | u), dA [I] float32,
 // weight w -> dGU [2I] bf16 (dg | du), hw [I] bf16 (w h); returns dA . h.
-// One warp; pad rows (w < 0 marks them) write zeros and return 0.
+// One warp, eight consecutive elements per lane and pass (I is a multiple of
+// 8: 16-byte loads and stores); pad rows write zeros and return 0.
 __device__ float swiglu_backward_row(const float* __restrict__ gu, const float* __restrict__ da_row, float w,
                                      int I, bf16* __restrict__ dgu, bf16* __restrict__ hw, bool pad) {
     const int lane = threadIdx.x % 32;
     float dot = 0.f;
-    for (int i = lane; i < I; i += 32) {
+    for (int i = lane * 8; i < I; i += 32 * 8) {
+        uint4 o_dg, o_du, o_hw;
         if (pad) {
-            dgu[i] = __float2bfloat16_rn(0.f);
-            dgu[I + i] = __float2bfloat16_rn(0.f);
-            hw[i] = __float2bfloat16_rn(0.f);
-            continue;
+            o_dg = o_du = o_hw = make_uint4(0, 0, 0, 0);
+        } else {
+            float g[8], u[8], d[8];
+            *reinterpret_cast<float4*>(g) = *reinterpret_cast<const float4*>(gu + i);
+            *reinterpret_cast<float4*>(g + 4) = *reinterpret_cast<const float4*>(gu + i + 4);
+            *reinterpret_cast<float4*>(u) = *reinterpret_cast<const float4*>(gu + I + i);
+            *reinterpret_cast<float4*>(u + 4) = *reinterpret_cast<const float4*>(gu + I + i + 4);
+            *reinterpret_cast<float4*>(d) = *reinterpret_cast<const float4*>(da_row + i);
+            *reinterpret_cast<float4*>(d + 4) = *reinterpret_cast<const float4*>(da_row + i + 4);
+            __nv_bfloat162 rg[4], ru[4], rh[4];
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                float vg[2], vu[2], vh[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const float gj = g[j + h2], uj = u[j + h2];
+                    const float sg = sigmoid_f32(gj);
+                    const float silu = gj * sg;
+                    const float h = __bfloat162float(__float2bfloat16_rn(silu * uj));  // the forward's bf16 h
+                    dot = fmaf(d[j + h2], h, dot);
+                    const float da = w * d[j + h2];
+                    vg[h2] = da * uj * sg * (1.f + gj * (1.f - sg));
+                    vu[h2] = da * silu;
+                    vh[h2] = w * h;
+                }
+                rg[j / 2] = __floats2bfloat162_rn(vg[0], vg[1]);
+                ru[j / 2] = __floats2bfloat162_rn(vu[0], vu[1]);
+                rh[j / 2] = __floats2bfloat162_rn(vh[0], vh[1]);
+            }
+            o_dg = *reinterpret_cast<const uint4*>(rg);
+            o_du = *reinterpret_cast<const uint4*>(ru);
+            o_hw = *reinterpret_cast<const uint4*>(rh);
         }
-        const float g = gu[i], u = gu[I + i];
-        const float sg = sigmoid_f32(g);
-        const float silu = g * sg;
-        const float h = __bfloat162float(__float2bfloat16_rn(silu * u));  // the forward's bf16 h
-        const float d = da_row[i];
-        dot = fmaf(d, h, dot);
-        const float da = w * d;
-        dgu[i] = __float2bfloat16_rn(da * u * sg * (1.f + g * (1.f - sg)));
-        dgu[I + i] = __float2bfloat16_rn(da * silu);
-        hw[i] = __float2bfloat16_rn(w * h);
+        *reinterpret_cast<uint4*>(dgu + i) = o_dg;
+        *reinterpret_cast<uint4*>(dgu + I + i) = o_du;
+        *reinterpret_cast<uint4*>(hw + i) = o_hw;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
@@ -176,12 +199,24 @@ __global__ void bwd_softmax_kernel(const int32_t* __restrict__ idx, const float*
     }
 }
 
-// db[e] = sum over tokens of dL32[t, e], in token order (one thread per expert).
-__global__ void bwd_bias_kernel(const float* __restrict__ dL32, int64_t T, int E, float* __restrict__ db) {
+// db[e] = sum over tokens of dL32[t, e], in two passes of fixed order:
+// block b sums its token range (thread e: column e, tokens in order; rows
+// read whole) into part[b][e], then thread e adds the parts in block order.
+constexpr int kBiasBlocks = 128;
+__global__ void __launch_bounds__(256) bwd_bias_part_kernel(const float* __restrict__ dL32, int64_t T, int E,
+                                                            float* __restrict__ part) {
+    const int64_t t0 = T * blockIdx.x / gridDim.x, t1 = T * (blockIdx.x + 1) / gridDim.x;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float acc = 0.f;
+        for (int64_t t = t0; t < t1; ++t) acc += dL32[t * E + e];
+        part[(int64_t)blockIdx.x * E + e] = acc;
+    }
+}
+__global__ void bwd_bias_kernel(const float* __restrict__ part, int nparts, int E, float* __restrict__ db) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= E) return;
     float acc = 0.f;
-    for (int64_t t = 0; t < T; ++t) acc += dL32[t * E + e];
+    for (int b = 0; b < nparts; ++b) acc += part[(int64_t)b * E + e];
     db[e] = acc;
 }
 
@@ -249,7 +284,7 @@ struct BwdPlan {
     int64_t Rp, Tpad, Epad;
     int32_t *poff, *prow_tok, *prow_slot, *slot_prow, *aux;
     bf16 *xp, *dyp, *dgu, *hw, *dgus, *hws, *dL;
-    float *gu, *da, *dxp, *gus, *das, *dxs, *dw_slot, *dl_slot, *dL32, *dwr;
+    float *gu, *da, *dxp, *gus, *das, *dxs, *dw_slot, *dl_slot, *dL32, *dwr, *bias_part;
     size_t bytes;
 };
 
@@ -287,6 +322,7 @@ static size_t bwd_plan(const Plan& p, void* base, BwdPlan* b) {
     b->dL32 = (float*)take(4 * T * p.E);
     b->dL = (bf16*)take(2 * T * b->Epad);
     b->dwr = (float*)take(4 * b->Epad * H);
+    b->bias_part = (float*)take(4 * kBiasBlocks * p.E);
     b->bytes = off;
     return off;
 }
@@ -340,7 +376,8 @@ static cudaError_t run_backward(const Plan& p, const BwdPlan& b, const void* x, 
     trace_before("bwd_softmax", st);
     bwd_softmax_kernel<<<blocks(T, 256), 256, 0, st>>>(idx, topk_w, b.dw_slot, T, k, E, (int)b.Epad, b.dl_slot,
                                                        b.dL32, b.dL);
-    bwd_bias_kernel<<<(E + 255) / 256, 256, 0, st>>>(b.dL32, T, E, d_router_b);
+    bwd_bias_part_kernel<<<kBiasBlocks, 256, 0, st>>>(b.dL32, T, E, b.bias_part);
+    bwd_bias_kernel<<<(E + 255) / 256, 256, 0, st>>>(b.bias_part, kBiasBlocks, E, d_router_b);
     trace_after(st);
     BWD_TRY(cudaGetLastError());
     // the experts' input gradient rows, then dx

@@ -286,6 +286,20 @@ __device__ __forceinline__ void row_dots_mx(const uint4* const (&codes)[NR], con
         for (int u = 0; u < kMxUnroll; ++u) {
             const int b = b0 + 32 * u;
             if (b < nblk) {
+                // the block's 32 codes of each row as f16x2 pairs, once for
+                // all token vectors
+                uint32_t hw[NR][16];
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const uint32_t cw[4] = {w[r][u].x, w[r][u].y, w[r][u].z, w[r][u].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t h4[4];
+                        e2m1x8_to_f16x2(cw[q], h4);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) hw[r][4 * q + j] = h4[j];
+                    }
+                }
 #pragma unroll
                 for (int n = 0; n < NV; ++n) {
                     uint32_t xv[16];
@@ -299,16 +313,16 @@ __device__ __forceinline__ void row_dots_mx(const uint4* const (&codes)[NR], con
                     }
 #pragma unroll
                     for (int r = 0; r < NR; ++r) {
-                        const uint32_t cw[4] = {w[r][u].x, w[r][u].y, w[r][u].z, w[r][u].w};
-                        uint32_t p = 0u;  // f16x2 zero
+                        // four independent f16x2 chains of four FMAs each
+                        uint32_t p[4] = {0u, 0u, 0u, 0u};  // f16x2 zeros
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t hw[4];
-                            e2m1x8_to_f16x2(cw[q], hw);
+                        for (int q = 0; q < 4; ++q)
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) p = hfma2_u32(hw[j], xv[4 * q + j], p);
-                        }
-                        const __half2 ph = *reinterpret_cast<const __half2*>(&p);
+                            for (int j = 0; j < 4; ++j) p[j] = hfma2_u32(hw[r][4 * q + j], xv[4 * q + j], p[j]);
+                        const __half2 ph = __hadd2(__hadd2(*reinterpret_cast<const __half2*>(&p[0]),
+                                                           *reinterpret_cast<const __half2*>(&p[1])),
+                                                   __hadd2(*reinterpret_cast<const __half2*>(&p[2]),
+                                                           *reinterpret_cast<const __half2*>(&p[3])));
                         const float part = __low2float(ph) + __high2float(ph);
                         acc[r][n] = fmaf(part, e8m0_value(sb[r][u]), acc[r][n]);
                     }

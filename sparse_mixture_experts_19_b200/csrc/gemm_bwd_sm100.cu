@@ -50,6 +50,24 @@ constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kMnBox = 64 * kBK * 2;  // one 64 x 64 bf16 box of an MN-major tile (8 KB)
+// Epilogue staging: each epilogue warp owns 4 KB for its 32 rows x 32 float32
+// columns (128 B per row), 16-byte chunk c of row r at r * 128 + ((c ^ (r %
+// 8)) * 16), so that both the row-wise writes (a lane per row) and the
+// column-wise reads (8 lanes per row) are free of bank conflicts, and each
+// global store instruction writes 4 rows x 128 contiguous bytes.
+constexpr int kEpiStageBytes = 32 * 128;
+constexpr size_t kEpiOff = (kStages * kStageBytes + 256 + 2 * (kMaxExperts + 2) * sizeof(int32_t) + 127) / 128 * 128;
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
 
 struct BwdArgs {
     int groups;
@@ -285,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(
     } else {
         // ------------------------------------------------ epilogue warps 2..5
         const int q = warp & 3;
-        const int r = q * 32 + lane;
+        const uint32_t stage = smem_u32(smem + kEpiOff) + (uint32_t)(q * kEpiStageBytes);
         uint32_t tc = 0;
         for (int64_t t = blockIdx.x; t < sc.total; t += gridDim.x, ++tc) {
             Tile ti;
@@ -294,38 +312,41 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(
             if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
             tc_fence_after();
             const uint32_t tq = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
-            // output row and the columns of this tile
-            float* dst = nullptr;
-            int ncols = 0;
+            // the columns of this tile, and the output row of tile row m
             const int c0 = out_col(a, sc, ti.n0);
-            if (a.n_split > 0)
-                ncols = (c0 < a.n_split ? a.n_split : a.N) - c0;
-            else
-                ncols = a.N - c0;
-            if (r < ti.rows) {
-                if (!a.kgroups) {
-                    dst = a.out0 + (ti.row0 + r) * (int64_t)a.ldo + c0;
-                } else {
-                    const int m = (int)ti.row0 + r;
-                    dst = m < a.m_split ? a.out0 + ((int64_t)ti.g * a.m_split + m) * a.N + c0
-                                        : a.out1 + ((int64_t)ti.g * (a.M - a.m_split) + (m - a.m_split)) * a.N + c0;
-                }
-            }
+            const int ncols = (a.n_split > 0 ? (c0 < a.n_split ? a.n_split : a.N) : a.N) - c0;
+            auto row_dst = [&](int m) -> float* {
+                if (m >= ti.rows) return nullptr;
+                if (!a.kgroups) return a.out0 + (ti.row0 + m) * (int64_t)a.ldo + c0;
+                const int mm = (int)ti.row0 + m;
+                return mm < a.m_split ? a.out0 + ((int64_t)ti.g * a.m_split + mm) * a.N + c0
+                                      : a.out1 + ((int64_t)ti.g * (a.M - a.m_split) + (mm - a.m_split)) * a.N + c0;
+            };
 #pragma unroll 1
-            for (int j0 = 0; j0 < kBN; j0 += 64) {
-                float v[64];
-                tmem_ld64(tq + j0, v);
-                if (dst) {
+            for (int j0 = 0; j0 < kBN; j0 += 32) {
+                float v[32];
+                tmem_ld32(tq + j0, v);
+                if (ti.nkb == 0) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int n = j0 + 4 * i;
-                        if (n < ncols) {
-                            float4 o = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                            if (ti.nkb == 0) o = make_float4(0.f, 0.f, 0.f, 0.f);
-                            *reinterpret_cast<float4*>(dst + n) = o;
-                        }
-                    }
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
                 }
+                // this lane's row into the warp's stage, then 4 rows per store
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(stage + (uint32_t)(lane * 128 + ((c ^ (lane & 7)) << 4)),
+                                 make_uint4(__float_as_uint(v[4 * c]), __float_as_uint(v[4 * c + 1]),
+                                            __float_as_uint(v[4 * c + 2]), __float_as_uint(v[4 * c + 3])));
+                __syncwarp();
+                const int cc = lane & 7;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = 4 * i + (lane >> 3);
+                    const uint4 w = ld_shared_v4(stage + (uint32_t)(rr * 128 + ((cc ^ (rr & 7)) << 4)));
+                    float* dst = row_dst(q * 32 + rr);
+                    const int n = j0 + 4 * cc;
+                    if (dst && n < ncols) *reinterpret_cast<uint4*>(dst + n) = w;
+                }
+                __syncwarp();
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
@@ -338,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(
     if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + 256 + 2 * (kMaxExperts + 2) * sizeof(int32_t);
+constexpr size_t kSmemBytes = 1024 + kEpiOff + 4 * kEpiStageBytes;
 
 // Rank-3 map of a bf16 tensor [depth][rows][inner]: K-major operands take
 // 64 x box_rows boxes, MN-major ones 64 x 64 boxes (64 contiguous M/N
