@@ -51,9 +51,11 @@ def parse_args():
     ap.add_argument("--workload", default="fine_grained_e256_layer")
     ap.add_argument("--T", type=int, default=0, help="override the token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=["forward", "route", "mxfp4", "backward"], default="forward",
+    ap.add_argument("--stage", choices=["forward", "route", "mxfp4", "backward", "ep"], default="forward",
                     help="route: time moe_route alone (only x and the router weights are allocated); "
-                         "mxfp4: moe_forward_mxfp4 at decode sizes; backward: moe_backward")
+                         "mxfp4: moe_forward_mxfp4 at decode sizes; backward: moe_backward; "
+                         "ep: each rank's expert-parallel compute on one GPU")
+    ap.add_argument("--shards", type=int, default=8, help="with --stage ep: the number of expert shards")
     ap.add_argument("--importance", action="store_true",
                     help="with --stage route: also time moe_route_importance (router importance as a side output)")
     ap.add_argument("--no-graph", action="store_true",
@@ -701,11 +703,49 @@ def run_backward_stage(args, wl):
                          "peak_kind": f"{pk_kind} bf16 dense, burst"}}
 
 
+def run_ep_stage(args, wl):
+    """Expert parallelism on one GPU: the routing once, then each of the N
+    ranks' compute (moe_forward_expert_shard over the whole batch with its
+    E/N experts, float32 partial output) timed alone, and the reduction of
+    the N partials (moe_reduce_partials).  The exchange between GPUs (an
+    all-reduce of the partials) is not timed: one GPU."""
+    import torch
+
+    moe, inp, d = _stage_setup(wl)
+    n = args.shards
+    cfg = moe.config(wl.T, wl.H, wl.I, wl.E, wl.k, wl.I_shared, wl.capacity_factor, "bf16")
+    ws = moe.workspace(cfg)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    moe.moe_route(cfg, d["x"], d["router_w"], d["router_b"], idx, w, ws)
+    parts = torch.empty((n, wl.T, wl.H), dtype=torch.float32, device="cuda")
+    shard_ms = []
+    for r in range(n):
+        e0, e1 = r * wl.E // n, (r + 1) * wl.E // n
+        shared = (d["ws_gate"], d["ws_up"], d["ws_down"]) if r == 0 else (None, None, None)
+        call = lambda: moe.moe_forward_expert_shard(cfg, d["x"], idx, w, e0, e1 - e0, d["w_gate"][e0:e1],
+                                                    d["w_up"][e0:e1], d["w_down"][e0:e1], *shared, parts[r],
+                                                    ws=ws)
+        shard_ms.append(_time_calls(args, call))
+        if moe.moe_get_device_status(cfg, ws) != 0:
+            raise SystemExit("device check flags set")
+    y = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    red_ms = _time_calls(args, lambda: moe.moe_reduce_partials(cfg, parts, y))
+    # a rank's step: its shard and the reduction (the slowest rank sets it)
+    step = max(shard_ms) + red_ms
+    return {"stage": "ep", "config": dict(config_of(wl), parallelism=f"ep{n}"), "shards": n,
+            "shard_ms": shard_ms, "reduce_ms": red_ms, "rank_step_ms_without_exchange": step,
+            "tokens_per_s_per_rank_without_exchange": wl.T / (step / 1e3),
+            "exchange_bytes_per_rank": n * wl.T * wl.H * 4,
+            "note": "one GPU: each rank's compute timed alone; the all-reduce of the float32 partials is not timed"}
+
+
 def main():
     args = parse_args()
     wl = workload(args)
     if args.stage != "forward":
-        run = {"route": run_route_stage, "mxfp4": run_mxfp4_stage, "backward": run_backward_stage}[args.stage]
+        run = {"route": run_route_stage, "mxfp4": run_mxfp4_stage, "backward": run_backward_stage,
+               "ep": run_ep_stage}[args.stage]
         print(json.dumps(run(args, wl)), flush=True)
         return
     world, rank, local = dist_setup(args)
