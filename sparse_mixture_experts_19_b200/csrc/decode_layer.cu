@@ -410,6 +410,16 @@ __device__ float group_absmax(const bf16* src, int n, bool l2_only, float* red, 
     return r;
 }
 
+// double -> unsigned 64-bit with the same order (-0 taken as +0, so that
+// equal doubles get equal keys), and back.
+__device__ __forceinline__ unsigned long long ordered_key64(double v) {
+    const unsigned long long u = (unsigned long long)__double_as_longlong(v == 0.0 ? 0.0 : v);
+    return (u >> 63) ? ~u : (u | (1ull << 63));
+}
+__device__ __forceinline__ double from_ordered_key64(unsigned long long k) {
+    return __longlong_as_double((long long)((k >> 63) ? (k & ~(1ull << 63)) : ~k));
+}
+
 // Part of an exact score x[t] . W_r[e] in fp64: the 16-byte chunks
 // [cb, ce) of the two rows, summed by one warp (every lane gets the sum).
 __device__ __forceinline__ double exact_dot_part(const bf16* x, const bf16* w, int cb, int ce) {
@@ -558,14 +568,18 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
                         be = e;
                     }
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    if (ov > bv || (ov == bv && oe < be)) {
-                        bv = ov;
-                        be = oe;
-                    }
+                {
+                    // warp arg-max over order-preserving 64-bit keys: the
+                    // largest high word, then the largest low word among the
+                    // lanes holding it, then the lowest expert index among
+                    // the lanes holding both (single-instruction reductions)
+                    const unsigned long long key = ordered_key64(bv);
+                    const unsigned hi = (unsigned)(key >> 32), lo = (unsigned)key;
+                    const unsigned mhi = __reduce_max_sync(0xffffffffu, hi);
+                    const unsigned mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+                    const bool top = hi == mhi && lo == mlo;
+                    be = (int)__reduce_min_sync(0xffffffffu, top ? (unsigned)be : 0xffffffffu);
+                    bv = from_ordered_key64(((unsigned long long)mhi << 32) | mlo);
                 }
                 if (j == 0) v0 = bv;
                 pv = bv;
