@@ -37,7 +37,9 @@
 //      CTA's output columns j in [H c / G, H (c+1) / G), while the gate/up
 //      warps stream the next groups.  So the down rows are read during the
 //      gate/up stream instead of after it, and no grid barrier separates
-//      the two.
+//      the two.  The gate/up warps, done with their rows, prefetch the last
+//      group's down rows of their CTA into L2 and then share that group's
+//      columns with the down warps.
 //   3. y[t][j] = bf16(sum over the token's slots in order of w * d, + the
 //      shared expert's d): y is bit-reproducible without atomics.
 #include <algorithm>

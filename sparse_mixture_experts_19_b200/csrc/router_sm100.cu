@@ -12,11 +12,13 @@
 //    TMEM (E padded to a multiple of 16; the padding rows of the weight box
 //    read as zero) and writes the float32 partial scores P_c[t, e].  The MMA
 //    warp's idle lanes also read every staged x row and router row from
-//    shared memory for their squared norms over the chunk.
-// 2. router_select_kernel (CUDA cores, a thread per token): the partials are
-//    summed in fp64 with the bias, the selection is made certain against a
-//    bound on the difference from the exact scores, the uncertain experts
-//    are rescored exactly, and the k selected experts are ordered exactly.
+//    shared memory for their squared norms over the chunk.  Two CTAs share
+//    an SM, so one's drain of its partials overlaps the other's MMAs.
+// 2. router_select_kernel (CUDA cores, 32 tokens per block): the partials
+//    are summed in float32 in chunk order with the bias, the selection is
+//    made certain against a bound on the difference from the exact scores,
+//    the uncertain experts are rescored exactly, and the k selected experts
+//    are ordered exactly.
 //
 // Bound.  Each partial score is a float32 tensor-core sum of at most
 // n = 4 * ceil(chunk / 64) MMA steps of 16 exact bf16 products.  Model of the
