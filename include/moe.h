@@ -232,11 +232,11 @@ moe_status_t moe_combine(const moe_config_t* cfg, const float* expert_out, const
  * rounded once to the layer dtype.
  *   y [T,H] (layer dtype).  Optional outputs (NULL to skip): topk_idx_out
  *   [T,top_k] int32, counts_out [E] and dropped_out [E] int32.
- * With T*top_k <= 8 (bf16) no rows are grouped: two weight-streaming
- * kernels read each selected expert's weight rows once and sum each
- * token's k weighted FFN outputs (then the shared expert's) in float32 in
- * slot order, rounded once; the routed outputs are not rounded to bf16
- * before that sum.
+ * With T*top_k <= 8 (bf16) no rows are grouped: one cooperative
+ * weight-streaming kernel reads each selected expert's weight rows once and
+ * sums each token's k weighted FFN outputs (then the shared expert's) in
+ * float32 in slot order, rounded once; the routed outputs are not rounded to
+ * bf16 before that sum.
  * y is bit-reproducible for given inputs (fixed summation order; the only
  * atomics are arrival counters that pick which warp does a fixed-order sum).
  */
@@ -372,9 +372,12 @@ moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, co
  * each block's 32 products are summed in f16 with the token vector scaled by
  * a power of two into f16's range, and the blocks' sums in float32; h is
  * rounded to bf16 between the two projections as in moe_forward.
- * Limits: T * top_k <= 8, no shared expert (I_shared = 0), H and I multiples
- * of 32; otherwise MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG before anything
- * is enqueued.  Outputs and errors otherwise as moe_forward.
+ * Limits: T * top_k <= 32 (gpt-oss-sized layers up to T = 8) with the
+ * kernel's shared memory within 200 KB (the token vectors, T*H*2 bytes, one
+ * expert's h vectors, T*I*2 bytes, and the partial dots), no shared expert
+ * (I_shared = 0), H and I multiples of 32; otherwise MOE_ERR_UNSUPPORTED /
+ * MOE_ERR_INVALID_ARG before anything is enqueued.  Outputs and errors
+ * otherwise as moe_forward.
  */
 moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const void* router_w, const float* router_b,
                                const uint8_t* w_gate_blocks, const uint8_t* w_gate_scales, const uint8_t* w_up_blocks,

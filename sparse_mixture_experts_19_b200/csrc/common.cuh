@@ -17,8 +17,9 @@ constexpr int kPermuteChunk = 2048;  // slots per histogram chunk in moe_permute
 constexpr int kWsAlign = 256;
 constexpr int kGemmTileRows = 128;  // rows per tile of the tcgen05 grouped GEMMs
 constexpr int64_t kNoAllocMaxSlots = 1 << 20;  // T*k limit of moe_permute_noalloc
-constexpr int kDecodeMaxSlots = 8;             // T*k limit of the decode FFN kernels
-constexpr int kDecodeCounters = 2 + kDecodeMaxSlots;  // decode layer: grid barrier + one per expert group
+constexpr int kDecodeMaxSlots = 8;             // T*k limit of the decode layer on bf16 experts
+constexpr int kDecodeMaxSlotsMx = 32;          // T*k limit of the decode layer on MXFP4 experts
+constexpr int kDecodeCounters = 2 + kDecodeMaxSlotsMx;  // decode layer: grid barrier + one per expert group
 constexpr int kRouterMaxSplits = 8;            // reduction chunks of the tensor-core router
 
 // Everything the kernels of one call need, carved out of the caller's workspace.
@@ -51,7 +52,7 @@ struct Plan {
     float* rt_part;       // tensor-core router: [splits, T, E] float32 partial scores
     float* rt_xn2;        // [splits, T] squared norms of the x rows over each chunk
     float* rt_wn2;        // [splits, E] squared norms of the router rows over each chunk
-    double* dec_scores;   // decode layer (S <= kDecodeMaxSlots): [T, E] router scores
+    double* dec_scores;   // decode layer (S <= kDecodeMaxSlotsMx): [T, E] router scores
     unsigned int* dec_bar;  // decode layer: [kDecodeCounters] arrival counters
     size_t bytes;         // total workspace bytes
 };
@@ -99,6 +100,8 @@ constexpr int64_t kDecodeRouterMaxMacs = int64_t(1) << 26;
 // kernel, y written directly; also writes counts and dropped, and
 // topk_idx_out when non-null.
 bool decode_ffn_eligible(const Plan& p);
+// The MXFP4 variant's size limit (T*k <= kDecodeMaxSlotsMx, shared memory).
+bool decode_mxfp4_eligible(const Plan& p);
 cudaError_t launch_decode_layer(const Plan& p, const void* x, const void* router_w, const float* router_b,
                                 const int32_t* topk_idx_in, const float* topk_w_in, int32_t* topk_idx_out,
                                 const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,

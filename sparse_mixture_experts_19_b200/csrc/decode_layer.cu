@@ -55,7 +55,8 @@ using namespace sm100;
 
 constexpr int kDlThreads = 512;
 constexpr int kDlWarps = kDlThreads / 32;
-constexpr int kDlMaxGroups = kDecodeMaxSlots + 1;  // distinct routed experts + the shared one
+constexpr int kDlMaxSlots = kDecodeMaxSlotsMx;     // slots of either variant
+constexpr int kDlMaxGroups = kDlMaxSlots + 1;      // distinct routed experts + the shared one
 constexpr int kDlBatch = 4;                        // token vectors per pass over a weight row
 constexpr int kDlUnroll = 6;                       // 16-byte chunks per lane in flight, per row
 constexpr int kDlMaxCols = 64;                     // output columns per CTA in phase 3 (H <= 64 * grid)
@@ -101,10 +102,10 @@ struct DlPlan {
     int ng;
     int gexp[kDlMaxGroups];                  // expert id; E marks the shared expert
     int gcnt[kDlMaxGroups];                  // vectors of the group
-    int gvec[kDlMaxGroups][kDecodeMaxSlots]; // routed: slot s; shared: token t
-    int e_of[kDecodeMaxSlots];
-    int kept[kDecodeMaxSlots];
-    float wslot[kDecodeMaxSlots];
+    int gvec[kDlMaxGroups][kDlMaxSlots];     // routed: slot s; shared: token t
+    int e_of[kDlMaxSlots];
+    int kept[kDlMaxSlots];
+    float wslot[kDlMaxSlots];
 };
 
 __device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
@@ -499,8 +500,8 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
     __shared__ DlPlan pl;
     __shared__ int ok_s;
     __shared__ float red[2 * kDlWarps];        // block reductions (the down warps use the second half)
-    __shared__ float inv_sx[kDecodeMaxSlots];  // MXFP4: 1 / staging scale of each token vector
-    __shared__ float inv_sh[kDecodeMaxSlots];  // MXFP4: 1 / staging scale of each h vector
+    __shared__ float inv_sx[kDlMaxSlots];      // MXFP4: 1 / staging scale of each token vector
+    __shared__ float inv_sh[kDlMaxSlots];      // MXFP4: 1 / staging scale of each h vector
     __shared__ double dpart[kDlWarps];         // parts of the router scores
     __shared__ int up_done[kDlMaxGroups];      // gate/up warps done with each group
     __shared__ int down_ok;
@@ -662,9 +663,9 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
     const uint64_t pol_dn = policy_evict_first();
     // Down items of group g (its h rows staged at hsm): column pairs q =
     // first, first + step, ... of this CTA's columns.  A warp takes two
-    // adjacent columns at a time (bf16 rows): their down rows share the
-    // group's h vectors, and twice the loads are in flight per pass.
-    constexpr int kCols = kMx ? 1 : 2;
+    // adjacent columns at a time: their down rows share the group's h
+    // vectors, and twice the loads are in flight per pass.
+    constexpr int kCols = 2;
     const int cp = (cols + kCols - 1) / kCols;
     auto down_items = [&](int g, int first, int step) {
         const bool sh = pl.gexp[g] == a.E;
@@ -891,12 +892,17 @@ int64_t dl_smem_bytes(const Plan& p, int grid) {
 
 }  // namespace
 
-bool decode_ffn_eligible(const Plan& p) {
-    if (!p.bf16 || p.S < 1 || p.S > kDecodeMaxSlots) return false;
+namespace {
+bool decode_fits(const Plan& p, int max_slots) {
+    if (!p.bf16 || p.S < 1 || p.S > max_slots) return false;
     const int grid = device_sm_count();
     if ((p.H + grid - 1) / grid > kDlMaxCols) return false;
     return dl_smem_bytes(p, grid) <= kDlSmemMax;
 }
+}  // namespace
+
+bool decode_ffn_eligible(const Plan& p) { return decode_fits(p, kDecodeMaxSlots); }
+bool decode_mxfp4_eligible(const Plan& p) { return decode_fits(p, kDecodeMaxSlotsMx); }
 
 namespace {
 
@@ -979,7 +985,7 @@ cudaError_t launch_decode_layer(const Plan& p, const void* x, const void* router
 cudaError_t launch_decode_layer_mxfp4(const Plan& p, const void* x, const void* router_w, const float* router_b,
                                       int32_t* topk_idx_out, const uint8_t* const (&mx)[6], void* y, int32_t* counts,
                                       int32_t* dropped, cudaStream_t st) {
-    if (!decode_ffn_eligible(p) || p.Is > 0 || p.H % 32 || p.I % 32) return cudaErrorInvalidValue;
+    if (!decode_mxfp4_eligible(p) || p.Is > 0 || p.H % 32 || p.I % 32) return cudaErrorInvalidValue;
     DlArgs a = base_args(p, x, router_w, router_b, nullptr, nullptr, topk_idx_out, y, counts, dropped);
     a.mgb = mx[0];
     a.mgs = mx[1];

@@ -138,7 +138,7 @@ static void make_plan(const moe_config_t* c, void* ws, Plan* p) {
     p->rt_part = (float*)take(tc_router ? sizeof(float) * kRouterMaxSplits * p->T * p->E : 0);
     p->rt_xn2 = (float*)take(tc_router ? sizeof(float) * kRouterMaxSplits * p->T : 0);
     p->rt_wn2 = (float*)take(tc_router ? sizeof(float) * kRouterMaxSplits * p->E : 0);
-    const bool dec = p->S <= kDecodeMaxSlots;
+    const bool dec = p->S <= kDecodeMaxSlotsMx;
     p->dec_scores = (double*)take(dec ? sizeof(double) * p->T * p->E : 0);
     p->dec_bar = (unsigned int*)take(dec ? kDecodeCounters * sizeof(unsigned int) : 0);
     p->bytes = off;
@@ -590,9 +590,9 @@ moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const voi
         if (dropped_out) CUDA_TRY(cudaMemsetAsync(dropped_out, 0, sizeof(int32_t) * p.E, st), "memset");
         return MOE_OK;
     }
-    if (!decode_ffn_eligible(p))
+    if (!decode_mxfp4_eligible(p))
         return fail(MOE_ERR_UNSUPPORTED, "moe_forward_mxfp4 serves T*top_k <= %d routed slots (got %lld)",
-                    kDecodeMaxSlots, (long long)p.S);
+                    kDecodeMaxSlotsMx, (long long)p.S);
     REQUIRE_PTR(x);
     REQUIRE_PTR(router_w);
     OPTIONAL_PTR(router_b);

@@ -25,6 +25,8 @@ from parity_util import TOL, cap_of, check_selection, host_f64, rowwise_rel_err,
 CASES = [
     mi.GPTOSS.with_(name="gpt_oss_mxfp4_T1", T=1),
     mi.GPTOSS.with_(name="gpt_oss_mxfp4_T2", T=2),
+    mi.GPTOSS.with_(name="gpt_oss_mxfp4_T8", T=8),  # 32 slots, the size limit
+    mi.Workload("mxfp4_ragged_T7", T=7, H=352, I=160, E=24, k=4),  # 28 slots, 3 columns per CTA with a tail
     mi.Workload("mxfp4_small_cap", T=2, H=256, I=128, E=8, k=4, capacity_factor=0.5),
     mi.Workload("mxfp4_one_expert", T=8, H=128, I=96, E=1, k=1),
     mi.Workload("mxfp4_e256", T=1, H=512, I=256, E=256, k=8, zipf_s=1.1),
@@ -101,3 +103,4 @@ def test_mxfp4_validates():
     assert call(_cfg(H=264)) == 1 and "32" in moe_pkg.moe_last_error()
     assert call(_cfg(dtype="f32")) == 2
     assert call(_cfg(T=0)) == 0
+    assert call(_cfg(T=9)) == 2 and "32" in moe_pkg.moe_last_error()  # 36 slots
