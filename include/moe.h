@@ -354,9 +354,17 @@ moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, co
                                       int32_t* dropped_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_mxfp4_workspace_size -- bytes of workspace moe_forward_mxfp4 needs for
+ * cfg: moe_workspace_size(cfg), plus the bf16 copies of the expert weights
+ * (3*E*H*I*2 bytes, 256-aligned) when the size takes the dequantizing tile
+ * path.  0 for an invalid cfg (see moe_last_error).
+ */
+size_t moe_mxfp4_workspace_size(const moe_config_t* cfg);
+
+/*
  * moe_forward_mxfp4 -- moe_forward with the routed experts' weights in the
- * MXFP4 format of the OCP Microscaling (MX) v1.0 specification, for decode
- * sizes ("Mixture of Experts (MoEs) in Transformers", section From Dense to
+ * MXFP4 format of the OCP Microscaling (MX) v1.0 specification
+ * ("Mixture of Experts (MoEs) in Transformers", section From Dense to
  * Sparse: the gpt-oss generation speed is set by the bytes of the active
  * parameters, and native mxfp4 kernels would raise it further).  An element
  * is FP4 E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa bit); each
@@ -372,11 +380,18 @@ moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, co
  * each block's 32 products are summed in f16 with the token vector scaled by
  * a power of two into f16's range, and the blocks' sums in float32; h is
  * rounded to bf16 between the two projections as in moe_forward.
- * Limits: T * top_k <= 32 (gpt-oss-sized layers up to T = 8) with the
- * kernel's shared memory within 200 KB (the token vectors, T*H*2 bytes, one
- * expert's h vectors, T*I*2 bytes, and the partial dots), no shared expert
- * (I_shared = 0), H and I multiples of 32; otherwise MOE_ERR_UNSUPPORTED /
- * MOE_ERR_INVALID_ARG before anything is enqueued.  Outputs and errors
+ * Two paths by size.  T * top_k <= 32 (gpt-oss-sized layers up to T = 8)
+ * with the decode kernel's shared memory within 200 KB (the token vectors,
+ * T*H*2 bytes, one expert's h vectors, T*I*2 bytes, and the partial dots):
+ * one weight-streaming kernel reads the MXFP4 rows themselves; the workspace
+ * is moe_workspace_size(cfg).  Larger: the gate, up and down weights are
+ * dequantized to bf16 (exact: every value e * 2^(s-127) fits bf16 down to
+ * 2^-133; above bf16's range it becomes +-inf) into the workspace after
+ * moe_forward's scratch, then moe_forward's tile path runs on them; the
+ * workspace must hold moe_mxfp4_workspace_size(cfg) bytes (3*E*H*I*2 more),
+ * else MOE_ERR_WORKSPACE.  No shared expert (I_shared = 0), H and I
+ * multiples of 32; otherwise MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG.
+ * Every error is returned before anything is enqueued.  Outputs and errors
  * otherwise as moe_forward.
  */
 moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const void* router_w, const float* router_b,

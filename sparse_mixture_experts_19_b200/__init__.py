@@ -43,6 +43,7 @@ class moe_trace_record_t(ctypes.Structure):
 _P = ctypes.c_void_p
 _SIGS = {
     "moe_workspace_size": ([ctypes.POINTER(moe_config_t)], ctypes.c_size_t),
+    "moe_mxfp4_workspace_size": ([ctypes.POINTER(moe_config_t)], ctypes.c_size_t),
     "moe_capacity": ([ctypes.POINTER(moe_config_t)], ctypes.c_int64),
     "moe_route": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_route_importance": ([ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
@@ -279,12 +280,27 @@ def moe_forward_mxfp4(cfg, x, router_w, router_b, w_gate_blocks, w_gate_scales, 
                       w_down_blocks, w_down_scales, y, topk_idx_out=None, counts_out=None, dropped_out=None, ws=None,
                       stream=None):
     """moe_forward with MXFP4 routed experts (uint8 blocks [E, rows, K/32, 16]
-    and scales [E, rows, K/32]); decode sizes, T * top_k <= 8."""
+    and scales [E, rows, K/32]).  ws: moe_mxfp4_workspace_size(cfg) bytes
+    (mxfp4_workspace); up to 32 routed slots that is moe_workspace_size."""
     p, n = _ws(ws)
     _check(load().moe_forward_mxfp4(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(w_gate_blocks),
                                     _ptr(w_gate_scales), _ptr(w_up_blocks), _ptr(w_up_scales), _ptr(w_down_blocks),
                                     _ptr(w_down_scales), _ptr(y), _ptr(topk_idx_out), _ptr(counts_out),
                                     _ptr(dropped_out), p, n, _stream(stream)))
+
+
+def moe_mxfp4_workspace_size(cfg) -> int:
+    n = load().moe_mxfp4_workspace_size(ctypes.byref(cfg))
+    if n == 0:
+        raise MoeError(1, load().moe_last_error().decode())
+    return n
+
+
+def mxfp4_workspace(cfg: moe_config_t, device="cuda"):
+    """A zeroed workspace for moe_forward_mxfp4 (see workspace)."""
+    import torch
+
+    return torch.zeros(moe_mxfp4_workspace_size(cfg), dtype=torch.uint8, device=device)
 
 
 def moe_backward_workspace_size(cfg) -> int:

@@ -113,6 +113,10 @@ cudaError_t launch_decode_layer(const Plan& p, const void* x, const void* router
 cudaError_t launch_decode_layer_mxfp4(const Plan& p, const void* x, const void* router_w, const float* router_b,
                                       int32_t* topk_idx_out, const uint8_t* const (&mx)[6], void* y, int32_t* counts,
                                       int32_t* dropped, cudaStream_t st);
+// MXFP4 rows (blocks [rows, K/32, 16], scales [rows, K/32]; K a multiple of
+// 32) -> bf16 rows [rows, K] at out (16-byte aligned), exact within bf16's range.
+cudaError_t launch_mxfp4_dequant(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int K, void* out,
+                                 cudaStream_t st);
 cudaError_t launch_permute(const Plan& p, const int32_t* topk_idx, int32_t* counts,
                            int32_t* offsets, int32_t* perm_rows, int32_t* row_of,
                            int32_t* dropped, cudaStream_t st);

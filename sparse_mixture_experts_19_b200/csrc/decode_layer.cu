@@ -45,6 +45,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "mxfp4.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
 
@@ -237,24 +238,6 @@ __device__ __forceinline__ void row_dots_n(const uint4* const (&rows)[NR], int K
 // stays in range), then widened to float32, scaled by the block's 2^(s-127)
 // and accumulated in float32.
 constexpr int kMxUnroll = 4;  // blocks per lane in flight, per row
-
-// Four bytes of E2M1 pairs -> four f16x2 values (byte j -> elements 2j, 2j+1).
-__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&o)[4]) {
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
-        : "r"(w));
-}
-
-// 2^(s - 127) for an E8M0 byte: s = 0 is the subnormal 2^-127, s = 255 NaN.
-__device__ __forceinline__ float e8m0_value(uint32_t s) {
-    if (s == 255u) return __int_as_float(0x7fc00000);
-    return s == 0u ? __int_as_float(0x00400000) : __int_as_float((int)(s << 23));
-}
 
 __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;

@@ -570,6 +570,21 @@ moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, co
                                  dropped, st);
 }
 
+// Bytes of the bf16 copies of the gate, up and down weights that the MXFP4
+// tile path makes in the workspace after moe_forward's own scratch; 0 when
+// the decode kernel serves the size.
+static size_t mxfp4_dequant_bytes(const Plan& p) {
+    if (p.T == 0 || decode_mxfp4_eligible(p)) return 0;
+    return align_up((size_t)3 * p.E * p.H * p.I * 2);
+}
+
+size_t moe_mxfp4_workspace_size(const moe_config_t* cfg) {
+    if (check_config(cfg) != MOE_OK) return 0;
+    Plan p;
+    make_plan(cfg, nullptr, &p);
+    return p.bytes + mxfp4_dequant_bytes(p);
+}
+
 moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const void* router_w, const float* router_b,
                                const uint8_t* w_gate_blocks, const uint8_t* w_gate_scales, const uint8_t* w_up_blocks,
                                const uint8_t* w_up_scales, const uint8_t* w_down_blocks, const uint8_t* w_down_scales,
@@ -590,9 +605,12 @@ moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const voi
         if (dropped_out) CUDA_TRY(cudaMemsetAsync(dropped_out, 0, sizeof(int32_t) * p.E, st), "memset");
         return MOE_OK;
     }
-    if (!decode_mxfp4_eligible(p))
-        return fail(MOE_ERR_UNSUPPORTED, "moe_forward_mxfp4 serves T*top_k <= %d routed slots (got %lld)",
-                    kDecodeMaxSlotsMx, (long long)p.S);
+    const size_t dq_bytes = mxfp4_dequant_bytes(p);
+    if (ws_bytes < p.bytes + dq_bytes)
+        return fail(MOE_ERR_WORKSPACE,
+                    "moe_forward_mxfp4 with %lld routed slots dequantizes the experts into the workspace: it needs "
+                    "moe_mxfp4_workspace_size(cfg) = %zu bytes, got %zu",
+                    (long long)p.S, p.bytes + dq_bytes, ws_bytes);
     REQUIRE_PTR(x);
     REQUIRE_PTR(router_w);
     OPTIONAL_PTR(router_b);
@@ -605,9 +623,24 @@ moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const voi
     const uint8_t* mx[6] = {w_gate_blocks, w_gate_scales, w_up_blocks, w_up_scales, w_down_blocks, w_down_scales};
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
-    CUDA_TRY(launch_decode_layer_mxfp4(p, x, router_w, router_b, topk_idx_out, mx, y, counts, dropped, st),
-             "decode_layer_mxfp4");
-    return MOE_OK;
+    if (dq_bytes == 0) {
+        // decode sizes: routing, the expert FFNs on the MXFP4 rows and the
+        // combine in one weight-streaming kernel
+        CUDA_TRY(launch_decode_layer_mxfp4(p, x, router_w, router_b, topk_idx_out, mx, y, counts, dropped, st),
+                 "decode_layer_mxfp4");
+        return MOE_OK;
+    }
+    // more slots: the weights dequantized (exactly) to bf16 in the workspace,
+    // then moe_forward's routing, grouping, tcgen05 grouped GEMMs and combine
+    bf16* wg = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + p.bytes);
+    bf16* wu = wg + p.E * p.I * p.H;
+    bf16* wd = wu + p.E * p.I * p.H;
+    CUDA_TRY(launch_mxfp4_dequant(mx[0], mx[1], p.E * p.I, (int)p.H, wg, st), "mxfp4_dequant");
+    CUDA_TRY(launch_mxfp4_dequant(mx[2], mx[3], p.E * p.I, (int)p.H, wu, st), "mxfp4_dequant");
+    CUDA_TRY(launch_mxfp4_dequant(mx[4], mx[5], p.E * p.H, (int)p.I, wd, st), "mxfp4_dequant");
+    int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
+    CUDA_TRY(run_router(p, x, router_w, router_b, idx, p.topk_w, st), "router");
+    return forward_after_routing(p, x, idx, wg, wu, wd, nullptr, nullptr, nullptr, y, counts, dropped, st);
 }
 
 moe_status_t moe_reduce_partials(const moe_config_t* cfg, const float* partials, int32_t n, void* y,
