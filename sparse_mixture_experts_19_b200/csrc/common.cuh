@@ -147,6 +147,15 @@ cudaError_t launch_gateup_sm100(const Plan& p, const void* x, const void* w_gate
                                 const void* ws_gate, const void* ws_up, cudaStream_t st);
 cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_down, int mode,
                               void* out, cudaStream_t st);
+// The same GEMMs with the routed experts' weights in MXFP4 (E2M1 code blocks
+// [E, N, K/32, 16] and E8M0 scales [E, N, K/32], K = H for gate/up, I for
+// down), converted to bf16 in shared memory: bf16 layer, no shared expert,
+// H and I multiples of 32 and at most 3072 (mx_gemm_eligible).
+bool mx_gemm_eligible(const Plan& p);
+cudaError_t launch_gateup_mx_sm100(const Plan& p, const uint8_t* gate_blocks, const uint8_t* gate_scales,
+                                   const uint8_t* up_blocks, const uint8_t* up_scales, cudaStream_t st);
+cudaError_t launch_down_mx_sm100(const Plan& p, const uint8_t* down_blocks, const uint8_t* down_scales, int mode,
+                                 void* out, cudaStream_t st);
 // y[t] = sum_j rows[row_of[t,j]] (j in order, dropped slots skipped) + rows[S + t]
 // (shared), summed in float32 and rounded once to the layer dtype.
 cudaError_t launch_combine_rows(const Plan& p, const void* rows, const int32_t* row_of, void* y,

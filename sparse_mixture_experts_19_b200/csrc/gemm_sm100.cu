@@ -33,7 +33,10 @@
 // the CTA unwinds and frees its TMEM.
 #include <algorithm>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
+#include "mxfp4.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
 
@@ -660,6 +663,395 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
     if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
+// ---------------------------------------------------- MXFP4 weights (B)
+// The same grouped GEMMs with the expert weights in MXFP4 (E2M1 codes with
+// one E8M0 scale per 32 along K).  The codes of a k-step (256 rows x 64 K =
+// 8 KB, a quarter of the bf16 bytes) arrive by TMA into a ring of 8 slots;
+// eight converter warps turn them into the bf16 B tile in shared memory, in
+// the 128-byte-swizzled K-major layout the MMA reads (chunk c of row r at
+// r*128 + ((c ^ r%8) * 16)), and the MMA runs as on bf16 weights.  Three
+// rings, each as deep as it needs to be: A tiles (3 x 16 KB, TMA), converted
+// B tiles (2 x 32 KB) and codes (8 x 8 KB): the codes ring keeps 64 KB of
+// weight reads in flight per SM; a producer warp of its own refills a codes
+// slot as soon as the converters have read it.  The conversion is integer
+// work plus one bf16 multiply per two elements (see mx_chunk_to_bf16): the
+// float conversion instructions run at a fraction of the ALU rate.  Every
+// converted value e * 2^(s-127) is exact in bf16 (normal or subnormal;
+// above bf16's range it becomes +-inf), so the products are those of the
+// dequantized weights.  A tile's scale bytes (its
+// rows x K/32, contiguous per 128 rows) are copied into shared memory when
+// the tile starts; K <= 32 * kMxMaxScales.
+constexpr int kMxAStages = 3;
+constexpr int kMxBStages = 2;
+constexpr int kMxCStages = 8;
+constexpr int kMxCodeBytes = kBRows * kBK / 2;  // 8 KB of codes per k-step
+constexpr int kMxMaxScales = 96;                 // scale bytes per row a tile holds: K <= 3072
+constexpr int kMxConvWarps = 8;
+constexpr int kMxConvThreads = kMxConvWarps * 32;
+constexpr int kMxCodeWarp = (kThreads + kMxConvThreads) / 32;  // the codes producer
+constexpr int kMxThreads = kThreads + kMxConvThreads + 32;
+constexpr size_t kMxBOff = (size_t)kMxAStages * kABytes;
+constexpr size_t kMxCOff = kMxBOff + (size_t)kMxBStages * kBBytes;
+constexpr size_t kMxBarOff = kMxCOff + (size_t)kMxCStages * kMxCodeBytes;
+constexpr size_t kMxTablesOff = kMxBarOff + 512;
+constexpr size_t kMxScaleOff = (kMxTablesOff + sizeof(Tables) + 127) / 128 * 128;
+constexpr size_t kMxEpiStageOff = (kMxScaleOff + (size_t)kBRows * kMxMaxScales + 127) / 128 * 128;
+constexpr size_t kMxSmemBytes = kMxEpiStageOff + 4 * kEpiStageBytes + 1024;
+static_assert(kMxSmemBytes <= 227 * 1024, "MXFP4 GEMM shared memory");
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Named barrier of n threads that also returns whether every one of them
+// passed v = true.
+__device__ __forceinline__ bool named_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Eight E2M1 codes (byte q: element 2q in the low nibble, 2q+1 in the high)
+// with E8M0 scale byte s -> eight bf16 values e * 2^(s-127) in o[0..3].
+// A nibble's sign bit moved to bit 15 and its three exponent/mantissa bits
+// to bits 8..6 form the bf16 of e * 2^-126 exactly (exponent field 0 makes
+// the codes 0 and 0.5 the subnormals 0 and 2^-127); one rounding multiply
+// by 2^(s-1) (two, by 2^126 then 2^(s-127), when 2^(s-1) exceeds bf16's
+// range) then gives e * 2^(s-127), exact wherever bf16 holds it.
+__device__ __forceinline__ void mx_chunk_to_bf16(uint32_t w, uint32_t s, uint32_t (&o)[4]) {
+    uint32_t pre = 0u, sc;
+    if (s <= 128u) {
+        sc = ((s + 126u) << 7) * 0x10001u;  // 2^(s-1)
+    } else if (s == 255u) {
+        sc = 0x7fc07fc0u;  // NaN
+    } else {
+        pre = 0x7e807e80u;  // 2^126
+        sc = (s << 7) * 0x10001u;  // 2^(s-127)
+    }
+    const uint32_t lo = w & 0x0f0f0f0fu, hi = (w >> 4) & 0x0f0f0f0fu;
+    // selector q: byte q of lo, byte q of hi into the two halves, the other
+    // bytes the (zero) sign of a nibble byte
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t sel = (uint32_t)q | ((8u | q) << 4) | ((4u + q) << 8) | ((12u + q) << 12);
+        const uint32_t t = prmt(lo, hi, sel);
+        uint32_t v = ((t & 0x00080008u) << 12) | ((t & 0x00070007u) << 6);
+        if (pre) v = mul_bf16x2(v, pre);
+        o[q] = mul_bf16x2(v, sc);
+    }
+}
+
+struct MxArgs {
+    const uint8_t* sc0;  // scales of the B rows: gate / down [E, N, K/32]
+    const uint8_t* sc1;  // up [E, N, K/32] (gate/up only)
+};
+
+// The k-steps of this CTA's tiles in order: (tile, k-step) of step `it`.
+struct StepCursor {
+    int64_t t;
+    int kb, nkb;
+    TileInfo ti;
+};
+
+__device__ __forceinline__ bool cursor_start(StepCursor& c, const Tables& tb, const Sched& sc, const GemmArgs& a,
+                                             int BN) {
+    c.t = blockIdx.x;
+    c.kb = 0;
+    if (c.t >= sc.total) return false;
+    decode_tile(c.t, tb, sc, a, BN, c.ti);
+    c.nkb = (c.ti.K + kBK - 1) / kBK;
+    return true;
+}
+
+__device__ __forceinline__ bool cursor_next(StepCursor& c, const Tables& tb, const Sched& sc, const GemmArgs& a,
+                                            int BN) {
+    if (++c.kb < c.nkb) return true;
+    c.t += gridDim.x;
+    c.kb = 0;
+    if (c.t >= sc.total) return false;
+    decode_tile(c.t, tb, sc, a, BN, c.ti);
+    c.nkb = (c.ti.K + kBK - 1) / kBK;
+    return true;
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAsm,
+    const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1, const GemmArgs a,
+    const MxArgs mxa) {
+    constexpr int BN = kGateUp ? kBRows / 2 : kBRows;
+    extern __shared__ uint8_t smem_raw[];
+    // aligned by pointer arithmetic, so that accesses through it stay shared-memory accesses
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* afull = reinterpret_cast<uint64_t*>(smem + kMxBarOff);
+    uint64_t* aempty = afull + kMxAStages;
+    uint64_t* bfull = aempty + kMxAStages;   // converted B tile ready (converters)
+    uint64_t* bempty = bfull + kMxBStages;   // B tile consumed (MMA)
+    uint64_t* cfull = bempty + kMxBStages;   // codes landed (TMA)
+    uint64_t* cempty = cfull + kMxCStages;   // codes slot read (converters)
+    uint64_t* tfull = cempty + kMxCStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    Tables* tb = reinterpret_cast<Tables*>(smem + kMxTablesOff);
+    uint8_t* sscale = smem + kMxScaleOff;
+    const uint32_t epi_stage = smem_u32(smem + kMxEpiStageOff) + (uint32_t)(((threadIdx.x / 32) & 3) * kEpiStageBytes);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int i = threadIdx.x; i < a.E + 2; i += kMxThreads) tb->off[i] = a.offsets[i];
+    for (int i = threadIdx.x; i < a.E + 1; i += kMxThreads) tb->mtp[i] = a.mtile_prefix[i];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kMxAStages; ++s) {
+            mbar_init(&afull[s], 1);
+            mbar_init(&aempty[s], 1);
+        }
+        for (int s = 0; s < kMxBStages; ++s) {
+            mbar_init(&bfull[s], 1);
+            mbar_init(&bempty[s], 1);
+        }
+        for (int s = 0; s < kMxCStages; ++s) {
+            mbar_init(&cfull[s], 1);
+            mbar_init(&cempty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], kEpiThreads);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) tma_prefetch_map(&tmA);
+    if (warp == kMxCodeWarp && lane == 0) {
+        tma_prefetch_map(&tmC0);
+        if (kGateUp) tma_prefetch_map(&tmC1);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    Sched sc;
+    sc.E = a.E;
+    sc.nb_r = (a.N + BN - 1) / BN;
+    sc.nb_s = 0;
+    sc.mt_s = 0;
+    sc.gm_r = band_tiles(a.K, kBM);
+    sc.gm_s = 1;
+    sc.routed_tiles = (int64_t)tb->mtp[a.E] * sc.nb_r;
+    sc.total = sc.routed_tiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer of A
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+                TileInfo ti;
+                decode_tile(t, *tb, sc, a, BN, ti);
+                const bool small = ti.rows <= kSmallRows;
+                const CUtensorMap* mA = small ? &tmAsm : &tmA;
+                const uint32_t a_tx = small ? kSmallABytes : kABytes;
+                const int nkb = (ti.K + kBK - 1) / kBK;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kMxAStages;
+                    const uint32_t ph = (it / kMxAStages) & 1;
+                    if (!wait_or_abort(&aempty[s], ph ^ 1, abort_flag, a.flags)) break;
+                    mbar_arrive_expect_tx(&afull[s], a_tx);
+                    tma_load_3d(smem + s * kABytes, mA, &afull[s], kb * kBK, ti.arow, 0);
+                }
+            }
+            // never leave with copies in flight (bounded waits)
+            for (uint32_t j = (it > (uint32_t)kMxAStages ? it - kMxAStages : 0); j < it; ++j)
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&afull[j % kMxAStages], (j / kMxAStages) & 1);
+                     ++i) {
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            for (int64_t t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x, ++tc) {
+                TileInfo ti;
+                decode_tile(t, *tb, sc, a, BN, ti);
+                const int nkb = (ti.K + kBK - 1) / kBK;
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!wait_or_abort(&tempty[acc], aph ^ 1, abort_flag, a.flags)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * kAccCols;
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int sa = it % kMxAStages, sb = it % kMxBStages;
+                    if (!wait_or_abort(&afull[sa], (it / kMxAStages) & 1, abort_flag, a.flags) ||
+                        !wait_or_abort(&bfull[sb], (it / kMxBStages) & 1, abort_flag, a.flags)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + sa * kABytes);
+                    const uint32_t b0 = smem_u32(smem + kMxBOff + sb * kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_bf16(d, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), kIdesc,
+                                 (kb | kk) != 0);
+                    mma_commit(&aempty[sa]);
+                    mma_commit(&bempty[sb]);
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+            }
+            mma_commit(drain);
+            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(drain, 0); ++i) {
+            }
+        }
+    } else if (warp < kThreads / 32) {
+        // ------------------------------------------------ epilogue warps 2..5
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        uint32_t tc = 0;
+        for (int64_t t = blockIdx.x; t < sc.total; t += gridDim.x, ++tc) {
+            TileInfo ti;
+            decode_tile(t, *tb, sc, a, BN, ti);
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
+            tc_fence_after();
+            epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r, epi_stage);
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+        }
+    } else if (warp == kMxCodeWarp) {
+        // ------------------------------------------------ TMA producer of the codes
+        if (lane == 0) {
+            StepCursor c{};
+            uint32_t it = 0;
+            for (bool more = cursor_start(c, *tb, sc, a, BN); more && !*abort_flag;
+                 more = cursor_next(c, *tb, sc, a, BN), ++it) {
+                const int s = it % kMxCStages;
+                if (!wait_or_abort(&cempty[s], ((it / kMxCStages) & 1) ^ 1, abort_flag, a.flags)) break;
+                uint8_t* dst = smem + kMxCOff + s * kMxCodeBytes;
+                mbar_arrive_expect_tx(&cfull[s], kMxCodeBytes);
+                if (kGateUp) {
+                    tma_load_3d(dst, &tmC0, &cfull[s], c.kb * (kBK / 2), c.ti.n0, c.ti.e);
+                    tma_load_3d(dst + kMxCodeBytes / 2, &tmC1, &cfull[s], c.kb * (kBK / 2), c.ti.n0, c.ti.e);
+                } else {
+                    tma_load_3d(dst, &tmC0, &cfull[s], c.kb * (kBK / 2), c.ti.n0, c.ti.e);
+                }
+            }
+            // never leave with copies in flight (bounded waits)
+            for (uint32_t j = (it > (uint32_t)kMxCStages ? it - kMxCStages : 0); j < it; ++j)
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&cfull[j % kMxCStages], (j / kMxCStages) & 1);
+                     ++i) {
+                }
+        }
+    } else {
+        // ------------------------------------------------ converter warps 6..13
+        // Thread ct converts chunk j = ct % 8 (8 elements) of rows ct / 8 + 32 i:
+        // a warp reads 4 rows x 32 bytes of codes and writes 4 rows x 128 bytes.
+        const int ct = threadIdx.x - kThreads;
+        const int j = ct & 7, r0 = ct >> 3;
+        const int nsb = a.K / 32;  // scale bytes per row
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < sc.total && ok; t += gridDim.x) {
+            TileInfo ti;
+            decode_tile(t, *tb, sc, a, BN, ti);
+            // the tile's scale bytes -> sscale[row][nsb] (rows past N left as
+            // they are: their codes are zeros and their columns are not stored)
+            named_and(2, kMxConvThreads, true);  // every converter is done with the previous tile's
+            {
+                // every load of the copy issued before its stores (one round
+                // trip per tile, not one per word)
+                constexpr int kHalf = kGateUp ? kBRows / 2 : kBRows;
+                constexpr int kWords = kHalf * kMxMaxScales / 4 / kMxConvThreads;  // per thread and source
+                const int bytes = min(kHalf, ti.N - ti.n0) * nsb;  // 32 | N - n0, so 4 | bytes
+#pragma unroll
+                for (int src = 0; src < (kGateUp ? 2 : 1); ++src) {
+                    const uint8_t* g = (src ? mxa.sc1 : mxa.sc0) + ((int64_t)ti.e * ti.N + ti.n0) * nsb;
+                    uint8_t* d = sscale + src * kHalf * nsb;
+                    if (((uintptr_t)g & 3) == 0) {  // 32 | N and 128 | n0 keep g word-aligned if the array is
+                        uint32_t v[kWords];
+#pragma unroll
+                        for (int u = 0; u < kWords; ++u) {
+                            const int w = ct + u * kMxConvThreads;
+                            v[u] = w < bytes / 4 ? __ldg(reinterpret_cast<const uint32_t*>(g) + w) : 0u;
+                        }
+#pragma unroll
+                        for (int u = 0; u < kWords; ++u) {
+                            const int w = ct + u * kMxConvThreads;
+                            if (w < bytes / 4) reinterpret_cast<uint32_t*>(d)[w] = v[u];
+                        }
+                    } else {
+                        for (int b = ct; b < bytes; b += kMxConvThreads) d[b] = __ldg(g + b);
+                    }
+                }
+            }
+            named_and(2, kMxConvThreads, true);
+            const int nkb = (ti.K + kBK - 1) / kBK;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int cs = it % kMxCStages, bs = it % kMxBStages;
+                const bool got = wait_or_abort(&cfull[cs], (it / kMxCStages) & 1, abort_flag, a.flags) &&
+                                 wait_or_abort(&bempty[bs], ((it / kMxBStages) & 1) ^ 1, abort_flag, a.flags);
+                ok = named_and(2, kMxConvThreads, got);
+                if (!ok) break;
+                // plain shared-memory accesses (the waits and barriers around
+                // them are compiler barriers): the 8 chunks' loads issue
+                // together instead of one chunk's chain after another
+                const uint32_t* cw =
+                    reinterpret_cast<const uint32_t*>(smem + kMxCOff + cs * kMxCodeBytes) + r0 * 8 + j;
+                const int bi = kb * 2 + (j >> 2);  // this chunk's 32-element block along K
+                const uint8_t* ss = sscale + r0 * nsb + bi;
+                uint8_t* bst = smem + kMxBOff + bs * kBBytes;
+                uint32_t w[kBRows / 32], sv[kBRows / 32];
+#pragma unroll
+                for (int i = 0; i < kBRows / 32; ++i) {
+                    w[i] = cw[i * 32 * 8];
+                    sv[i] = bi < nsb ? ss[i * 32 * nsb] : 0u;  // a block past K: zero codes (TMA fill)
+                }
+#pragma unroll
+                for (int i = 0; i < kBRows / 32; ++i) {
+                    uint32_t o[4];
+                    mx_chunk_to_bf16(w[i], sv[i], o);
+                    *reinterpret_cast<uint4*>(bst + stage_off(r0 + 32 * i, j)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                fence_proxy_async_smem();  // these generic-proxy writes, before the MMA's async reads
+                named_and(2, kMxConvThreads, true);  // every converter is done with the slot and the tile
+                if (ct == 0) {
+                    mbar_arrive(&bfull[bs]);
+                    mbar_arrive(&cempty[cs]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
 // ------------------------------------------------------------------ host side
 constexpr size_t kSmemBytes = kEpiStageOff + 4 * kEpiStageBytes + 1024;
 
@@ -702,6 +1094,20 @@ cudaError_t launch_grouped_pair(const Plan& p, const CUtensorMap (&maps)[7], con
 // B (its half from its own shared memory, the other half from the peer's),
 // so shared-memory traffic drops only by about a sixth.
 bool use_pairs(const Plan& p) { return p.I <= 1024 && p.S >= 512 * p.E; }
+
+template <bool kGateUp>
+cudaError_t launch_grouped_mx(const Plan& p, const CUtensorMap (&maps)[4], const GemmArgs& args, const MxArgs& mx,
+                              cudaStream_t st) {
+    constexpr int BN = kGateUp ? kBRows / 2 : kBRows;
+    cudaError_t e = ensure_smem_attr(grouped_gemm_mx_kernel<kGateUp>, kMxSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int64_t nb_r = (args.N + BN - 1) / BN;
+    const int64_t ub = ((p.S + kBM - 1) / kBM + p.E) * nb_r;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), ub));
+    grouped_gemm_mx_kernel<kGateUp><<<grid, kMxThreads, kMxSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                            args, mx);
+    return cudaGetLastError();
+}
 
 GemmArgs base_args(const Plan& p) {
     GemmArgs a{};
@@ -781,6 +1187,56 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     if (pairs) a.mtile_prefix = p.mpair_prefix;
     trace_before(mode ? "down_sm100_weighted" : "down_sm100", st);
     cudaError_t e = pairs ? launch_grouped_pair<false>(p, m, a, st) : launch_grouped<false>(p, m, a, st);
+    trace_after(st);
+    return e;
+}
+
+bool mx_gemm_eligible(const Plan& p) {
+    return p.bf16 && p.Is == 0 && p.H % 32 == 0 && p.I % 32 == 0 && p.H / 32 <= kMxMaxScales &&
+           p.I / 32 <= kMxMaxScales;
+}
+
+cudaError_t launch_gateup_mx_sm100(const Plan& p, const uint8_t* gate_blocks, const uint8_t* gate_scales,
+                                   const uint8_t* up_blocks, const uint8_t* up_scales, cudaStream_t st) {
+    if (p.T == 0) return cudaSuccess;
+    if (!mx_gemm_eligible(p)) return cudaErrorInvalidValue;
+    CUtensorMap m[4];
+    const bool ok = make_map_bf16(&m[0], p.xperm, p.H, p.S, 1, kBK, kBM) &&
+                    make_map_bf16(&m[1], p.xperm, p.H, p.S, 1, kBK, kSmallRows) &&
+                    make_map_u8(&m[2], gate_blocks, p.H / 2, p.I, p.E, kBK / 2, kBRows / 2) &&
+                    make_map_u8(&m[3], up_blocks, p.H / 2, p.I, p.E, kBK / 2, kBRows / 2);
+    if (!ok) return cudaErrorInvalidValue;
+    GemmArgs a = base_args(p);
+    a.N = (int)p.I;
+    a.K = a.Ks = (int)p.H;
+    a.h = (bf16*)p.h;
+    a.hs = (bf16*)p.h + p.S * p.I;
+    trace_before("gateup_mx_sm100", st);
+    cudaError_t e = launch_grouped_mx<true>(p, m, a, MxArgs{gate_scales, up_scales}, st);
+    trace_after(st);
+    return e;
+}
+
+cudaError_t launch_down_mx_sm100(const Plan& p, const uint8_t* down_blocks, const uint8_t* down_scales, int mode,
+                                 void* out, cudaStream_t st) {
+    if (p.T == 0) return cudaSuccess;
+    if (!mx_gemm_eligible(p)) return cudaErrorInvalidValue;
+    CUtensorMap m[4];
+    const bool ok = make_map_bf16(&m[0], p.h, p.I, p.S, 1, kBK, kBM) &&
+                    make_map_bf16(&m[1], p.h, p.I, p.S, 1, kBK, kSmallRows) &&
+                    make_map_u8(&m[2], down_blocks, p.I / 2, p.H, p.E, kBK / 2, kBRows);
+    if (!ok) return cudaErrorInvalidValue;
+    m[3] = m[2];
+    GemmArgs a = base_args(p);
+    a.N = a.Ns = (int)p.H;
+    a.K = (int)p.I;
+    a.perm_rows = p.perm_rows;
+    a.topk_w = p.topk_w;
+    a.out = mode == 0 ? (float*)out : nullptr;
+    a.rows = mode == 1 ? (bf16*)out : nullptr;
+    a.mode = mode;
+    trace_before(mode ? "down_mx_sm100_weighted" : "down_mx_sm100", st);
+    cudaError_t e = launch_grouped_mx<false>(p, m, a, MxArgs{down_scales, nullptr}, st);
     trace_after(st);
     return e;
 }

@@ -571,10 +571,10 @@ moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, co
 }
 
 // Bytes of the bf16 copies of the gate, up and down weights that the MXFP4
-// tile path makes in the workspace after moe_forward's own scratch; 0 when
-// the decode kernel serves the size.
+// dequantizing path makes in the workspace after moe_forward's own scratch;
+// 0 when the decode kernel or the MXFP4 GEMMs serve the size.
 static size_t mxfp4_dequant_bytes(const Plan& p) {
-    if (p.T == 0 || decode_mxfp4_eligible(p)) return 0;
+    if (p.T == 0 || decode_mxfp4_eligible(p) || mx_gemm_eligible(p)) return 0;
     return align_up((size_t)3 * p.E * p.H * p.I * 2);
 }
 
@@ -623,22 +623,34 @@ moe_status_t moe_forward_mxfp4(const moe_config_t* cfg, const void* x, const voi
     const uint8_t* mx[6] = {w_gate_blocks, w_gate_scales, w_up_blocks, w_up_scales, w_down_blocks, w_down_scales};
     int32_t* counts = counts_out ? counts_out : p.counts;
     int32_t* dropped = dropped_out ? dropped_out : p.dropped;
-    if (dq_bytes == 0) {
+    if (decode_mxfp4_eligible(p)) {
         // decode sizes: routing, the expert FFNs on the MXFP4 rows and the
         // combine in one weight-streaming kernel
         CUDA_TRY(launch_decode_layer_mxfp4(p, x, router_w, router_b, topk_idx_out, mx, y, counts, dropped, st),
                  "decode_layer_mxfp4");
         return MOE_OK;
     }
-    // more slots: the weights dequantized (exactly) to bf16 in the workspace,
-    // then moe_forward's routing, grouping, tcgen05 grouped GEMMs and combine
+    int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
+    if (dq_bytes == 0) {
+        // moe_forward's tile path with grouped GEMMs that read the MXFP4
+        // codes and convert them to bf16 in shared memory
+        CUDA_TRY(run_router(p, x, router_w, router_b, idx, p.topk_w, st), "router");
+        CUDA_TRY(launch_permute(p, idx, counts, p.offsets, p.perm_rows, p.row_of, dropped, st), "permute");
+        CUDA_TRY(launch_scatter_x_rows(p, x, p.row_of, p.xperm, st), "gather_rows");
+        CUDA_TRY(launch_gateup_mx_sm100(p, mx[0], mx[1], mx[2], mx[3], st), "gateup_mx");
+        CUDA_TRY(launch_down_mx_sm100(p, mx[4], mx[5], 1, p.rows, st), "down_mx");
+        CUDA_TRY(launch_combine_rows(p, p.rows, p.row_of, y, st), "combine_rows");
+        return MOE_OK;
+    }
+    // H or I above the MXFP4 GEMMs' limit: the weights dequantized (exactly)
+    // to bf16 in the workspace, then moe_forward's routing, grouping, tcgen05
+    // grouped GEMMs and combine
     bf16* wg = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + p.bytes);
     bf16* wu = wg + p.E * p.I * p.H;
     bf16* wd = wu + p.E * p.I * p.H;
     CUDA_TRY(launch_mxfp4_dequant(mx[0], mx[1], p.E * p.I, (int)p.H, wg, st), "mxfp4_dequant");
     CUDA_TRY(launch_mxfp4_dequant(mx[2], mx[3], p.E * p.I, (int)p.H, wu, st), "mxfp4_dequant");
     CUDA_TRY(launch_mxfp4_dequant(mx[4], mx[5], p.E * p.H, (int)p.I, wd, st), "mxfp4_dequant");
-    int32_t* idx = topk_idx_out ? topk_idx_out : p.topk_idx;
     CUDA_TRY(run_router(p, x, router_w, router_b, idx, p.topk_w, st), "router");
     return forward_after_routing(p, x, idx, wg, wu, wd, nullptr, nullptr, nullptr, y, counts, dropped, st);
 }

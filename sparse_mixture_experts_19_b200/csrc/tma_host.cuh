@@ -69,6 +69,51 @@ inline bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint
     return true;
 }
 
+// Rank-3 map of a byte tensor [depth][rows][inner] (inner contiguous, a
+// multiple of 16 bytes) with box {box_inner, box_rows, 1}, no swizzle (rows
+// land box_inner bytes apart); out-of-range bytes of a box read as zero.
+// Cached like make_map_bf16.
+inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                        uint32_t box_inner, uint32_t box_rows) {
+    struct Entry {
+        const void* base;
+        uint64_t inner, rows, depth;
+        uint32_t box_inner, box_rows;
+        CUtensorMap map;
+    };
+    constexpr int kCache = 32;
+    static Entry cache[kCache];
+    static int used = 0, next = 0;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i) {
+            const Entry& c = cache[i];
+            if (c.base == base && c.inner == inner && c.rows == rows && c.depth == depth &&
+                c.box_inner == box_inner && c.box_rows == box_rows) {
+                *m = c.map;
+                return true;
+            }
+        }
+    }
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {inner, rows, depth};
+    cuuint64_t strides[2] = {inner, inner * rows};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry& c = cache[next];
+    c = Entry{base, inner, rows, depth, box_inner, box_rows, *m};
+    next = (next + 1) % kCache;
+    if (used < kCache) ++used;
+    return true;
+}
+
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel (by
 // address), device and size.
 template <typename Kernel>

@@ -27,10 +27,12 @@ CASES = [
     mi.GPTOSS.with_(name="gpt_oss_mxfp4_T2", T=2),
     mi.GPTOSS.with_(name="gpt_oss_mxfp4_T8", T=8),  # 32 slots, the size limit
     mi.Workload("mxfp4_ragged_T7", T=7, H=352, I=160, E=24, k=4),  # 28 slots, 3 columns per CTA with a tail
-    # above 32 slots: dequantized weights on the tile path
+    # above 32 slots: the tile path, its GEMMs converting the codes in shared memory
     mi.GPTOSS.with_(name="gpt_oss_mxfp4_T64", T=64),
     mi.Workload("mxfp4_tile_ragged", T=45, H=352, I=160, E=24, k=4),  # 180 slots, ragged tiles
     mi.Workload("mxfp4_tile_cap", T=40, H=256, I=128, E=8, k=2, capacity_factor=0.75),
+    # I / 32 above the MXFP4 GEMMs' 96 scale bytes per row: dequantized to bf16 first
+    mi.Workload("mxfp4_dequant_path", T=40, H=256, I=3104, E=4, k=1),
     mi.Workload("mxfp4_small_cap", T=2, H=256, I=128, E=8, k=4, capacity_factor=0.5),
     mi.Workload("mxfp4_one_expert", T=8, H=128, I=96, E=1, k=1),
     mi.Workload("mxfp4_e256", T=1, H=512, I=256, E=256, k=8, zipf_s=1.1),
@@ -73,7 +75,7 @@ def test_mxfp4_layer_matches_oracle(gpu_lib, wl):
 def test_mxfp4_nan_scale_reaches_only_the_tokens_that_read_it(gpu_lib, T):
     """A scale byte of 255 (NaN) in one expert's gate rows: the tokens routed
     to that expert get NaN outputs, as in the oracle; the others do not
-    (4 slots: the decode kernel; 48: the dequantizing tile path)."""
+    (4 slots: the decode kernel; 48: the tile path's MXFP4 GEMMs)."""
     wl = mi.Workload("mxfp4_nan", T=T, H=256, I=128, E=8, k=2)
     inp = mi.make_inputs(wl, router_only=True)
     mx = mi.make_mxfp4_experts(wl)
@@ -109,10 +111,13 @@ def test_mxfp4_validates():
     assert call(_cfg(H=264)) == 1 and "32" in moe_pkg.moe_last_error()
     assert call(_cfg(dtype="f32")) == 2
     assert call(_cfg(T=0)) == 0
-    # 36 slots take the dequantizing tile path, which needs the larger workspace
-    c = _cfg(T=9)
-    assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c)) + 3 * 8 * 256 * 128 * 2
+    # 36 slots with I = 3104 (> 3072): the dequantizing path, which needs the larger workspace
+    c = _cfg(T=9, I=3104)
+    assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c)) + 3 * 8 * 256 * 3104 * 2
     assert call(c) == 3 and "moe_mxfp4_workspace_size" in moe_pkg.moe_last_error()
+    # 36 slots within the MXFP4 GEMMs' limits: no extra workspace
+    c = _cfg(T=9)
+    assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c))
     # up to 32 slots the decode kernel needs no more than moe_forward
     c = _cfg(T=8)
     assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c))
