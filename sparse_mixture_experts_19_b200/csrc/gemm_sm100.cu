@@ -671,9 +671,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
 // the 128-byte-swizzled K-major layout the MMA reads (chunk c of row r at
 // r*128 + ((c ^ r%8) * 16)), and the MMA runs as on bf16 weights.  Three
 // rings, each as deep as it needs to be: A tiles (3 x 16 KB, TMA), converted
-// B tiles (2 x 32 KB) and codes (8 x 8 KB): the codes ring keeps 64 KB of
-// weight reads in flight per SM; a producer warp of its own refills a codes
-// slot as soon as the converters have read it.  The conversion is integer
+// B tiles (2 x 32 KB) and codes (2 x 32 KB, four k-steps of 256 rows x 32
+// bytes per slot, so that a TMA row is a whole 128-byte line and the TMA
+// unit is not held up by narrow rows ahead of the A copies): 64 KB of weight
+// reads in flight per SM; a producer warp of its own refills a codes slot as
+// soon as the converters have read it.  The conversion is integer
 // work plus one bf16 multiply per two elements (see mx_chunk_to_bf16): the
 // float conversion instructions run at a fraction of the ALU rate.  Every
 // converted value e * 2^(s-127) is exact in bf16 (normal or subnormal;
@@ -683,8 +685,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) grouped
 // the tile starts; K <= 32 * kMxMaxScales.
 constexpr int kMxAStages = 3;
 constexpr int kMxBStages = 2;
-constexpr int kMxCStages = 8;
-constexpr int kMxCodeBytes = kBRows * kBK / 2;  // 8 KB of codes per k-step
+constexpr int kMxGroupSteps = 4;                                // k-steps per codes copy (128-byte rows)
+constexpr int kMxCStages = 2;
+constexpr int kMxCodeBytes = kBRows * kBK / 2 * kMxGroupSteps;  // 32 KB of codes per slot
 constexpr int kMxMaxScales = 96;                 // scale bytes per row a tile holds: K <= 3072
 constexpr int kMxConvWarps = 8;
 constexpr int kMxConvThreads = kMxConvWarps * 32;
@@ -763,6 +766,7 @@ __device__ __forceinline__ void mx_chunk_to_bf16(uint32_t w, uint32_t s, uint32_
 struct MxArgs {
     const uint8_t* sc0;  // scales of the B rows: gate / down [E, N, K/32]
     const uint8_t* sc1;  // up [E, N, K/32] (gate/up only)
+    int keep_a;          // the A rows fit in L2: read them with evict_last, the codes with evict_first
 };
 
 // The k-steps of this CTA's tiles in order: (tile, k-step) of step `it`.
@@ -783,8 +787,9 @@ __device__ __forceinline__ bool cursor_start(StepCursor& c, const Tables& tb, co
 }
 
 __device__ __forceinline__ bool cursor_next(StepCursor& c, const Tables& tb, const Sched& sc, const GemmArgs& a,
-                                            int BN) {
-    if (++c.kb < c.nkb) return true;
+                                            int BN, int stride = 1) {
+    c.kb += stride;
+    if (c.kb < c.nkb) return true;
     c.t += gridDim.x;
     c.kb = 0;
     if (c.t >= sc.total) return false;
@@ -826,12 +831,12 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
             mbar_init(&aempty[s], 1);
         }
         for (int s = 0; s < kMxBStages; ++s) {
-            mbar_init(&bfull[s], 1);
+            mbar_init(&bfull[s], kMxConvWarps);  // one arrival per converter warp
             mbar_init(&bempty[s], 1);
         }
         for (int s = 0; s < kMxCStages; ++s) {
             mbar_init(&cfull[s], 1);
-            mbar_init(&cempty[s], 1);
+            mbar_init(&cempty[s], kMxConvWarps);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
@@ -868,6 +873,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
     if (warp == 0) {
         // ------------------------------------------------ TMA producer of A
         if (lane == 0) {
+            // A tiles are read once per column block: when they fit in L2
+            // they are kept there ahead of the codes streaming past
+            const uint64_t pol = mxa.keep_a ? l2_policy_evict_last() : 0;
             uint32_t it = 0;
             for (int64_t t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
                 TileInfo ti;
@@ -881,7 +889,10 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
                     const uint32_t ph = (it / kMxAStages) & 1;
                     if (!wait_or_abort(&aempty[s], ph ^ 1, abort_flag, a.flags)) break;
                     mbar_arrive_expect_tx(&afull[s], a_tx);
-                    tma_load_3d(smem + s * kABytes, mA, &afull[s], kb * kBK, ti.arow, 0);
+                    if (mxa.keep_a)
+                        tma_load_3d_hint(smem + s * kABytes, mA, &afull[s], kb * kBK, ti.arow, 0, pol);
+                    else
+                        tma_load_3d(smem + s * kABytes, mA, &afull[s], kb * kBK, ti.arow, 0);
                 }
             }
             // never leave with copies in flight (bounded waits)
@@ -945,19 +956,23 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
     } else if (warp == kMxCodeWarp) {
         // ------------------------------------------------ TMA producer of the codes
         if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
             StepCursor c{};
             uint32_t it = 0;
+            // one copy per group of kMxGroupSteps k-steps of a tile (it counts groups)
             for (bool more = cursor_start(c, *tb, sc, a, BN); more && !*abort_flag;
-                 more = cursor_next(c, *tb, sc, a, BN), ++it) {
+                 more = cursor_next(c, *tb, sc, a, BN, kMxGroupSteps), ++it) {
                 const int s = it % kMxCStages;
                 if (!wait_or_abort(&cempty[s], ((it / kMxCStages) & 1) ^ 1, abort_flag, a.flags)) break;
                 uint8_t* dst = smem + kMxCOff + s * kMxCodeBytes;
+                const int x = c.kb * (kBK / 2);  // byte column of the group's first k-step
                 mbar_arrive_expect_tx(&cfull[s], kMxCodeBytes);
-                if (kGateUp) {
-                    tma_load_3d(dst, &tmC0, &cfull[s], c.kb * (kBK / 2), c.ti.n0, c.ti.e);
-                    tma_load_3d(dst + kMxCodeBytes / 2, &tmC1, &cfull[s], c.kb * (kBK / 2), c.ti.n0, c.ti.e);
+                if (mxa.keep_a) {  // each tile's codes are read once
+                    tma_load_3d_hint(dst, &tmC0, &cfull[s], x, c.ti.n0, c.ti.e, pol);
+                    if (kGateUp) tma_load_3d_hint(dst + kMxCodeBytes / 2, &tmC1, &cfull[s], x, c.ti.n0, c.ti.e, pol);
                 } else {
-                    tma_load_3d(dst, &tmC0, &cfull[s], c.kb * (kBK / 2), c.ti.n0, c.ti.e);
+                    tma_load_3d(dst, &tmC0, &cfull[s], x, c.ti.n0, c.ti.e);
+                    if (kGateUp) tma_load_3d(dst + kMxCodeBytes / 2, &tmC1, &cfull[s], x, c.ti.n0, c.ti.e);
                 }
             }
             // never leave with copies in flight (bounded waits)
@@ -973,9 +988,13 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
         const int ct = threadIdx.x - kThreads;
         const int j = ct & 7, r0 = ct >> 3;
         const int nsb = a.K / 32;  // scale bytes per row
-        uint32_t it = 0;
-        bool ok = true;
-        for (int64_t t = blockIdx.x; t < sc.total && ok; t += gridDim.x) {
+        // Each warp reports a step done with its own arrivals on bfull and
+        // cempty, so the warps meet only when a tile starts (its scale
+        // bytes).  After an abort every wait returns at once: the warps walk
+        // the remaining steps without work and still meet at the same
+        // barriers.
+        uint32_t it = 0, gi = 0;  // k-steps, codes groups
+        for (int64_t t = blockIdx.x; t < sc.total; t += gridDim.x) {
             TileInfo ti;
             decode_tile(t, *tb, sc, a, BN, ti);
             // the tile's scale bytes -> sscale[row][nsb] (rows past N left as
@@ -1011,37 +1030,43 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
             named_and(2, kMxConvThreads, true);
             const int nkb = (ti.K + kBK - 1) / kBK;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int cs = it % kMxCStages, bs = it % kMxBStages;
-                const bool got = wait_or_abort(&cfull[cs], (it / kMxCStages) & 1, abort_flag, a.flags) &&
+                const int cs = gi % kMxCStages, bs = it % kMxBStages, pos = kb % kMxGroupSteps;
+                const bool got = (pos != 0 || wait_or_abort(&cfull[cs], (gi / kMxCStages) & 1, abort_flag, a.flags)) &&
                                  wait_or_abort(&bempty[bs], ((it / kMxBStages) & 1) ^ 1, abort_flag, a.flags);
-                ok = named_and(2, kMxConvThreads, got);
-                if (!ok) break;
-                // plain shared-memory accesses (the waits and barriers around
-                // them are compiler barriers): the 8 chunks' loads issue
-                // together instead of one chunk's chain after another
-                const uint32_t* cw =
-                    reinterpret_cast<const uint32_t*>(smem + kMxCOff + cs * kMxCodeBytes) + r0 * 8 + j;
-                const int bi = kb * 2 + (j >> 2);  // this chunk's 32-element block along K
-                const uint8_t* ss = sscale + r0 * nsb + bi;
-                uint8_t* bst = smem + kMxBOff + bs * kBBytes;
-                uint32_t w[kBRows / 32], sv[kBRows / 32];
+                if (__all_sync(0xffffffffu, got)) {
+                    // plain shared-memory accesses (the waits and barriers around
+                    // them are compiler barriers): the 8 chunks' loads issue
+                    // together instead of one chunk's chain after another
+                    // word j of this k-step in row r (128-byte rows, the TMA's
+                    // 128-byte swizzle: 16-byte chunk c at c ^ (r % 8); r % 8
+                    // = r0 % 8 for every row of the thread)
+                    const int byte = pos * (kBK / 2) + j * 4;
+                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(
+                        smem + kMxCOff + cs * kMxCodeBytes + r0 * 128 + ((((byte >> 4) ^ (r0 & 7)) << 4) | (byte & 15)));
+                    const int bi = kb * 2 + (j >> 2);  // this chunk's 32-element block along K
+                    const uint8_t* ss = sscale + r0 * nsb + bi;
+                    uint8_t* bst = smem + kMxBOff + bs * kBBytes;
+                    uint32_t w[kBRows / 32], sv[kBRows / 32];
 #pragma unroll
-                for (int i = 0; i < kBRows / 32; ++i) {
-                    w[i] = cw[i * 32 * 8];
-                    sv[i] = bi < nsb ? ss[i * 32 * nsb] : 0u;  // a block past K: zero codes (TMA fill)
-                }
+                    for (int i = 0; i < kBRows / 32; ++i) {
+                        w[i] = cw[i * 32 * 32];  // 32 rows of 128 bytes further
+                        sv[i] = bi < nsb ? ss[i * 32 * nsb] : 0u;  // a block past K: zero codes (TMA fill)
+                    }
 #pragma unroll
-                for (int i = 0; i < kBRows / 32; ++i) {
-                    uint32_t o[4];
-                    mx_chunk_to_bf16(w[i], sv[i], o);
-                    *reinterpret_cast<uint4*>(bst + stage_off(r0 + 32 * i, j)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    for (int i = 0; i < kBRows / 32; ++i) {
+                        uint32_t o[4];
+                        mx_chunk_to_bf16(w[i], sv[i], o);
+                        *reinterpret_cast<uint4*>(bst + stage_off(r0 + 32 * i, j)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                    fence_proxy_async_smem();  // these generic-proxy writes, before the MMA's async reads
                 }
-                fence_proxy_async_smem();  // these generic-proxy writes, before the MMA's async reads
-                named_and(2, kMxConvThreads, true);  // every converter is done with the slot and the tile
-                if (ct == 0) {
+                __syncwarp();
+                const bool group_end = pos == kMxGroupSteps - 1 || kb == nkb - 1;
+                if (lane == 0) {  // this warp's rows of the step are written (and the group's codes read)
                     mbar_arrive(&bfull[bs]);
-                    mbar_arrive(&cempty[cs]);
+                    if (group_end) mbar_arrive(&cempty[cs]);
                 }
+                if (group_end) ++gi;
             }
         }
     }
@@ -1191,9 +1216,14 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     return e;
 }
 
+// Used where it is the faster path: up to 256 rows per expert on average
+// (the weight-bound sizes).  With more rows the tiles are compute-bound and
+// the converters' integer work per k-step (about twice the MMA's time)
+// decides, so one bf16 conversion of the weights followed by the bf16 GEMMs
+// is faster there.
 bool mx_gemm_eligible(const Plan& p) {
     return p.bf16 && p.Is == 0 && p.H % 32 == 0 && p.I % 32 == 0 && p.H / 32 <= kMxMaxScales &&
-           p.I / 32 <= kMxMaxScales;
+           p.I / 32 <= kMxMaxScales && p.S <= 256 * p.E;
 }
 
 cudaError_t launch_gateup_mx_sm100(const Plan& p, const uint8_t* gate_blocks, const uint8_t* gate_scales,
@@ -1203,8 +1233,8 @@ cudaError_t launch_gateup_mx_sm100(const Plan& p, const uint8_t* gate_blocks, co
     CUtensorMap m[4];
     const bool ok = make_map_bf16(&m[0], p.xperm, p.H, p.S, 1, kBK, kBM) &&
                     make_map_bf16(&m[1], p.xperm, p.H, p.S, 1, kBK, kSmallRows) &&
-                    make_map_u8(&m[2], gate_blocks, p.H / 2, p.I, p.E, kBK / 2, kBRows / 2) &&
-                    make_map_u8(&m[3], up_blocks, p.H / 2, p.I, p.E, kBK / 2, kBRows / 2);
+                    make_map_u8(&m[2], gate_blocks, p.H / 2, p.I, p.E, kBK / 2 * kMxGroupSteps, kBRows / 2) &&
+                    make_map_u8(&m[3], up_blocks, p.H / 2, p.I, p.E, kBK / 2 * kMxGroupSteps, kBRows / 2);
     if (!ok) return cudaErrorInvalidValue;
     GemmArgs a = base_args(p);
     a.N = (int)p.I;
@@ -1212,7 +1242,9 @@ cudaError_t launch_gateup_mx_sm100(const Plan& p, const uint8_t* gate_blocks, co
     a.h = (bf16*)p.h;
     a.hs = (bf16*)p.h + p.S * p.I;
     trace_before("gateup_mx_sm100", st);
-    cudaError_t e = launch_grouped_mx<true>(p, m, a, MxArgs{gate_scales, up_scales}, st);
+    // A rows that fit in a quarter of L2 stay there across the column blocks
+    const int keep_a = p.S * p.H * 2 <= (32ll << 20);
+    cudaError_t e = launch_grouped_mx<true>(p, m, a, MxArgs{gate_scales, up_scales, keep_a}, st);
     trace_after(st);
     return e;
 }
@@ -1224,7 +1256,7 @@ cudaError_t launch_down_mx_sm100(const Plan& p, const uint8_t* down_blocks, cons
     CUtensorMap m[4];
     const bool ok = make_map_bf16(&m[0], p.h, p.I, p.S, 1, kBK, kBM) &&
                     make_map_bf16(&m[1], p.h, p.I, p.S, 1, kBK, kSmallRows) &&
-                    make_map_u8(&m[2], down_blocks, p.I / 2, p.H, p.E, kBK / 2, kBRows);
+                    make_map_u8(&m[2], down_blocks, p.I / 2, p.H, p.E, kBK / 2 * kMxGroupSteps, kBRows);
     if (!ok) return cudaErrorInvalidValue;
     m[3] = m[2];
     GemmArgs a = base_args(p);
@@ -1236,7 +1268,8 @@ cudaError_t launch_down_mx_sm100(const Plan& p, const uint8_t* down_blocks, cons
     a.rows = mode == 1 ? (bf16*)out : nullptr;
     a.mode = mode;
     trace_before(mode ? "down_mx_sm100_weighted" : "down_mx_sm100", st);
-    cudaError_t e = launch_grouped_mx<false>(p, m, a, MxArgs{down_scales, nullptr}, st);
+    const int keep_a = p.S * p.I * 2 <= (32ll << 20);
+    cudaError_t e = launch_grouped_mx<false>(p, m, a, MxArgs{down_scales, nullptr, keep_a}, st);
     trace_after(st);
     return e;
 }

@@ -70,9 +70,10 @@ inline bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint
 }
 
 // Rank-3 map of a byte tensor [depth][rows][inner] (inner contiguous, a
-// multiple of 16 bytes) with box {box_inner, box_rows, 1}, no swizzle (rows
-// land box_inner bytes apart); out-of-range bytes of a box read as zero.
-// Cached like make_map_bf16.
+// multiple of 16 bytes) with box {box_inner, box_rows, 1}; box_inner = 128
+// takes the 128-byte swizzle (16-byte chunk c of box row r at c ^ (r % 8)),
+// other widths none (rows box_inner bytes apart).  Out-of-range bytes of a
+// box read as zero.  Cached like make_map_bf16.
 inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                         uint32_t box_inner, uint32_t box_rows) {
     struct Entry {
@@ -103,7 +104,8 @@ inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64
     cuuint32_t box[3] = {box_inner, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     if (fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, box_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
     std::lock_guard<std::mutex> lock(mu);

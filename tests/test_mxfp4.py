@@ -33,6 +33,8 @@ CASES = [
     mi.Workload("mxfp4_tile_cap", T=40, H=256, I=128, E=8, k=2, capacity_factor=0.75),
     # I / 32 above the MXFP4 GEMMs' 96 scale bytes per row: dequantized to bf16 first
     mi.Workload("mxfp4_dequant_path", T=40, H=256, I=3104, E=4, k=1),
+    # more than 256 rows per expert: dequantized to bf16 first
+    mi.Workload("mxfp4_dequant_rows", T=600, H=256, I=128, E=4, k=2),
     mi.Workload("mxfp4_small_cap", T=2, H=256, I=128, E=8, k=4, capacity_factor=0.5),
     mi.Workload("mxfp4_one_expert", T=8, H=128, I=96, E=1, k=1),
     mi.Workload("mxfp4_e256", T=1, H=512, I=256, E=256, k=8, zipf_s=1.1),
@@ -118,6 +120,9 @@ def test_mxfp4_validates():
     # 36 slots within the MXFP4 GEMMs' limits: no extra workspace
     c = _cfg(T=9)
     assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c))
+    # 2400 slots over 8 experts (> 256 rows each): the dequantizing path again
+    c = _cfg(T=600)
+    assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c)) + 3 * 8 * 256 * 128 * 2
     # up to 32 slots the decode kernel needs no more than moe_forward
     c = _cfg(T=8)
     assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c))
