@@ -670,7 +670,7 @@ def run_mxfp4_stage(args, wl):
     conf = dict(config_of(wl), l2="L2 flushed before each timed call (a 256 MB write outside the events)")
     return {"stage": "mxfp4", "config": conf, "ms_per_call": ms, "tokens_per_s": wl.T / (ms / 1e3),
             "path": "decode kernel" if wl.T * wl.k <= 32 else (
-                "tile path, MXFP4 GEMMs" if max(wl.H, wl.I) <= 3072 and wl.T * wl.k <= 256 * wl.E
+                "tile path, MXFP4 GEMMs" if max(wl.H, wl.I) <= 3072 and wl.T * wl.k <= 128 * wl.E
                 else "dequantized to bf16, tile GEMMs"),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "bytes_per_launch": nbytes, "active_experts": active,

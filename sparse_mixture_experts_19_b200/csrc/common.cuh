@@ -150,7 +150,7 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
 // The same GEMMs with the routed experts' weights in MXFP4 (E2M1 code blocks
 // [E, N, K/32, 16] and E8M0 scales [E, N, K/32], K = H for gate/up, I for
 // down), converted to bf16 in shared memory: bf16 layer, no shared expert,
-// H and I multiples of 32 and at most 3072, T*k at most 256 rows per expert
+// H and I multiples of 32 and at most 3072, T*k at most 128 rows per expert
 // (mx_gemm_eligible).
 bool mx_gemm_eligible(const Plan& p);
 cudaError_t launch_gateup_mx_sm100(const Plan& p, const uint8_t* gate_blocks, const uint8_t* gate_scales,

@@ -1216,14 +1216,14 @@ cudaError_t launch_down_sm100(const Plan& p, const void* w_down, const void* ws_
     return e;
 }
 
-// Used where it is the faster path: up to 256 rows per expert on average
-// (the weight-bound sizes).  With more rows the tiles are compute-bound and
-// the converters' integer work per k-step (about twice the MMA's time)
+// Used where it is the faster path (measured at gpt-oss size): up to 128
+// rows per expert on average.  With more rows the tiles turn compute-bound
+// and the converters' integer work per k-step (about twice the MMA's time)
 // decides, so one bf16 conversion of the weights followed by the bf16 GEMMs
 // is faster there.
 bool mx_gemm_eligible(const Plan& p) {
     return p.bf16 && p.Is == 0 && p.H % 32 == 0 && p.I % 32 == 0 && p.H / 32 <= kMxMaxScales &&
-           p.I / 32 <= kMxMaxScales && p.S <= 256 * p.E;
+           p.I / 32 <= kMxMaxScales && p.S <= 128 * p.E;
 }
 
 cudaError_t launch_gateup_mx_sm100(const Plan& p, const uint8_t* gate_blocks, const uint8_t* gate_scales,

@@ -33,7 +33,7 @@ CASES = [
     mi.Workload("mxfp4_tile_cap", T=40, H=256, I=128, E=8, k=2, capacity_factor=0.75),
     # I / 32 above the MXFP4 GEMMs' 96 scale bytes per row: dequantized to bf16 first
     mi.Workload("mxfp4_dequant_path", T=40, H=256, I=3104, E=4, k=1),
-    # more than 256 rows per expert: dequantized to bf16 first
+    # more than 128 rows per expert: dequantized to bf16 first
     mi.Workload("mxfp4_dequant_rows", T=600, H=256, I=128, E=4, k=2),
     mi.Workload("mxfp4_small_cap", T=2, H=256, I=128, E=8, k=4, capacity_factor=0.5),
     mi.Workload("mxfp4_one_expert", T=8, H=128, I=96, E=1, k=1),
@@ -120,7 +120,7 @@ def test_mxfp4_validates():
     # 36 slots within the MXFP4 GEMMs' limits: no extra workspace
     c = _cfg(T=9)
     assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c))
-    # 2400 slots over 8 experts (> 256 rows each): the dequantizing path again
+    # 2400 slots over 8 experts (> 128 rows each): the dequantizing path again
     c = _cfg(T=600)
     assert lib.moe_mxfp4_workspace_size(ctypes.byref(c)) == lib.moe_workspace_size(ctypes.byref(c)) + 3 * 8 * 256 * 128 * 2
     # up to 32 slots the decode kernel needs no more than moe_forward
