@@ -737,29 +737,29 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 // with E8M0 scale byte s -> eight bf16 values e * 2^(s-127) in o[0..3].
 // A nibble's sign bit moved to bit 15 and its three exponent/mantissa bits
 // to bits 8..6 form the bf16 of e * 2^-126 exactly (exponent field 0 makes
-// the codes 0 and 0.5 the subnormals 0 and 2^-127); one rounding multiply
-// by 2^(s-1) (two, by 2^126 then 2^(s-127), when 2^(s-1) exceeds bf16's
-// range) then gives e * 2^(s-127), exact wherever bf16 holds it.
+// the codes 0 and 0.5 the subnormals 0 and 2^-127).  With one nibble per
+// 16-bit lane, t * 0x1040 = (t << 12) | (t << 6) (the copies do not
+// overlap), and the mask keeps bits 15 and 8..6 of each lane.  One rounding
+// multiply by 2^(s-1) (two, by 2^126 then 2^(s-127), when 2^(s-1) exceeds
+// bf16's range) then gives e * 2^(s-127), exact wherever bf16 holds it.
 __device__ __forceinline__ void mx_chunk_to_bf16(uint32_t w, uint32_t s, uint32_t (&o)[4]) {
-    uint32_t pre = 0u, sc;
-    if (s <= 128u) {
-        sc = ((s + 126u) << 7) * 0x10001u;  // 2^(s-1)
-    } else if (s == 255u) {
-        sc = 0x7fc07fc0u;  // NaN
-    } else {
-        pre = 0x7e807e80u;  // 2^126
-        sc = (s << 7) * 0x10001u;  // 2^(s-127)
-    }
     const uint32_t lo = w & 0x0f0f0f0fu, hi = (w >> 4) & 0x0f0f0f0fu;
-    // selector q: byte q of lo, byte q of hi into the two halves, the other
-    // bytes the (zero) sign of a nibble byte
+    uint32_t t[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
+        // byte q of lo and of hi into the two lanes, zeros (the sign of a
+        // nibble byte) above them
         const uint32_t sel = (uint32_t)q | ((8u | q) << 4) | ((4u + q) << 8) | ((12u + q) << 12);
-        const uint32_t t = prmt(lo, hi, sel);
-        uint32_t v = ((t & 0x00080008u) << 12) | ((t & 0x00070007u) << 6);
-        if (pre) v = mul_bf16x2(v, pre);
-        o[q] = mul_bf16x2(v, sc);
+        t[q] = (prmt(lo, hi, sel) * 0x1040u) & 0x81c081c0u;
+    }
+    if (s <= 128u) {
+        const uint32_t sc = (s + 126u) * 0x00800080u;  // 2^(s-1) in both lanes
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] = mul_bf16x2(t[q], sc);
+    } else {
+        const uint32_t sc = s == 255u ? 0x7fc07fc0u : s * 0x00800080u;  // NaN, or 2^(s-127)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] = mul_bf16x2(mul_bf16x2(t[q], 0x7e807e80u), sc);  // x 2^126 first
     }
 }
 
@@ -947,7 +947,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
             TileInfo ti;
             decode_tile(t, *tb, sc, a, BN, ti);
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-            if (!wait_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
+            // a whole tile's wait: sleep in try_wait instead of taking issue
+            // slots from the converters on the same schedulers
+            if (!wait_sleep_or_abort(&tfull[acc], aph, abort_flag, a.flags)) break;
             tc_fence_after();
             epilogue_tile<kGateUp, BN>(ti, a, tmem_base + acc * kAccCols, q, r, epi_stage);
             tc_fence_before();
@@ -983,10 +985,13 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(
         }
     } else {
         // ------------------------------------------------ converter warps 6..13
-        // Thread ct converts chunk j = ct % 8 (8 elements) of rows ct / 8 + 32 i:
-        // a warp reads 4 rows x 32 bytes of codes and writes 4 rows x 128 bytes.
+        // Thread ct converts chunk j = ct % 8 (8 elements) of rows r0 + 32 i, a
+        // warp's four lane groups taking rows two apart (r0 % 8 = 0,2,4,6 or
+        // 1,3,5,7), so that the swizzled code chunks they read fall in
+        // different banks; a warp writes 4 rows x 128 bytes.
         const int ct = threadIdx.x - kThreads;
-        const int j = ct & 7, r0 = ct >> 3;
+        const int cw_ = ct >> 5, j = ct & 7;
+        const int r0 = (cw_ >> 1) * 8 + (cw_ & 1) + 2 * ((ct >> 3) & 3);
         const int nsb = a.K / 32;  // scale bytes per row
         // Each warp reports a step done with its own arrivals on bfull and
         // cempty, so the warps meet only when a tile starts (its scale
