@@ -356,8 +356,9 @@ moe_status_t moe_forward_expert_shard(const moe_config_t* cfg, const void* x, co
 /*
  * moe_mxfp4_workspace_size -- bytes of workspace moe_forward_mxfp4 needs for
  * cfg: moe_workspace_size(cfg), plus the bf16 copies of the expert weights
- * (3*E*H*I*2 bytes, 256-aligned) when the size takes the dequantizing tile
- * path.  0 for an invalid cfg (see moe_last_error).
+ * (3*E*H*I*2 bytes, 256-aligned) when the size takes the converting path
+ * (more than 128 rows per expert, or H or I above 3072).  0 for an invalid
+ * cfg (see moe_last_error).
  */
 size_t moe_mxfp4_workspace_size(const moe_config_t* cfg);
 
@@ -376,21 +377,27 @@ size_t moe_mxfp4_workspace_size(const moe_config_t* cfg);
  *   w_up_scales [E, I, H/32] uint8; w_down_blocks [E, H, I/32, 16],
  *   w_down_scales [E, H, I/32].  Blocks 16-byte aligned; scales any alignment.
  *   x, router_w, y bf16 (cfg->dtype MOE_BF16); the router is moe_forward's.
- * The weights are used exactly (every dequantized value is exact in float32);
- * each block's 32 products are summed in f16 with the token vector scaled by
- * a power of two into f16's range, and the blocks' sums in float32; h is
- * rounded to bf16 between the two projections as in moe_forward.
- * Two paths by size.  T * top_k <= 32 (gpt-oss-sized layers up to T = 8)
+ * The weights are used exactly (every dequantized value is exact in float32).
+ * On the decode kernel each block's 32 products are summed in f16 with the
+ * token vector scaled by a power of two into f16's range, and the blocks'
+ * sums in float32; on the tile paths the tensor cores multiply the bf16
+ * activations by the weights converted to bf16 and accumulate in float32.
+ * h is rounded to bf16 between the two projections as in moe_forward.
+ * Three paths by size.  T * top_k <= 32 (gpt-oss-sized layers up to T = 8)
  * with the decode kernel's shared memory within 200 KB (the token vectors,
  * T*H*2 bytes, one expert's h vectors, T*I*2 bytes, and the partial dots):
- * one weight-streaming kernel reads the MXFP4 rows themselves; the workspace
- * is moe_workspace_size(cfg).  Larger: the gate, up and down weights are
- * dequantized to bf16 (exact: every value e * 2^(s-127) fits bf16 down to
- * 2^-133; above bf16's range it becomes +-inf) into the workspace after
- * moe_forward's scratch, then moe_forward's tile path runs on them; the
- * workspace must hold moe_mxfp4_workspace_size(cfg) bytes (3*E*H*I*2 more),
- * else MOE_ERR_WORKSPACE.  No shared expert (I_shared = 0), H and I
- * multiples of 32; otherwise MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG.
+ * one weight-streaming kernel reads the MXFP4 rows themselves.  Up to 128
+ * rows per expert on average (T * top_k <= 128 * E) with H and I <= 3072:
+ * moe_forward's tile path with grouped GEMMs that read the codes and scales
+ * and convert them to bf16 in shared memory.  Both take a workspace of
+ * moe_workspace_size(cfg).  Otherwise the gate, up and down weights are
+ * converted to bf16 into the workspace after moe_forward's scratch, then
+ * moe_forward's tile path runs on them; the workspace must hold
+ * moe_mxfp4_workspace_size(cfg) bytes (3*E*H*I*2 more), else
+ * MOE_ERR_WORKSPACE.  Every path uses each dequantized value e * 2^(s-127)
+ * exactly (bf16 holds it down to 2^-133; above bf16's range it becomes
+ * +-inf).  No shared expert (I_shared = 0), H and I multiples of 32;
+ * otherwise MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG.
  * Every error is returned before anything is enqueued.  Outputs and errors
  * otherwise as moe_forward.
  */
