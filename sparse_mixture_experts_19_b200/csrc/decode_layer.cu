@@ -218,6 +218,34 @@ __device__ __forceinline__ void row_dots(const uint4* const (&rows)[NR], int K8,
         for (int n = 0; n < NV; ++n) d[r][n] = warp_sum(acc[r][n].x + acc[r][n].y);
 }
 
+// d[r] = row_r . v for NR weight rows (streamed with policy pol) and one
+// vector v read from L2 alongside them (a group with one vector: the loads
+// of both are in flight together, and nothing is staged).
+template <int NR>
+__device__ __forceinline__ void row_dots_l2(const uint4* const (&rows)[NR], int K8, const uint4* v, uint64_t pol,
+                                            float (&d)[NR][kDlBatch]) {
+    const int lane = threadIdx.x & 31;
+    float2 acc[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) acc[r] = make_float2(0.f, 0.f);
+    for (int c0 = lane; c0 < K8; c0 += 32 * kDlUnroll) {
+        uint4 w[NR][kDlUnroll], x[kDlUnroll];
+#pragma unroll
+        for (int u = 0; u < kDlUnroll; ++u) {
+            const bool in = c0 + 32 * u < K8;
+            x[u] = in ? __ldcg(v + c0 + 32 * u) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) w[r][u] = in ? ld_stream(rows[r] + c0 + 32 * u, pol) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kDlUnroll; ++u)
+#pragma unroll
+            for (int r = 0; r < NR; ++r) dot8(w[r][u], x[u], acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < NR; ++r) d[r][0] = warp_sum(acc[r].x + acc[r].y);
+}
+
 template <int NR>
 __device__ __forceinline__ void row_dots_n(const uint4* const (&rows)[NR], int K8, const uint32_t (&vec)[kDlBatch],
                                            int nv, uint64_t pol, float (&d)[NR][kDlBatch]) {
@@ -650,6 +678,10 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
     // vectors, and twice the loads are in flight per pass.
     constexpr int kCols = 2;
     const int cp = (cols + kCols - 1) / kCols;
+    // bf16 groups of one vector read it from L2 in the dot products; the
+    // others (and MXFP4, whose vectors are rescaled to f16) are staged in
+    // shared memory first
+    auto h_direct = [&](int g) { return !kMx && pl.gcnt[g] == 1; };
     auto down_items = [&](int g, int first, int step) {
         const bool sh = pl.gexp[g] == a.E;
         const int R = sh ? a.Is : a.I;
@@ -674,6 +706,10 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
                 float d[kCols][kDlBatch];
                 if (kMx)
                     row_dots_mx_n<kCols>(rows, scl, R / 32, vec, nv, pol_dn, d);
+                else if (h_direct(g))  // the group's one h vector, read from L2
+                    row_dots_l2<kCols>(rows, R / 8,
+                                       reinterpret_cast<const uint4*>((sh ? a.hs : a.h) + (int64_t)pl.gvec[g][0] * R),
+                                       pol_dn, d);
                 else
                     row_dots_n<kCols>(rows, R / 8, vec, nv, pol_dn, d);
 #pragma unroll
@@ -815,7 +851,7 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
             }
             named_sync(1, kDn);  // also: every down warp is done with group g-1's h
             if (!down_ok) break;
-            for (int n = 0; n < pl.gcnt[g]; ++n) {
+            for (int n = 0; n < (h_direct(g) ? 0 : pl.gcnt[g]); ++n) {
                 const int id = pl.gvec[g][n];
                 const bf16* hrow = sh ? a.hs + (int64_t)id * R : a.h + (int64_t)id * R;
                 uint8_t* dst = dsm + xbytes + n * R * 2;
@@ -830,7 +866,7 @@ __global__ void __launch_bounds__(kDlThreads, 1) decode_layer_kernel(const DlArg
                     for (int i = dt; i < R / 8; i += kDn) d4[i] = __ldcg(src + i);
                 }
             }
-            named_sync(1, kDn);
+            if (!h_direct(g)) named_sync(1, kDn);
             if (g + 1 < ng) {
                 down_items(g, dw, kDlDownWarps);
             } else {
