@@ -31,6 +31,8 @@ CASES = [
     mi.GPTOSS.with_(name="gpt_oss_mxfp4_T64", T=64),
     mi.Workload("mxfp4_tile_ragged", T=45, H=352, I=160, E=24, k=4),  # 180 slots, ragged tiles
     mi.Workload("mxfp4_tile_cap", T=40, H=256, I=128, E=8, k=2, capacity_factor=0.75),
+    # H = I = 3072: 96 scale bytes per row, the MXFP4 GEMMs' limit
+    mi.Workload("mxfp4_tile_kmax", T=40, H=3072, I=3072, E=4, k=2),
     # I / 32 above the MXFP4 GEMMs' 96 scale bytes per row: dequantized to bf16 first
     mi.Workload("mxfp4_dequant_path", T=40, H=256, I=3104, E=4, k=1),
     # more than 128 rows per expert: dequantized to bf16 first
